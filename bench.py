@@ -1,0 +1,488 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant codec on B200.
+
+Step (timed unit): encode then decode the K and V tensors of one Llama-style
+KV-cache layer [8, 8192, 8, 128] fp16 at 2, 3 and 4 bits -- 12 kernel launches
+(per width: encode K, encode V, then decode K, decode V, each on a tensor not
+touched by the previous launch; every tensor is 128 MiB, larger than L2).
+
+value = fp16-equivalent bytes of the step (2 * d bytes per vector per encode
+or decode) / device time of the step, aggregated over ranks (weak scaling:
+each rank codes its own layer). The same JSON line carries the fused
+decode-step attention ("attn": 16 query tokens over 32768-position packed
+caches, K 4 bits / V 2 bits) and the streaming append ("append": 256
+sequences x 8 heads per step), each timed in its own loop, the roofline of
+the dominant kernel, the oracle CPU baseline, clocks and an end-to-end figure
+through the public API with host buffers.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+D = 128
+LAYER = (8, 8192, 8, 128)
+BITS = (2, 3, 4)
+ATTN = dict(B=16, Hq=32, Hkv=8, S=32768, d=128, kb=4, vb=2)
+APPEND = dict(n_seq=256, H=8, d=128, bits=4, s_max=1024)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for ln in open(self.path):
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(name)
+            os.remove(self.path)
+        except Exception:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "kv_cache_vector_turboquant_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _profile_traffic(kernel_file: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    has not changed since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for ln in open(path):
+        if ":" in ln:
+            k, v = ln.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != _source_hash(kernel_file):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def _ev(torch):
+    return torch.cuda.Event(enable_timing=True)
+
+
+def _codec_step_setup(K, W, torch, rank):
+    """Buffers and the 12 launches of one step (closures on the current stream)."""
+    k, v = W.llama_layer(device="cuda", k_seed=1 + 100 * rank, v_seed=2 + 100 * rank)
+    n = k.numel() // D
+    xs = {"K": k.reshape(n, D), "V": v.reshape(n, D)}
+    codecs = {b: K.TurboQuant(D, b) for b in BITS}
+    packed = {(b, t): torch.empty(n, codecs[b].packed_bytes, dtype=torch.uint8, device="cuda")
+              for b in BITS for t in "KV"}
+    norms = {(b, t): torch.empty(n, dtype=torch.float32, device="cuda") for b in BITS for t in "KV"}
+    out = torch.empty(n, D, dtype=torch.float16, device="cuda")
+    launches = []  # (kind, bits, fn, algorithmic bytes, fp16-equivalent bytes)
+    for b in BITS:
+        alg = n * (2 * D + codecs[b].packed_bytes + 4)
+        for t in "KV":
+            launches.append(("encode", b, (lambda b=b, t=t: K.tq_encode(codecs[b].ctx, xs[t], n, packed[b, t],
+                                                                         norms[b, t])), alg, 2 * D * n))
+    for b in BITS:
+        alg = n * (2 * D + codecs[b].packed_bytes + 4)
+        for t in "KV":
+            launches.append(("decode", b, (lambda b=b, t=t: K.tq_decode(codecs[b].ctx, packed[b, t], norms[b, t], n,
+                                                                         out)), alg, 2 * D * n))
+    return dict(n=n, xs=xs, codecs=codecs, packed=packed, norms=norms, out=out, launches=launches)
+
+
+def _bench_attention(K, W, torch, steps, warmup):
+    a = ATTN
+    q, k, v = W.decode_step(a["B"], a["Hq"], a["Hkv"], a["S"], a["d"])
+    kc, vc = K.TurboQuant(a["d"], a["kb"]), K.TurboQuant(a["d"], a["vb"])
+    kp, kn = kc.encode(k)
+    vp, vn = vc.encode(v)
+    del k, v
+    pos = torch.full((a["B"],), a["S"], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    wsb = K.tq_attend_workspace_bytes(a["B"], a["Hq"], a["d"], a["S"])
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+
+    def call():
+        K.tq_attend_decode(kc.ctx, vc.ctx, q, a["B"], a["Hq"], a["Hkv"], kp, kn, vp, vn, a["S"], pos, out, ws, wsb)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(_ev(torch), _ev(torch)) for _ in range(steps)]
+    for e0, e1 in evs:
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    t = statistics.mean(ms) / 1e3
+    pk, pv = a["d"] * a["kb"] // 8, a["d"] * a["vb"] // 8
+    alg = a["B"] * a["S"] * a["Hkv"] * (pk + pv + 8) + 2 * 2 * a["B"] * a["Hq"] * a["d"]
+    peak, kind = _peaks()
+    ach = alg / t / 1e9
+    st = K.tq_device_error()
+    return {"workload": "decode_step: q [16,32,128] fp16, K 4-bit / V 2-bit packed caches [16,32768,8,*]",
+            "tokens_per_s": a["B"] / t, "ms_per_step": t * 1e3, "ms_median": statistics.median(ms),
+            "cache_positions_heads_per_s": a["B"] * a["S"] * a["Hkv"] / t,
+            "launches_per_step": 2,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                         "traffic": None, "peak_kind": kind, "algorithmic_bytes": alg},
+            "device_error": list(st)}
+
+
+def _bench_append(K, W, torch, steps_per_run=256):
+    """Streaming append: K and V of 256 sequences x 8 heads, one token per step."""
+    res = {}
+    for d in (64, 128, 256):
+        for b in BITS:
+            c = K.TurboQuant(d, b)
+            P = c.packed_bytes
+            n_seq, H, s_max = APPEND["n_seq"], APPEND["H"], steps_per_run
+            toks = W.append_stream(run=d * 10 + b, steps=steps_per_run, n_seq=n_seq, H=H, d=d)
+            cache = {t: torch.empty(n_seq, s_max, H, P, dtype=torch.uint8, device="cuda") for t in "KV"}
+            cn = {t: torch.empty(n_seq, s_max, H, dtype=torch.float32, device="cuda") for t in "KV"}
+            slots = torch.arange(s_max, dtype=torch.int32, device="cuda")[:, None].expand(s_max, n_seq).contiguous()
+
+            def one(s):
+                for t in "KV":
+                    K.tq_encode_append(c.ctx, toks[s], n_seq, H, cache[t], cn[t], s_max, slots[s])
+
+            for s in range(8):
+                one(s)
+            torch.cuda.synchronize()
+            evs = [(_ev(torch), _ev(torch)) for _ in range(steps_per_run)]
+            for s, (e0, e1) in enumerate(evs):
+                e0.record()
+                one(s)
+                e1.record()
+            torch.cuda.synchronize()
+            ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+            total = sum(ms) / 1e3
+            byts = steps_per_run * 2 * n_seq * H * (2 * d + P + 4)
+            res[f"d{d}_b{b}"] = {"p50_us": ms[len(ms) // 2] * 1e3, "p99_us": ms[int(len(ms) * 0.99) - 1] * 1e3,
+                                 "GBps": byts / total / 1e9}
+            del cache, cn, toks
+    return res
+
+
+def _cpu_baseline(seconds_target=12.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload:
+    encode + decode of sampled K rows of the layer at 4 bits."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    k, _ = W.llama_layer(device="cpu")
+    flat = k.reshape(-1, D)
+    rows = torch.randperm(flat.shape[0], generator=torch.Generator().manual_seed(0))
+    done, t_total, chunk = 0, 0.0, 16384
+    while t_total < seconds_target and done + chunk <= flat.shape[0]:
+        xs = flat[rows[done:done + chunk]].numpy()
+        t0 = time.perf_counter()
+        p, nrm = O.encode(xs, 4, 42)
+        O.decode(p, nrm, 4, 42, D)
+        t_total += time.perf_counter() - t0
+        done += chunk
+    fp16eq = 2 * (2 * D) * done  # encode + decode of `done` vectors
+    return {"value": fp16eq / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} random rows of the layer's K tensor, encode+decode at 4 bits, fp64 numpy "
+                      f"({t_total:.1f} s)"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import kv_cache_vector_turboquant_b200 as K
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    S = _codec_step_setup(K, W, torch, rank)
+    launches = S["launches"]
+    fp16eq_step = sum(L[4] for L in launches)
+
+    def step(evs=None):
+        for i, L in enumerate(launches):
+            if evs is not None:
+                evs[i][0].record()
+            L[2]()
+            if evs is not None:
+                evs[i][1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    err = K.tq_device_error()
+    evs = [[(_ev(torch), _ev(torch)) for _ in launches] for _ in range(args.steps)]
+    t0, t1 = _ev(torch), _ev(torch)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record()
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = tt.item()
+    ms_step = ms / args.steps
+
+    # per-kernel averages inside the timed region
+    per = {}
+    for s in range(args.steps):
+        for i, L in enumerate(launches):
+            per.setdefault((L[0], L[1]), []).append((evs[s][i][0].elapsed_time(evs[s][i][1]), L[3]))
+    peak, peak_kind = _peaks()
+    kernels = {}
+    for (kind, b), vals in per.items():
+        avg = statistics.mean(v[0] for v in vals) / 1e3
+        kernels[f"{kind}_b{b}"] = {"us": avg * 1e6, "GBps": vals[0][1] / avg / 1e9,
+                                   "frac": vals[0][1] / avg / 1e9 / peak, "share": sum(v[0] for v in vals)}
+    tot = sum(v["share"] for v in kernels.values())
+    for v in kernels.values():
+        v["share"] = v["share"] / tot
+    dom_name = max(kernels, key=lambda n: kernels[n]["share"])
+    dom = kernels[dom_name]
+    src = "tq_encode.cu" if dom_name.startswith("encode") else "tq_decode.cu"
+    traffic = _profile_traffic(src, f"{dom_name.split('_')[0]}_llama_layer_{dom_name.split('_')[1]}.txt")
+    roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom["GBps"], "peak": peak, "unit": "GB/s",
+            "frac": dom["frac"], "traffic": traffic, "peak_kind": f"{peak_kind} copy (MEASURED_PEAKS.json hbm_gbs)",
+            "algorithmic_bytes_per_launch": per[tuple([dom_name.split('_')[0], int(dom_name[-1])])][0][1]}
+
+    result = {
+        "metric": "encode/decode GB/s (fp16-equivalent) & % of HBM roofline; fused attn tokens/s",
+        "value": fp16eq_step * args.steps * world / (ms / 1e3) / 1e9,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "llama_layer: K and V fp16 [8,8192,8,128] (K with 4 x10 channels per head), "
+                               "encode+decode at bits 2,3,4", "head_dim": D, "vectors_per_tensor": S["n"],
+                   "l2": "inputs larger than L2 (128 MiB per tensor; no launch re-reads what the previous wrote)",
+                   "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
+        "roofline": roof,
+        "kernels": kernels,
+        "clocks": clk.summary(),
+        "gpu_launches": len(launches) * args.steps,
+        "device_error_after_warmup": list(err),
+    }
+    # end to end through the public API with pinned host buffers
+    result["e2e"] = _e2e(K, torch, S, max(2, min(args.steps, 3)), world, dist)
+    if not args.skip_extras:
+        result["attn"] = _bench_attention(K, W, torch, max(args.steps, 5), max(args.warmup, 3))
+        result["append"] = _bench_append(K, W, torch)
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        result["cpu_baseline"] = _cpu_baseline()
+    return result
+
+
+def _e2e(K, torch, S, steps, world, dist):
+    n = S["n"]
+    host_x = {t: S["xs"][t].cpu().pin_memory() for t in "KV"}
+    host_p = {k: v.cpu().pin_memory() for k, v in S["packed"].items()}
+    host_n = {k: v.cpu().pin_memory() for k, v in S["norms"].items()}
+    host_o = torch.empty(n, D, dtype=torch.float16).pin_memory()
+    dx = torch.empty(n, D, dtype=torch.float16, device="cuda")
+    dp = {b: torch.empty(n, S["codecs"][b].packed_bytes, dtype=torch.uint8, device="cuda") for b in BITS}
+    dn = torch.empty(n, dtype=torch.float32, device="cuda")
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        for b in BITS:
+            c = S["codecs"][b].ctx
+            for t in "KV":  # encode: x host -> device, codes back to the host
+                dx.copy_(host_x[t], non_blocking=True)
+                K.tq_encode(c, dx, n, dp[b], dn)
+                host_p[b, t].copy_(dp[b], non_blocking=True)
+                host_n[b, t].copy_(dn, non_blocking=True)
+            for t in "KV":  # decode: codes host -> device, fp16 rows back to the host
+                dp[b].copy_(host_p[b, t], non_blocking=True)
+                dn.copy_(host_n[b, t], non_blocking=True)
+                K.tq_decode(c, dp[b], dn, n, dx)
+                host_o.copy_(dx, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    e0, e1 = _ev(torch), _ev(torch)
+    if world > 1:
+        dist.barrier()
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = tt.item()
+    for b in BITS:
+        P = S["codecs"][b].packed_bytes
+        h2d += 2 * (n * 2 * D) + 2 * (n * P + n * 4)
+        d2h += 2 * (n * P + n * 4) + 2 * (n * 2 * D)
+    fp16eq = 12 * 2 * D * n
+    return {"value": fp16eq * steps * world / (ms / 1e3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "note": "tq_encode/tq_decode with inputs copied from pinned host memory and results copied back, "
+                    "one stream"}
+
+
+def run_reference(args):
+    """The fp64 oracle on the host cores, as it stands, on a bounded sample."""
+    base = _cpu_baseline(seconds_target=max(2.0, 20.0 / max(1, args.steps + args.warmup)))
+    # each step: encode + decode of a fixed 16384-row sample at 4 bits
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    k, _ = W.llama_layer(device="cpu")
+    xs = k.reshape(-1, D)[torch.randperm(k.numel() // D, generator=torch.Generator().manual_seed(1))[:16384]].numpy()
+    for _ in range(args.warmup):
+        O.decode(*O.encode(xs, 4, 42), 4, 42, D)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.decode(*O.encode(xs, 4, 42), 4, 42, D)
+    dt = time.perf_counter() - t0
+    val = 2 * 2 * D * len(xs) * args.steps / dt / 1e9
+    base["value"] = val
+    base["sample"] = f"16384 random rows of the layer's K tensor per step, encode+decode at 4 bits, fp64 numpy"
+    return {"impl": "reference", "metric": "encode/decode GB/s (fp16-equivalent) & % of HBM roofline; "
+                                           "fused attn tokens/s",
+            "value": val, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama_layer: K fp16 [8,8192,8,128], 16384 sampled rows per step, "
+                                   "encode+decode at 4 bits"},
+            "cpu_baseline": base, "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-extras", action="store_true", help="skip the attention and append loops")
+    ap.add_argument("--skip-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        from datetime import timedelta
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

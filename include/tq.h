@@ -1,0 +1,192 @@
+/*
+ * tq.h -- TurboQuant KV-cache codec for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The codec follows the "aither-kvcache" project page (pypi.org), section
+ * "Algorithm": each key or value vector of length head_dim is reduced to a
+ * float32 L2 norm and a unit direction; the direction is rotated by a fixed,
+ * data-oblivious random orthogonal map (here: a seeded +-1 sign flip followed
+ * by the orthonormal Walsh-Hadamard transform, as in the "TurboQuant efficient
+ * inference" post, section "What TurboQuant is"), each rotated coordinate is
+ * scaled by sqrt(head_dim) and rounded to the nearest level of the Lloyd-Max
+ * codebook for N(0,1) with 2^bits levels, and the indices are packed into a
+ * little-endian bitstream. Decoding reverses every step. The fused decode-step
+ * attention follows the same page, section "Zero-buffer fused attention":
+ * rotate the query once, score and accumulate in the rotated domain, rotate
+ * the output back once.
+ *
+ * Conventions for every call below:
+ *  - Ownership: the caller allocates and frees all device memory. The library
+ *    never allocates device memory and never frees caller memory. A context
+ *    (tq_ctx) is a small host object; it is immutable after tq_create and may
+ *    be shared by threads.
+ *  - Execution: device work is enqueued asynchronously on `stream` (a
+ *    cudaStream_t; NULL = the legacy default stream) of the current device.
+ *    Argument validation happens on the host before anything is enqueued; on
+ *    any error nothing is enqueued.
+ *  - Layout: fp16 data is IEEE binary16 stored as uint16; every tensor is
+ *    dense row-major; leading dimensions are flattened, so any [..., d] tensor
+ *    is `n` rows.
+ *  - Alignment: device pointers to fp16 rows and packed rows must be 16-byte
+ *    aligned; float pointers 4-byte aligned; int32 pointers 4-byte aligned.
+ *  - NaN or Inf input gives unspecified codes (never an out-of-bounds access).
+ *  - Device-side faults found by a kernel (a wait that ran out, an index out
+ *    of range) are recorded in a device error word; read it with
+ *    tq_device_error().
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_ctx tq_ctx;
+typedef void* tq_stream; /* cudaStream_t */
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1, /* bad size, null pointer, hq % hkv != 0 ... */
+  TQ_ERR_UNSUPPORTED = 2, /* head_dim not in {64,128,256} or bits not in {2,3,4} */
+  TQ_ERR_ALIGNMENT = 3,   /* a pointer violates the alignment rule above */
+  TQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+  TQ_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  TQ_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out */
+  TQ_ERR_NOMEM = 7,       /* host allocation failed */
+  TQ_ERR_DEVICE = 8       /* a kernel recorded an out-of-range index */
+} tq_status;
+
+/* Bits of the device error word (tq_device_error). */
+#define TQ_DEVERR_TIMEOUT 0x1u     /* an mbarrier wait ran out; the kernel returned early */
+#define TQ_DEVERR_SLOT_RANGE 0x2u  /* tq_encode_append: a slot outside [0, s_max) was skipped */
+#define TQ_DEVERR_POS_RANGE 0x4u   /* tq_attend_decode: a position > s_max was clamped */
+
+/* Human-readable name of a status. Never NULL. */
+const char* tq_status_string(tq_status s);
+
+/*
+ * Create a codec context ("aither-kvcache", section "API Reference":
+ * TurboQuant(head_dim, bits, seed=42)).
+ *   head_dim: 64, 128 or 256.   bits: 2, 3 or 4.
+ *   seed: seed of the splitmix64 stream whose i-th output (bit 63) gives the
+ *         sign of coordinate i.
+ * Builds, on the host only, the Lloyd-Max codebook for N(0,1) (fp64 Lloyd
+ * iteration, then levels rounded to the 2^-14 grid; boundaries are midpoints
+ * of the rounded levels) and the sign table. Touches no GPU.
+ * Returns TQ_ERR_UNSUPPORTED, TQ_ERR_INVALID_ARG (out == NULL) or
+ * TQ_ERR_NOMEM; *out is set only on TQ_OK.
+ */
+tq_status tq_create(int head_dim, int bits, uint64_t seed, tq_ctx** out);
+
+/* Free a context. NULL is ignored. The caller must not use it afterwards. */
+void tq_destroy(tq_ctx* ctx);
+
+/* Parameters of a context (for serialisation: a packed cache is decodable by
+ * any context created with the same three values). 0 for NULL. */
+int tq_head_dim(const tq_ctx* ctx);
+int tq_bits(const tq_ctx* ctx);
+uint64_t tq_seed(const tq_ctx* ctx);
+
+/* Packed bytes per vector, head_dim * bits / 8 ("aither-kvcache", "Quick
+ * Start -- TurboQuant": 128 fp16 -> 64 uint8 at 4 bits). 0 for NULL. */
+size_t tq_packed_bytes(const tq_ctx* ctx);
+
+/*
+ * Copy the context's tables to host memory (any of the pointers may be NULL):
+ *   levels[2^bits]      ascending float32 codebook levels (N(0,1) units),
+ *   boundaries[2^bits-1] float32 decision boundaries,
+ *   sign_bits[head_dim/8] bit i set <=> sign of coordinate i is -1
+ *                        (bit i%8 of byte i/8).
+ * Host only. TQ_ERR_INVALID_ARG for a NULL context.
+ */
+tq_status tq_get_tables(const tq_ctx* ctx, float* levels, float* boundaries, uint8_t* sign_bits);
+
+/*
+ * Encode n vectors ("aither-kvcache", section "Algorithm", steps 1-5).
+ *   x_f16   device, [n, head_dim] fp16, 16-byte aligned.
+ *   packed  device, [n, tq_packed_bytes] uint8 out, 16-byte aligned;
+ *           code i of a row occupies stream bits [i*bits, i*bits+bits),
+ *           stream bit k = bit (k mod 8) of byte k/8.
+ *   norms   device, [n] float32 out: the L2 norm of each input row.
+ * n == 0 is a no-op (pointers may then be NULL). Inputs and outputs must not
+ * overlap. The call is asynchronous on `stream`.
+ */
+tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms,
+                    tq_stream stream);
+
+/*
+ * Decode n vectors ("aither-kvcache", section "Algorithm": decoding reverses
+ * steps 4-1): x_hat = norm * D H (c[idx] / sqrt(head_dim)), rounded to fp16.
+ *   packed  device, [n, tq_packed_bytes] uint8, 16-byte aligned.
+ *   norms   device, [n] float32.
+ *   x_f16   device, [n, head_dim] fp16 out, 16-byte aligned.
+ * n == 0 is a no-op. Asynchronous on `stream`.
+ */
+tq_status tq_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
+                    tq_stream stream);
+
+/*
+ * Streaming append ("aither-kvcache", section "Custom inference loop": encode
+ * where the cache is written): encode one new token per sequence into a
+ * preallocated packed cache.
+ *   x_f16        device, [n_seq, h, head_dim] fp16, 16-byte aligned.
+ *   cache_packed device, [n_seq, s_max, h, tq_packed_bytes] uint8, 16-byte aligned.
+ *   cache_norms  device, [n_seq, s_max, h] float32.
+ *   slot         device, [n_seq] int32: the cache position written for each
+ *                sequence. A slot outside [0, s_max) is skipped and flagged
+ *                with TQ_DEVERR_SLOT_RANGE.
+ * The codes written are bit-identical to tq_encode of the same rows.
+ */
+tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int h, void* cache_packed,
+                           float* cache_norms, int64_t s_max, const int32_t* slot, tq_stream stream);
+
+/*
+ * Workspace (device bytes) that tq_attend_decode needs for a batch of B
+ * sequences, hq query heads, head_dim and caches of s_max positions: the
+ * split-S partial results (running max, sum and rotated accumulator per
+ * split). 0 for invalid sizes.
+ */
+size_t tq_attend_workspace_bytes(int B, int hq, int head_dim, int64_t s_max);
+
+/*
+ * One decode step of attention over packed K/V caches, without decoding them
+ * ("aither-kvcache", section "Zero-buffer fused attention"; "TurboQuant
+ * efficient inference", section "2. A fused decode path"):
+ *   o[b,h] = sum_t softmax_t(q[b,h] . k_hat[b,t,g(h)] / sqrt(d)) v_hat[b,t,g(h)]
+ * over t < positions[b], where g(h) = h / (hq / hkv) and k_hat, v_hat are the
+ * decoded cache rows. Computed as q~ = H D_K q once per head, scores
+ * (n_t / d) (1/sqrt(d)) q~ . c_K[idx_t], an accumulator of n_t c_V[idx_t] in
+ * the rotated domain, and o = D_V H acc / d at the end.
+ *   k, v        contexts of the key and value caches (same head_dim).
+ *   q_f16       device, [B, hq, d] fp16, 16-byte aligned.
+ *   k_packed    device, [B, s_max, hkv, Pk] uint8, 16-byte aligned.
+ *   k_norms     device, [B, s_max, hkv] float32.  (v likewise, Pv bytes)
+ *   positions   device, [B] int32: number of valid cache positions per
+ *               sequence. <= 0 gives a zero output row; > s_max is clamped
+ *               and flagged with TQ_DEVERR_POS_RANGE.
+ *   out_f16     device, [B, hq, d] fp16 out, 16-byte aligned.
+ *   workspace   device scratch of at least
+ *               tq_attend_workspace_bytes(B, hq, d, s_max) bytes, 16-byte
+ *               aligned; its contents on entry do not matter.
+ * Asynchronous on `stream`; calls that share a workspace must not overlap.
+ */
+tq_status tq_attend_decode(const tq_ctx* k, const tq_ctx* v, const void* q_f16, int B, int hq, int hkv,
+                           const void* k_packed, const float* k_norms, const void* v_packed,
+                           const float* v_norms, int64_t s_max, const int32_t* positions, void* out_f16,
+                           void* workspace, size_t ws_bytes, tq_stream stream);
+
+/*
+ * Read and clear the device error word of the current device (a bitwise OR
+ * of TQ_DEVERR_* set by kernels since the last call). Synchronises `stream`.
+ * Returns TQ_ERR_TIMEOUT if TQ_DEVERR_TIMEOUT was set, TQ_ERR_DEVICE if
+ * another bit was set, else TQ_OK; *bits (optional) receives the word.
+ */
+tq_status tq_device_error(tq_stream stream, uint32_t* bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

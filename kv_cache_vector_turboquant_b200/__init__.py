@@ -1,0 +1,116 @@
+"""TurboQuant KV-cache codec for NVIDIA B200 (sm_100a).
+
+The compute path is the CUDA library ``libtq.so`` behind the C ABI of
+``include/tq.h``; this package is its ctypes binding plus a small convenience
+layer with the call shapes of the "aither-kvcache" page ("Quick Start --
+TurboQuant", "API Reference": ``TurboQuant(head_dim, bits, seed=42)``,
+``encode(x) -> (packed, norms)``, ``decode(packed, norms)``,
+``compression_ratio()``). PyTorch supplies device memory and streams only.
+"""
+
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    LIB_PATH,
+    TQ_DEVERR_POS_RANGE,
+    TQ_DEVERR_SLOT_RANGE,
+    TQ_DEVERR_TIMEOUT,
+    TQ_ERR_ALIGNMENT,
+    TQ_ERR_CUDA,
+    TQ_ERR_DEVICE,
+    TQ_ERR_INVALID_ARG,
+    TQ_ERR_NOMEM,
+    TQ_ERR_TIMEOUT,
+    TQ_ERR_UNSUPPORTED,
+    TQ_ERR_WORKSPACE,
+    TQ_OK,
+    Ctx,
+    TQError,
+    tq_attend_decode,
+    tq_attend_workspace_bytes,
+    tq_create,
+    tq_decode,
+    tq_device_error,
+    tq_encode,
+    tq_encode_append,
+    tq_get_tables,
+    tq_status_string,
+)
+
+
+def _require(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+class TurboQuant:
+    """One codec (head_dim, bits, seed) on the current CUDA device."""
+
+    def __init__(self, head_dim: int = 128, bits: int = 4, seed: int = 42):
+        self.ctx = tq_create(head_dim, bits, seed)
+        self.head_dim, self.bits, self.seed = head_dim, bits, seed
+        self.packed_bytes = self.ctx.packed_bytes
+
+    def compression_ratio(self) -> float:
+        """fp16 bytes over stored bytes (packed codes + f32 norm) per vector."""
+        return 2.0 * self.head_dim / (self.packed_bytes + 4)
+
+    def encode(self, x, out=None, stream=None):
+        """[..., d] fp16 CUDA tensor -> ([..., d*b/8] uint8, [...] float32)."""
+        import torch
+
+        _require(x.is_cuda and x.dtype == torch.float16 and x.is_contiguous(), "x: contiguous fp16 CUDA tensor")
+        _require(x.shape[-1] == self.head_dim, "last dim must be head_dim")
+        lead = tuple(x.shape[:-1])
+        n = x.numel() // self.head_dim
+        if out is None:
+            packed = torch.empty(lead + (self.packed_bytes,), dtype=torch.uint8, device=x.device)
+            norms = torch.empty(lead, dtype=torch.float32, device=x.device)
+        else:
+            packed, norms = out
+        tq_encode(self.ctx, x, n, packed, norms, stream)
+        return packed, norms
+
+    def decode(self, packed, norms, out=None, stream=None):
+        """([..., d*b/8] uint8, [...] float32) -> [..., d] fp16."""
+        import torch
+
+        _require(packed.is_cuda and packed.dtype == torch.uint8 and packed.is_contiguous(), "packed: uint8 CUDA")
+        _require(packed.shape[-1] == self.packed_bytes, "last dim of packed must be head_dim*bits/8")
+        _require(norms.dtype == torch.float32 and norms.is_contiguous(), "norms: contiguous float32")
+        lead = tuple(packed.shape[:-1])
+        n = packed.numel() // self.packed_bytes
+        _require(norms.numel() == n, "norms must have one entry per vector")
+        x = out if out is not None else torch.empty(lead + (self.head_dim,), dtype=torch.float16,
+                                                    device=packed.device)
+        tq_decode(self.ctx, packed, norms, n, x, stream)
+        return x
+
+    def encode_append(self, x, cache_packed, cache_norms, slot, stream=None):
+        """Write one token per sequence: x [n_seq, h, d] into cache slot[s]."""
+        n_seq, h, d = x.shape
+        _require(d == self.head_dim, "last dim must be head_dim")
+        s_max = cache_packed.shape[1]
+        tq_encode_append(self.ctx, x, n_seq, h, cache_packed, cache_norms, s_max, slot, stream)
+
+
+def attend_decode(q, k_codec: TurboQuant, v_codec: TurboQuant, k_packed, k_norms, v_packed, v_norms,
+                  positions, out=None, workspace=None, stream=None):
+    """One decode step of attention over packed caches.
+
+    q [B, Hq, d] fp16; k_packed [B, S, Hkv, Pk] uint8; k_norms [B, S, Hkv] f32;
+    v likewise; positions [B] int32 (valid cache length per sequence).
+    Returns o [B, Hq, d] fp16.
+    """
+    import torch
+
+    B, hq, d = q.shape
+    s_max, hkv = k_packed.shape[1], k_packed.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = tq_attend_workspace_bytes(B, hq, d, s_max)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    tq_attend_decode(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_packed, k_norms, v_packed, v_norms, s_max,
+                     positions, out, workspace, workspace.numel(), stream)
+    return out

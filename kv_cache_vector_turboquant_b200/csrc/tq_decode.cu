@@ -1,0 +1,286 @@
+// Decode kernel: (packed codes, f32 norms) -> fp16 vectors.
+//
+// Method ("aither-kvcache" PyPI page, section "Algorithm": decoding reverses
+// steps 4-1): unpack the indices, look up the levels c[idx], undo the scaled
+// rotation and multiply by the norm:
+//   x_hat = N * D H (c[idx] / sqrt(d)) = D (H_pm c[idx]) * (N / d),
+// H_pm the unnormalised +-1 Walsh-Hadamard matrix. The levels lie on the
+// 2^-14 grid and |H_pm c| < 2^10, so H_pm c is exact in f32 in any order; the
+// only roundings are the product by N/d (a power-of-two scaling of N, exact)
+// in f32 and the final fp16 conversion.
+//
+// B200 mapping: one vector per lane (two lanes for d = 256). Each warp runs a
+// 3-stage pipeline of 1-D bulk copies (TMA) bringing its tile of packed rows
+// and norms into shared memory; a lane-replicated table indexed by two codes
+// returns (c[a] + c[b], c[a] - c[b]), i.e. the levels already through the
+// first butterfly; the other stages run in registers with f32x2 add/sub; the
+// fp16 rows are staged in padded shared rows and leave through per-row 1-D
+// bulk stores (TMA), so every DRAM write is a full line.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+constexpr int DEC_WARPS = 8;
+constexpr int DEC_STAGES = 3;
+
+template <int D, int BITS>
+struct DecCfg {
+  static constexpr int LPV = D > 128 ? 2 : 1;
+  static constexpr int C = D / LPV;
+  static constexpr int NP = C / 2;
+  static constexpr int VPW = 32 / LPV;
+  static constexpr int P = D * BITS / 8;
+  static constexpr int PL = P / LPV;       // packed bytes per lane
+  static constexpr int WL = PL / 4;        // packed words per lane
+  static constexpr int E = 1 << (2 * BITS);  // pair-table entries
+  static constexpr int TILE_P = VPW * P;   // packed bytes per full tile
+  static constexpr int IN_STAGE = ((TILE_P + 15) / 16) * 16 + 32 * 4;  // packed + norms
+  static constexpr int OUT_ROW = 2 * C + 16;  // padded fp16 lane-row
+  static constexpr int OUT = 32 * OUT_ROW;
+};
+
+template <int D, int BITS>
+struct DecSmem {
+  using Cfg = DecCfg<D, BITS>;
+  static constexpr int BAR = 0;
+  static constexpr int IN = 256;
+  static constexpr int OUT = IN + DEC_WARPS * DEC_STAGES * Cfg::IN_STAGE;
+  static constexpr int LUT = OUT + DEC_WARPS * Cfg::OUT;
+  static constexpr size_t BYTES = (size_t)LUT + (size_t)Cfg::E * 32 * 8;
+};
+
+struct DecArgs {
+  const uint8_t* packed;
+  const float* norms;
+  int64_t n;
+  __half* x;
+  uint32_t* err;
+  long long wait_limit;
+  int norms_bulk;  // norms pointer 16-byte aligned: norms tiles come by bulk copy
+};
+
+TQ_DEV f2 lds_f2(uint32_t addr) {
+  f2 r;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(r.x), "=f"(r.y) : "r"(addr));
+  return r;
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(DEC_WARPS * 32, 1)
+    decode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ DecArgs a) {
+  using Cfg = DecCfg<D, BITS>;
+  using Sm = DecSmem<D, BITS>;
+  constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, VPW = Cfg::VPW, WL = Cfg::WL;
+  constexpr int P = Cfg::P, E = Cfg::E;
+  constexpr uint32_t FULL = 0xffffffffu;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // pair table: entry (f, lane) with f = code_a | code_b << BITS holds
+  // (c[a] + c[b], c[a] - c[b]) -- exact in f32 (2^-14 grid).
+  {
+    f2* lut = reinterpret_cast<f2*>(smem + Sm::LUT);
+    for (int e = threadIdx.x; e < E * 32; e += blockDim.x) {
+      const int f = e >> 5;
+      const float ca = T.levels[f & ((1 << BITS) - 1)];
+      const float cb = T.levels[f >> BITS];
+      lut[e] = f2{ca + cb, ca - cb};
+    }
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::BAR) + warp * DEC_STAGES;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < DEC_STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  uint8_t* in0 = smem + Sm::IN + warp * DEC_STAGES * Cfg::IN_STAGE;
+  uint8_t* out_rows = smem + Sm::OUT + warp * Cfg::OUT;
+  const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
+
+  const int64_t n_tiles = (a.n + VPW - 1) / VPW;
+  const int64_t gw = (int64_t)blockIdx.x * DEC_WARPS + warp;
+  const int64_t n_warps = (int64_t)gridDim.x * DEC_WARPS;
+  constexpr int NORM_OFF = ((Cfg::TILE_P + 15) / 16) * 16;
+
+  // Full tiles come through bulk copies; the last, partial tile (if any) is
+  // read with plain loads (its byte count need not be a multiple of 16).
+  auto full_tile = [&](int64_t tile) { return (tile + 1) * VPW <= a.n; };
+  auto issue = [&](int64_t tile, int stage) {
+    if (!full_tile(tile)) return;
+    if (lane == 0) {
+      const uint32_t bar = smem_u32(&bars[stage]);
+      mbar_arrive_expect_tx(bar, (uint32_t)(Cfg::TILE_P + (a.norms_bulk ? VPW * 4 : 0)));
+      uint8_t* dst = in0 + stage * Cfg::IN_STAGE;
+      bulk_g2s(smem_u32(dst), a.packed + tile * Cfg::TILE_P, Cfg::TILE_P, bar);
+      if (a.norms_bulk) bulk_g2s(smem_u32(dst + NORM_OFF), a.norms + tile * VPW, VPW * 4, bar);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < DEC_STAGES; ++s) {
+    const int64_t t = gw + s * n_warps;
+    if (t < n_tiles) issue(t, s);
+  }
+
+  const int half = lane & (LPV - 1);
+  int stage = 0;
+  uint32_t parity = 0;
+  bool stored_once = false;
+  for (int64_t tile = gw; tile < n_tiles; tile += n_warps) {
+    const int64_t v0 = tile * VPW;
+    const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
+    const bool active = lane < valid_lanes;
+    const int vl = lane / LPV;  // vector within the tile
+    uint32_t words[WL];
+    float nrm = 0.f;
+    if (full_tile(tile)) {
+      // every lane polls; the warp acts on one agreed outcome
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u,
+                                                             a.wait_limit));
+    if (!ok) {
+        if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+#pragma unroll
+        for (int s = 1; s < DEC_STAGES; ++s) {
+          const int os = (stage + s) % DEC_STAGES;
+          if (tile + s * n_warps < n_tiles && full_tile(tile + s * n_warps))
+            (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
+        }
+        bulk_wait_all<0>();
+        return;
+      }
+      parity ^= 1u << stage;
+      const uint8_t* st = in0 + stage * Cfg::IN_STAGE;
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(st + vl * P + half * Cfg::PL);
+#pragma unroll
+      for (int w = 0; w < WL; ++w) words[w] = row[w];
+      nrm = a.norms_bulk ? reinterpret_cast<const float*>(st + NORM_OFF)[vl] : __ldg(a.norms + v0 + vl);
+    } else {
+#pragma unroll
+      for (int w = 0; w < WL; ++w) words[w] = 0;
+      if (active) {
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(a.packed + (v0 + vl) * P + half * Cfg::PL);
+#pragma unroll
+        for (int w = 0; w < WL; ++w) words[w] = __ldg(row + w);
+        nrm = __ldg(a.norms + v0 + vl);
+      }
+    }
+    __syncwarp();
+    // the stage has been read into registers: refill it
+    {
+      const int64_t next = tile + DEC_STAGES * n_warps;
+      if (next < n_tiles) issue(next, stage);
+    }
+
+    // ---- unpack pairs of codes -> levels through the first butterfly
+    f2 v[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      constexpr int FB = 2 * BITS;
+      const int off = j * FB;
+      uint32_t f = words[off >> 5] >> (off & 31);
+      if ((off & 31) + FB > 32) f |= words[(off >> 5) + 1] << (32 - (off & 31));
+      f &= (uint32_t)(E - 1);
+      v[j] = lds_f2(f * 256u + lut_lane);
+    }
+    wht_pairs<NP>(v);
+    if (LPV == 2) {
+      const f2 sg = half ? f2{-1.f, -1.f} : f2{1.f, 1.f};
+#pragma unroll
+      for (int k = 0; k < NP; ++k) {
+        f2 o;
+        o.x = __shfl_xor_sync(FULL, v[k].x, 1);
+        o.y = __shfl_xor_sync(FULL, v[k].y, 1);
+        v[k] = fma2(v[k], sg, o);
+      }
+    }
+
+    // ---- scale by N/d, round to fp16, apply the signs, stage the row
+    const float sc = nrm * (1.0f / (float)D);
+    const f2 sc2 = {sc, sc};
+    // the previous bulk store from this warp's staging rows must have read them
+    if (stored_once) bulk_wait_read<0>();
+    __syncwarp();
+    uint8_t* orow = out_rows + lane * Cfg::OUT_ROW;
+#pragma unroll
+    for (int c = 0; c < C / 8; ++c) {
+      uint32_t h[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = 4 * c + q;
+        const f2 y = mul2(v[k], sc2);
+        const __half2 hv = __floats2half2_rn(y.x, y.y);
+        uint32_t mask = T.sign_h2[k];
+        if (LPV == 2) mask = half ? T.sign_h2[NP + k] : T.sign_h2[k];
+        h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ mask;
+      }
+      *reinterpret_cast<uint4*>(orow + 16 * c) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (active) {
+      __half* dst = a.x + (v0 + vl) * D + half * C;
+      bulk_s2g(dst, smem_u32(orow), 2 * C);
+      bulk_commit();
+      stored_once = true;
+    }
+    if (++stage == DEC_STAGES) stage = 0;
+  }
+  bulk_wait_all<0>();
+}
+
+template <int D, int BITS>
+static cudaError_t launch_decode_t(const tq_codec_tables& T, const DecArgs& a, cudaStream_t st) {
+  using Cfg = DecCfg<D, BITS>;
+  constexpr size_t smem = DecSmem<D, BITS>::BYTES;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> configured{0};
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(decode_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const int64_t tiles = (a.n + Cfg::VPW - 1) / Cfg::VPW;
+  const int64_t ctas = (tiles + DEC_WARPS - 1) / DEC_WARPS;
+  const int grid = (int)std::min<int64_t>(ctas, (int64_t)tq_sm_count(dev));
+  decode_kernel<D, BITS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
+  return cudaGetLastError();
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
+                           void* stream) {
+  if (n == 0) return TQ_OK;
+  DecArgs a;
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.norms = norms;
+  a.n = n;
+  a.x = static_cast<__half*>(x);
+  a.err = tq_error_word();
+  if (!a.err) return TQ_ERR_CUDA;
+  a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
+  a.norms_bulk = (reinterpret_cast<uintptr_t>(norms) & 15u) == 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+#define TQ_DEC_CASE(D_, B_) \
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_t<D_, B_>(ctx->t, a, st);
+  TQ_DEC_CASE(64, 2) TQ_DEC_CASE(64, 3) TQ_DEC_CASE(64, 4)
+  TQ_DEC_CASE(128, 2) TQ_DEC_CASE(128, 3) TQ_DEC_CASE(128, 4)
+  TQ_DEC_CASE(256, 2) TQ_DEC_CASE(256, 3) TQ_DEC_CASE(256, 4)
+#undef TQ_DEC_CASE
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}

@@ -1,0 +1,65 @@
+// Internal definitions shared by the host code and the CUDA kernels of libtq.
+// Not part of the public ABI (include/tq.h is).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+#define TQ_MAX_D 256
+#define TQ_MAX_L 16
+
+// Codec tables, passed by value in every kernel launch (constant bank), so
+// warp-uniform lookups (sign masks, levels) cost no registers or loads.
+struct tq_codec_tables {
+  // XOR mask for the fp16 pair (2k, 2k+1): bit 15 set <=> coordinate 2k is
+  // negated, bit 31 set <=> coordinate 2k+1 is negated.
+  uint32_t sign_h2[TQ_MAX_D / 2];
+  float levels[TQ_MAX_L];      // format levels c_k (2^-14 grid), ascending
+  float bounds[TQ_MAX_L - 1];  // decision boundaries t_j in z units (2^-15 grid)
+  // Encode quantizer lookup table, in "q units" q = z * inv_delta + q_offset:
+  // cells are the unit intervals [n, n+1); each holds at most one boundary,
+  // at least `margin` away from the cell edges.
+  float tau[TQ_MAX_L - 1];  // boundaries in q units (exact in f32)
+  float q_offset;           // q of z = 0 (an integer + a fraction)
+  float inv_delta;          // 1/delta, a power of two
+  float guard_q;            // half-width of the f64 recheck band, q units
+  int lut_cells;            // number of cells (q in [0, lut_cells))
+  int d;
+  int bits;
+};
+
+struct tq_ctx {
+  int d;
+  int bits;
+  uint64_t seed;
+  double lloyd_max[TQ_MAX_L];  // unrounded fp64 Lloyd-Max levels
+  tq_codec_tables t;
+};
+
+// Guard band of the encode quantizer in z units (N(0,1) scale). The f32 path
+// decides every coordinate whose scaled rotated value is farther than this
+// from a boundary; the f32 rounding error bound is below 1.1e-5 for
+// head_dim <= 256 (see the error analysis in the design notes), so those
+// decisions equal the exact ones. Closer coordinates are redone in fp64.
+#define TQ_GUARD_Z 2.0e-5
+
+// Kernel launchers (defined in the .cu files). Arguments are validated by the
+// ABI layer before these are called.
+tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
+                           const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject);
+tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n,
+                           void* x, void* stream);
+tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
+                           const void* k_packed, const float* k_norms, const void* v_packed,
+                           const float* v_norms, int64_t s_max, const int32_t* positions, void* out,
+                           void* workspace, size_t ws_bytes, void* stream);
+size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max);
+
+// Number of SMs of device `dev` (cached).
+int tq_sm_count(int dev);
+
+// Device error word of the current device (device pointer), and its reader.
+uint32_t* tq_error_word(void);
+tq_status tq_read_error_word(void* stream, uint32_t* bits);

@@ -237,10 +237,10 @@ def unpack_codes(packed: np.ndarray, bits: int, d: int) -> np.ndarray:
     """Inverse of :func:`pack_codes`: [n, d*b/8] uint8 -> [n, d] int64 codes."""
     packed = np.asarray(packed, dtype=np.uint8)
     n = packed.shape[0]
-    stream = ((packed[:, :, None].astype(np.int64) >> np.arange(8)) & 1).reshape(n, -1)
+    stream = ((packed[:, :, None] >> np.arange(8, dtype=np.uint8)) & 1).reshape(n, -1)
     idx = np.zeros((n, d), dtype=np.int64)
     for j in range(bits):
-        idx |= stream[:, j::bits][:, :d] << j
+        idx |= stream[:, j::bits][:, :d].astype(np.int64) << j
     return idx
 
 

@@ -1,0 +1,164 @@
+"""The C ABI without a GPU: exports, context tables, host-side validation.
+
+No call here reaches a kernel launch: every call either touches host memory
+only (tq_create, tq_get_tables) or fails host validation first.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    import kv_cache_vector_turboquant_b200 as K
+
+    return K
+
+
+@pytest.fixture(scope="module")
+def lib(K):
+    return ctypes.CDLL(K.LIB_PATH)
+
+
+def _declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert {"tq_create", "tq_encode", "tq_decode", "tq_encode_append", "tq_attend_decode"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_tables_match_oracle(K, d, bits):
+    ctx = K.tq_create(d, bits, 42)
+    assert (ctx.head_dim, ctx.bits, ctx.seed, ctx.packed_bytes) == (d, bits, 42, d * bits // 8)
+    lv, bd, sb = K.tq_get_tables(ctx)
+    assert np.array_equal(lv, O.format_levels(bits).astype(np.float32))
+    assert np.array_equal(bd, O.format_boundaries(O.format_levels(bits)).astype(np.float32))
+    # the f32 tables are exact copies of the fp64 grid values
+    assert np.array_equal(lv.astype(np.float64), O.format_levels(bits))
+    s = O.sign_vector(42, d)
+    assert np.array_equal(sb, np.packbits((s < 0).astype(np.uint8), bitorder="little"))
+
+
+def test_seed_changes_signs_only(K):
+    a, b = K.tq_create(128, 4, 42), K.tq_create(128, 4, 7)
+    la, _, sa = K.tq_get_tables(a)
+    lb, _, sb = K.tq_get_tables(b)
+    assert np.array_equal(la, lb) and not np.array_equal(sa, sb)
+    s = O.sign_vector(7, 128)
+    assert np.array_equal(sb, np.packbits((s < 0).astype(np.uint8), bitorder="little"))
+
+
+def test_create_rejects_unsupported(K):
+    for d, b in [(32, 4), (96, 4), (512, 4), (128, 1), (128, 5), (0, 4)]:
+        with pytest.raises(K.TQError) as e:
+            K.tq_create(d, b)
+        assert e.value.status == K.TQ_ERR_UNSUPPORTED
+    vp = ctypes.c_void_p
+    assert K._binding._lib.tq_create(128, 4, 42, None) == K.TQ_ERR_INVALID_ARG
+
+
+def test_status_strings(K):
+    for s in range(9):
+        assert K.tq_status_string(s).startswith("TQ_")
+    assert K.tq_status_string(99) == "TQ_ERR_UNKNOWN"
+
+
+def test_null_context_queries(lib):
+    for fn in ("tq_head_dim", "tq_bits", "tq_packed_bytes"):
+        f = getattr(lib, fn)
+        f.argtypes = [ctypes.c_void_p]
+        assert f(None) == 0
+
+
+class _FakePtr:
+    """Stands in for a tensor: only its address is read by the binding."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _raw(K, name, *args):
+    return getattr(K._binding._lib, name)(*args)
+
+
+def test_encode_decode_validation(K):
+    ctx = K.tq_create(128, 4)
+    h = ctx.handle
+    A, B_, C = 0x10000, 0x20000, 0x30000
+    # null context, negative n
+    assert _raw(K, "tq_encode", None, A, 4, B_, C, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode", h, A, -1, B_, C, None) == K.TQ_ERR_INVALID_ARG
+    # n == 0 is a no-op, even with null pointers
+    assert _raw(K, "tq_encode", h, None, 0, None, None, None) == K.TQ_OK
+    assert _raw(K, "tq_decode", h, None, None, 0, None, None) == K.TQ_OK
+    # null pointers
+    assert _raw(K, "tq_encode", h, None, 4, B_, C, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_decode", h, A, None, 4, C, None) == K.TQ_ERR_INVALID_ARG
+    # misaligned pointers
+    assert _raw(K, "tq_encode", h, A + 8, 4, B_, C, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_encode", h, A, 4, B_ + 4, C, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_encode", h, A, 4, B_, C + 2, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_decode", h, A + 1, C, 4, B_, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_decode", h, A, C, 4, B_ + 8, None) == K.TQ_ERR_ALIGNMENT
+
+
+def test_append_validation(K):
+    ctx = K.tq_create(128, 3)
+    h = ctx.handle
+    A, B_, C, S = 0x10000, 0x20000, 0x30000, 0x40000
+    assert _raw(K, "tq_encode_append", h, A, 4, 0, B_, C, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_append", h, A, 4, 8, B_, C, 0, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_append", h, A, -1, 8, B_, C, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_append", h, A, 0, 8, B_, C, 16, S, None) == K.TQ_OK
+    assert _raw(K, "tq_encode_append", h, A, 4, 8, B_, C, 16, None, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_append", h, A, 4, 8, B_, C, 16, S + 2, None) == K.TQ_ERR_ALIGNMENT
+
+
+def test_attend_validation_and_workspace(K):
+    k4, v2 = K.tq_create(128, 4), K.tq_create(128, 2)
+    k64 = K.tq_create(64, 4)
+    ws = K.tq_attend_workspace_bytes(16, 32, 128, 32768)
+    assert ws > 0 and ws % 4 == 0
+    # the workspace holds (max, sum, d accumulators) per (sequence, head, split)
+    assert ws >= 16 * 32 * (128 + 2) * 4
+    assert K.tq_attend_workspace_bytes(0, 32, 128, 10) == 0
+    assert K.tq_attend_workspace_bytes(2, 8, 96, 10) == 0
+    A = 0x100000
+    args = lambda kc, vc, B, hq, hkv, s_max, ws_ptr, ws_b: (  # noqa: E731
+        kc.handle, vc.handle, A, B, hq, hkv, A, A, A, A, s_max, A, A, ws_ptr, ws_b, None)
+    need = K.tq_attend_workspace_bytes(2, 8, 128, 100)
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 2, 8, 3, 100, A, need)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_attend_decode", *args(k4, k64, 2, 8, 2, 100, A, need)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 2, 8, 2, 0, A, need)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 2, 8, 2, 100, A, need - 4)) == K.TQ_ERR_WORKSPACE
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 2, 8, 2, 100, None, need)) == K.TQ_ERR_WORKSPACE
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 2, 8, 2, 100, A + 4, need)) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_attend_decode", *args(k4, v2, 0, 8, 2, 100, A, need)) == K.TQ_OK
+
+
+def test_compression_ratio_matches_formula(K):
+    for b, want in ((2, 256 / 36), (3, 256 / 52), (4, 256 / 68)):
+        assert abs(K.TurboQuant(128, b).compression_ratio() - want) < 1e-12

@@ -1,0 +1,219 @@
+"""CUDA encode / decode / append against the fp64 oracle (needs a B200)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity import assert_decode_ulp, assert_norms, code_mismatches
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K(cuda_device):
+    import kv_cache_vector_turboquant_b200 as K
+
+    return K
+
+
+@pytest.fixture(scope="module")
+def W():
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    return W
+
+
+def _encode(tq, x):
+    packed, norms = tq.encode(x)
+    torch.cuda.synchronize()
+    return packed, norms
+
+
+def _full_parity(K, x16_cpu, d, bits, seed=42, max_boundary_frac=1e-6):
+    """Encode on the GPU, compare codes / norms / decode with the oracle."""
+    tq = K.TurboQuant(d, bits, seed)
+    x = x16_cpu.to("cuda")
+    packed, norms = _encode(tq, x)
+    xn = x16_cpu.numpy()
+    det = O.encode_detail(xn, bits, seed)
+    gp, gn = packed.cpu().numpy(), norms.cpu().numpy()
+    n_mis = code_mismatches(gp, det, bits, d, max_boundary_frac)
+    assert_norms(gn, det)
+    # decode of the GPU's own bytes vs the oracle decode of the same bytes
+    xd = tq.decode(packed, norms)
+    torch.cuda.synchronize()
+    ref = O.decode(gp, gn, bits, seed, d)
+    assert_decode_ulp(xd.cpu().numpy().reshape(ref.shape), ref)
+    st, bits_w = K.tq_device_error()
+    assert st == K.TQ_OK and bits_w == 0
+    return n_mis, gp, det
+
+
+def test_single_tensor_workload(K, W):
+    """4096 x 128 fp16 with 1% outlier vectors, 4 bits, seed 42: every code,
+    norm and decoded value."""
+    x = W.single_tensor()
+    n_mis, gp, det = _full_parity(K, x, 128, 4)
+    assert n_mis == 0
+    assert gp.shape == (4096, 64)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("n", [1, 31, 33, 1000, 4103])
+def test_ragged_sizes(K, W, d, bits, n):
+    x = W.single_tensor(n=n, d=d, seed=1000 + n + d + bits, outlier_frac=0.05)
+    n_mis, _, _ = _full_parity(K, x, d, bits)
+    assert n_mis == 0
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_degenerate_vectors(K, W, d, bits):
+    """Zero, constant, spike, extreme-magnitude and alternating rows. Exact ties
+    at a boundary occur here (e.g. z = 0 exactly), so only the boundary-band
+    rule applies, without the fraction bound."""
+    x = W.edge_vectors(d)
+    _full_parity(K, x, d, bits, max_boundary_frac=None)
+    # the zero vector: norm 0, every code 2^(b-1), decodes to exact zeros
+    tq = K.TurboQuant(d, bits)
+    packed, norms = _encode(tq, x[:1].cuda())
+    idx = O.unpack_codes(packed.cpu().numpy(), bits, d)
+    assert norms.item() == 0.0 and np.all(idx == (1 << bits) // 2)
+    assert torch.all(tq.decode(packed, norms) == 0)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_signed_hadamard_rows_rotate_to_spikes(K, d):
+    """x = D r_k rotates to z = sqrt(d) e_k: code L-1 at k, 2^(b-1) elsewhere
+    (exact ties at z = 0 go up)."""
+    import scipy.linalg
+
+    s = O.sign_vector(42, d)
+    R = scipy.linalg.hadamard(d)
+    rows = np.stack([s * R[k] for k in range(0, d, max(1, d // 16))]).astype(np.float16)
+    for bits in (2, 3, 4):
+        tq = K.TurboQuant(d, bits)
+        packed, norms = _encode(tq, torch.from_numpy(rows).cuda())
+        idx = O.unpack_codes(packed.cpu().numpy(), bits, d)
+        for r, k in enumerate(range(0, d, max(1, d // 16))):
+            want = np.full(d, (1 << bits) // 2)
+            want[k] = (1 << bits) - 1
+            assert np.array_equal(idx[r], want)
+        assert np.allclose(norms.cpu().numpy(), math.sqrt(d), rtol=1e-7)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_llama_layer_full_size_sampled(K, W, bits):
+    """Full [8, 8192, 8, 128] K and V layer on the GPU (the benchmarked
+    launch); 65,536 sampled rows per tensor against the oracle, and the
+    full-size distortion against the sphere-marginal value."""
+    k, v = W.llama_layer(device="cuda")
+    tq = K.TurboQuant(128, bits)
+    g = torch.Generator().manual_seed(77 + bits)
+    for x in (k, v):
+        flat = x.reshape(-1, 128)
+        packed, norms = tq.encode(flat)
+        dec = tq.decode(packed, norms)
+        torch.cuda.synchronize()
+        rows = torch.randperm(flat.shape[0], generator=g)[:65536].sort().values
+        xs = flat[rows.cuda()].cpu().numpy()
+        det = O.encode_detail(xs, bits, 42)
+        gp = packed[rows.cuda()].cpu().numpy()
+        gn = norms[rows.cuda()].cpu().numpy()
+        assert code_mismatches(gp, det, bits, 128) == 0
+        assert_norms(gn, det)
+        assert_decode_ulp(dec[rows.cuda()].cpu().numpy(), O.decode(gp, gn, bits, 42, 128))
+        # whole-tensor property: unit-direction distortion equals the sphere marginal
+        u = flat.float() / flat.float().norm(dim=1, keepdim=True)
+        uh = dec.float() / norms[:, None]
+        mse = ((u - uh) ** 2).sum(dim=1).mean().item()
+        want = O.sphere_marginal_mse(O.format_levels(bits), 128)
+        assert abs(mse - want) / want < 0.01, (mse, want)
+        del packed, norms, dec
+    assert K.tq_device_error()[0] == K.TQ_OK
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_append_matches_bulk_encode(K, W, d, bits):
+    """Streaming append of 6 steps x 256 sequences x 8 heads into a 16-slot
+    cache: written slots are bit-identical to a bulk encode of the same rows,
+    other slots untouched."""
+    n_seq, h, s_max, steps = 256, 8, 16, 6
+    tq = K.TurboQuant(d, bits)
+    P = tq.packed_bytes
+    toks = W.append_stream(run=bits + d, steps=steps, n_seq=n_seq, H=h, d=d)
+    cache = torch.full((n_seq, s_max, h, P), 0xAB, dtype=torch.uint8, device="cuda")
+    cnorm = torch.full((n_seq, s_max, h), -1.0, dtype=torch.float32, device="cuda")
+    slots = torch.randint(0, s_max, (steps, n_seq), generator=torch.Generator().manual_seed(d + bits),
+                          dtype=torch.int32)
+    # distinct slots per sequence across steps so later steps do not overwrite
+    slots = (torch.arange(steps, dtype=torch.int32)[:, None] * 2 + (slots % 2)) % s_max
+    for s in range(steps):
+        tq.encode_append(toks[s].contiguous(), cache, cnorm, slots[s].cuda())
+    torch.cuda.synchronize()
+    bp, bn = tq.encode(toks.reshape(-1, d).contiguous())
+    bp = bp.reshape(steps, n_seq, h, P).cpu()
+    bn = bn.reshape(steps, n_seq, h).cpu()
+    cache, cnorm = cache.cpu(), cnorm.cpu()
+    written = torch.zeros(n_seq, s_max, dtype=torch.bool)
+    for s in range(steps):
+        idx = torch.arange(n_seq)
+        assert torch.equal(cache[idx, slots[s].long()], bp[s])
+        assert torch.equal(cnorm[idx, slots[s].long()], bn[s])
+        written[idx, slots[s].long()] = True
+    assert torch.all(cache[~written] == 0xAB) and torch.all(cnorm[~written] == -1.0)
+    # and the bulk encode itself matches the oracle on a sample
+    xs = toks.reshape(-1, d)[:2048].cpu().numpy()
+    det = O.encode_detail(xs, bits, 42)
+    assert code_mismatches(bp.reshape(-1, P)[:2048].numpy(), det, bits, d) == 0
+
+
+def test_append_out_of_range_slot_is_skipped_and_flagged(K, W):
+    tq = K.TurboQuant(128, 4)
+    n_seq, h, s_max = 4, 8, 8
+    x = W.append_stream(run=0, steps=1, n_seq=n_seq, H=h, d=128)[0].contiguous()
+    cache = torch.zeros((n_seq, s_max, h, 64), dtype=torch.uint8, device="cuda")
+    cn = torch.zeros((n_seq, s_max, h), dtype=torch.float32, device="cuda")
+    slot = torch.tensor([0, -1, s_max, 3], dtype=torch.int32, device="cuda")
+    K.tq_device_error()  # clear
+    tq.encode_append(x, cache, cn, slot)
+    st, bits = K.tq_device_error()
+    assert st == K.TQ_ERR_DEVICE and bits & K.TQ_DEVERR_SLOT_RANGE
+    assert torch.all(cache[1] == 0) and torch.all(cache[2] == 0)
+    assert torch.any(cache[0, 0] != 0) and torch.any(cache[3, 3] != 0)
+
+
+def test_non_default_stream(K, W):
+    x = W.single_tensor(n=3000, seed=5).cuda()
+    tq = K.TurboQuant(128, 3)
+    ref_p, ref_n = _encode(tq, x)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        p, n = tq.encode(x, stream=s)
+    s.synchronize()
+    assert torch.equal(p, ref_p) and torch.equal(n, ref_n)
+
+
+def test_bounded_wait_times_out_and_context_survives(K, W):
+    """A kernel whose bulk copies never arrive: its bounded mbarrier wait runs
+    out, it records TQ_DEVERR_TIMEOUT and returns; the host reads the status
+    and the next call works."""
+    tq = K.TurboQuant(128, 4)
+    x = W.single_tensor(n=256).cuda()
+    p = torch.zeros(256, 64, dtype=torch.uint8, device="cuda")
+    nrm = torch.zeros(256, dtype=torch.float32, device="cuda")
+    K.tq_device_error()
+    assert K._binding.tq_test_encode_stalled(tq.ctx, x, 256, p, nrm) == K.TQ_OK
+    st, bits = K.tq_device_error()
+    assert st == K.TQ_ERR_TIMEOUT and bits & K.TQ_DEVERR_TIMEOUT
+    assert torch.all(p == 0)
+    # context usable afterwards, error word cleared
+    p2, n2 = _encode(tq, x)
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    det = O.encode_detail(x.cpu().numpy(), 4, 42)
+    assert code_mismatches(p2.cpu().numpy(), det, 4, 128) == 0
