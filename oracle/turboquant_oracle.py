@@ -55,6 +55,7 @@ __all__ = [
     "splitmix64",
     "sign_vector",
     "hadamard",
+    "hadamard_pm",
     "packed_bytes",
     "compressed_bytes_per_vector",
     "pack_codes",
@@ -187,15 +188,20 @@ def sign_vector(seed: int, d: int) -> np.ndarray:
 # section "What TurboQuant is"), dense, natural (Sylvester) order.
 # --------------------------------------------------------------------------
 
-def hadamard(d: int) -> np.ndarray:
-    """H[i, j] = (-1)^popcount(i & j) / sqrt(d), written entry by entry."""
+def hadamard_pm(d: int) -> np.ndarray:
+    """The unnormalised +-1 Walsh-Hadamard matrix, (-1)^popcount(i & j), entry by entry."""
     if d < 1 or d & (d - 1):
         raise ValueError("d must be a power of two")
     H = np.empty((d, d), dtype=np.float64)
     for i in range(d):
         for j in range(d):
             H[i, j] = -1.0 if bin(i & j).count("1") % 2 else 1.0
-    return H / math.sqrt(d)
+    return H
+
+
+def hadamard(d: int) -> np.ndarray:
+    """Orthonormal H[i, j] = (-1)^popcount(i & j) / sqrt(d)."""
+    return hadamard_pm(d) / math.sqrt(d)
 
 
 # --------------------------------------------------------------------------
@@ -279,14 +285,15 @@ def encode_detail(x_f16: np.ndarray, bits: int, seed: int) -> dict:
     d = x16.shape[-1]
     x = _as_rows(x16, d).astype(np.float64)  # fp16 -> fp64 is exact
     norm64 = np.sqrt((x * x).sum(axis=1))
-    # step 1: unit direction (zero vector -> zero direction)
-    safe = np.where(norm64 > 0.0, norm64, 1.0)
-    u = np.where(norm64[:, None] > 0.0, x / safe[:, None], 0.0)
-    # step 2: rotate: random sign flip, orthonormal Hadamard, then scale by sqrt(d)
+    # steps 1-2: z = sqrt(d) * H D (x / N) with H orthonormal, written as
+    # (H_pm D x) / N: H_pm D x is a sum of +-x_k, exact in fp64 for fp16 input
+    # (multiples of 2^-24 below 2^23), so the only rounding is the final
+    # division and a coordinate that is exactly 0 stays exactly 0.
+    # (zero vector -> z = 0)
     s = sign_vector(seed, d)
-    H = hadamard(d)
-    y = (u * s[None, :]) @ H.T
-    z = math.sqrt(d) * y
+    w = (x * s[None, :]) @ hadamard_pm(d).T
+    safe = np.where(norm64 > 0.0, norm64, 1.0)
+    z = np.where(norm64[:, None] > 0.0, w / safe[:, None], 0.0)
     # step 3: nearest level of the format codebook
     t = format_boundaries(format_levels(bits))
     idx = quantize(z, t)

@@ -23,7 +23,8 @@ from conftest import golden_lines
 def test_hadamard_is_sylvester_and_orthonormal(d):
     H = O.hadamard(d)
     # library routine: scipy's Sylvester construction, natural order
-    assert np.array_equal(H * math.sqrt(d), scipy.linalg.hadamard(d).astype(np.float64))
+    assert np.array_equal(O.hadamard_pm(d), scipy.linalg.hadamard(d).astype(np.float64))
+    assert np.array_equal(H, scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d))
     assert np.abs(H @ H - np.eye(d)).max() < 1e-12
     rng = np.random.default_rng(d)
     v = rng.standard_normal(d)
@@ -223,6 +224,21 @@ def test_rotation_order_on_signed_hadamard_rows(d, bits):
         assert np.abs(out["z"][0] - want).max() < 1e-12
         assert out["idx"][0, k] == (1 << bits) - 1
         assert abs(out["norm64"][0] - math.sqrt(d)) < 1e-12
+
+
+def test_exact_zero_coordinates_stay_zero():
+    """A rotated coordinate that is exactly 0 in real arithmetic gives z == 0
+    (and so the upper middle level), not a rounding residue of either sign."""
+    d = 128
+    s = O.sign_vector(42, d)
+    R = scipy.linalg.hadamard(d).astype(np.float64)
+    # x = D (r_1 + r_2): rotates to sqrt(d)/|x| (e_1 + e_2) * ..., every other coordinate exactly 0
+    x = (s * (R[1] + R[2]) * 0.375).astype(np.float16)[None, :]
+    out = O.encode_detail(x, 4, 42)
+    zero = np.ones(d, dtype=bool)
+    zero[[1, 2]] = False
+    assert np.all(out["z"][0, zero] == 0.0)
+    assert np.all(out["idx"][0, zero] == 8)
 
 
 def test_norm_is_float32_of_fp64_norm():
