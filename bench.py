@@ -135,6 +135,22 @@ def _ev(torch):
     return torch.cuda.Event(enable_timing=True)
 
 
+def reduce_max_ms(ms: float, world: int, dist=None, device=None) -> float:
+    """Max over ranks of a per-rank time (the slowest rank sets the job time)."""
+    if world <= 1:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step_per_rank: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: the bytes all ranks processed / the max-over-ranks time."""
+    return bytes_per_step_per_rank * steps * world / (ms_max / 1e3) / 1e9
+
+
 def _codec_step_setup(K, W, torch, rank):
     """Buffers and the 12 launches of one step (closures on the current stream)."""
     k, v = W.llama_layer(device="cuda", k_seed=1 + 100 * rank, v_seed=2 + 100 * rank)
@@ -292,22 +308,24 @@ def run_ours(args, rank, world, local_rank):
     err = K.tq_device_error()
     evs = [[(_ev(torch), _ev(torch)) for _ in launches] for _ in range(args.steps)]
     t0, t1 = _ev(torch), _ev(torch)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        # keep the GPU under the same load for ~1 s so the sampler (200 ms
+        # period) records clocks under load, then time exactly `steps` steps
+        settle0 = time.perf_counter()
+        while time.perf_counter() - settle0 < 1.0:
+            step()
+            torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         t0.record()
         for s in range(args.steps):
             step(evs[s])
         t1.record()
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = tt.item()
+        if world > 1:
+            dist.barrier()
+    ms = reduce_max_ms(t0.elapsed_time(t1), world, dist, "cuda")
     ms_step = ms / args.steps
 
     # per-kernel averages inside the timed region
@@ -334,7 +352,7 @@ def run_ours(args, rank, world, local_rank):
 
     result = {
         "metric": "encode/decode GB/s (fp16-equivalent) & % of HBM roofline; fused attn tokens/s",
-        "value": fp16eq_step * args.steps * world / (ms / 1e3) / 1e9,
+        "value": job_throughput(fp16eq_step, args.steps, world, ms),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -401,17 +419,13 @@ def _e2e(K, torch, S, steps, world, dist):
         step()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = tt.item()
+    ms = reduce_max_ms(e0.elapsed_time(e1), world, dist, "cuda")
     for b in BITS:
         P = S["codecs"][b].packed_bytes
         h2d += 2 * (n * 2 * D) + 2 * (n * P + n * 4)
         d2h += 2 * (n * P + n * 4) + 2 * (n * 2 * D)
     fp16eq = 12 * 2 * D * n
-    return {"value": fp16eq * steps * world / (ms / 1e3) / 1e9, "unit": "GB/s",
+    return {"value": job_throughput(fp16eq, steps, world, ms), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "note": "tq_encode/tq_decode with inputs copied from pinned host memory and results copied back, "
                     "one stream"}
@@ -449,8 +463,52 @@ def run_reference(args):
                                           "d2h_bytes_per_step": 0}}
 
 
+PROFILE_CASES = ["encode_b2", "encode_b3", "encode_b4", "decode_b2", "decode_b3", "decode_b4", "attn"]
+
+
+def run_profile_case(case: str, launches: int = 3):
+    """A small, self-contained case for Nsight Compute: a few launches of one
+    kernel on the benchmark's shapes (the layer tensor is 128 MiB, larger than
+    L2; the decode-step cache is ~0.4 GB), after one warm-up launch."""
+    import torch
+
+    import kv_cache_vector_turboquant_b200 as K
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    torch.cuda.set_device(0)
+    if case == "attn":
+        a = ATTN
+        q, k, v = W.decode_step(a["B"], a["Hq"], a["Hkv"], a["S"], a["d"])
+        kc, vc = K.TurboQuant(a["d"], a["kb"]), K.TurboQuant(a["d"], a["vb"])
+        kp, kn = kc.encode(k)
+        vp, vn = vc.encode(v)
+        del k, v
+        pos = torch.full((a["B"],), a["S"], dtype=torch.int32, device="cuda")
+        for _ in range(1 + launches):
+            K.attend_decode(q, kc, vc, kp, kn, vp, vn, pos)
+    else:
+        kind, b = case.split("_b")
+        b = int(b)
+        _, v = W.llama_layer(device="cuda")
+        x = v.reshape(-1, D)
+        del _
+        c = K.TurboQuant(D, b)
+        p, n = c.encode(x)
+        out = torch.empty_like(x)
+        for _ in range(1 + launches):
+            if kind == "encode":
+                c.encode(x, out=(p, n))
+            else:
+                c.decode(p, n, out=out)
+    torch.cuda.synchronize()
+    st = K.tq_device_error()
+    print(json.dumps({"profile_case": case, "launches": 1 + launches, "device_error": list(st)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", choices=PROFILE_CASES, default=None,
+                    help="run a few launches of one kernel for Nsight Compute and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
@@ -460,6 +518,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

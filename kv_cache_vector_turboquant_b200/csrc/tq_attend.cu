@@ -9,15 +9,30 @@
 //   acc = sum_t p_t n^V_t c_V[idx^V_t],   o = D_V H_pm (acc / l) / d,
 // and rotated back once at the end.
 //
-// Split-S: the grid is (n_split, B, kv-head groups of 8). Each CTA owns a
-// chunk of cache positions of one sequence and up to 8 kv heads (one warp
-// each). Position rows (all heads of one position, contiguous in the
-// [B, S, Hkv, P] layout) are brought into padded shared rows by 1-D bulk
-// copies (TMA, no multicast) through a 3-stage mbarrier pipeline; tiles are 32
-// positions. Per tile and kv head: scores with lane = position, online softmax
-// in the exp2 domain, value accumulation with lane = coordinate block. The
-// partial (max, sum, accumulator) of every split goes to the workspace; a
-// second kernel merges the splits (log-sum-exp) and applies D_V H / d.
+// Split-S: the grid is (n_split, B, kv-head groups). Each CTA owns a chunk of
+// cache positions of one sequence and a group of kv heads; each warp owns one
+// kv head (and, for more than 4 query heads per kv head, one group of 4 query
+// heads). Position rows of the group (contiguous in the [B, S, Hkv, P]
+// layout) arrive in padded shared rows by 1-D bulk copies (TMA, no
+// multicast) through a 2-stage mbarrier pipeline of 32-position tiles.
+//
+// Both contractions run on the tensor cores (mma.sync m16n8k16, fp16 inputs,
+// f32 accumulation); the packed codes are turned into fp16 operand fragments
+// in registers through lane-replicated shared tables indexed by two codes,
+// never into fp16 tiles in memory:
+//  * scores: A = 16 positions x 16 dims of K levels, B = 16 dims x 8 columns
+//    holding the rotated query of 4 heads split as fp16 hi + lo parts (so the
+//    query keeps ~22 bits); the two parts are summed from the accumulator.
+//    The d dims are visited in a permuted order so that each thread's codes
+//    are one contiguous quarter of the row; q~ uses the same order.
+//  * values: A = 16 dims x 16 positions of V levels (dims permuted so each
+//    thread's codes are a contiguous eighth of the row, and the accumulator
+//    comes out in natural order), B = 16 positions x 8 columns of
+//    p_t n^V_t split as fp16 hi + lo, transposed through a small per-warp
+//    buffer.
+// Online softmax in the exp2 domain per 32-position tile. The partial (max,
+// sum, accumulator) of every split goes to the workspace; a second kernel
+// merges the splits (log-sum-exp) and applies D_V H / d.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,9 +43,9 @@
 
 namespace tq {
 
-constexpr int ATT_WARPS = 8;   // kv heads per CTA (one warp each)
-constexpr int ATT_STAGES = 3;  // position tiles in flight
-constexpr int ATT_TILE = 32;   // positions per tile
+constexpr int ATT_WARPS = 8;   // warps per CTA: one per (kv head, group of 4 query heads)
+constexpr int ATT_STAGES = 2;  // position tiles in flight
+constexpr int ATT_TILE = 32;   // positions per tile (two blocks of 16)
 constexpr int ATT_MAXG = 8;    // query heads per kv head supported
 constexpr int ATT_TARGET_CTAS = 296;
 
@@ -55,6 +70,8 @@ struct AttnArgs {
   int64_t s_max;
   int n_split;
   int chunk;  // positions per split (multiple of ATT_TILE)
+  int nt;     // column tiles per kv head: 1 (<= 4 query heads per kv head) or 2
+  int hw_max; // kv heads per CTA: 8 / nt
   float q_scale;  // log2(e) / (d sqrt(d))
 };
 
@@ -63,7 +80,7 @@ struct AttnArgs {
 // workspace size does too.
 inline void attn_split(int B, int64_t s_max, int* n_split, int* chunk) {
   const int64_t tiles = (s_max + ATT_TILE - 1) / ATT_TILE;
-  int64_t ns = (ATT_TARGET_CTAS + (int64_t)B - 1) / (int64_t)B;
+  int64_t ns = ATT_TARGET_CTAS / (int64_t)B;  // one wave of CTAs
   ns = std::max<int64_t>(1, std::min<int64_t>(ns, tiles));
   const int64_t tiles_per = (tiles + ns - 1) / ns;
   *chunk = (int)(tiles_per * ATT_TILE);
@@ -72,67 +89,143 @@ inline void attn_split(int B, int64_t s_max, int* n_split, int* chunk) {
 
 template <int D, int KB, int VB>
 struct AttCfg {
-  static constexpr int PK = D * KB / 8;
+  static constexpr int PK = D * KB / 8;  // packed bytes of a K row (one head)
   static constexpr int PV = D * VB / 8;
-  static constexpr int LK = 1 << KB;
-  static constexpr int LV = 1 << VB;
-  static constexpr int CPL = D / 32;  // coordinates per lane in the value phase
+  static constexpr int KT = PK / 4;  // K bytes per thread: a quarter of the row
+  static constexpr int VT = PV / 8;  // V bytes per thread: an eighth of the row
+  static constexpr int KW = (KT + 3) / 4 + 1;  // words holding a thread's K bits (+1 for straddling)
+  static constexpr int VW = (VT + 3) / 4 + 1;
+  static constexpr int KF = 2 * KB;  // bits of a two-code field
+  static constexpr int VF = 2 * VB;
+  static constexpr int LK2 = 1 << KF;  // two-code table entries
+  static constexpr int LV2 = 1 << VF;
+  static constexpr int NB = D / 16;  // k-blocks (scores) = m-blocks (values)
 };
 
+inline int round_units(int bytes, int unit, int mod, int rem) {
+  int u = (bytes + unit - 1) / unit;
+  while (u % mod != rem) ++u;
+  return u * unit;
+}
 
 // Shared-memory layout of the partial kernel (bytes); identical on host and device.
 struct AttSmem {
-  int bar, qt, kst, vst, pw, lutk, lutv, total;
-  int krow, vrow, stage;
-  __host__ __device__ AttSmem(int D, int PK, int PV, int LK, int LV, int g) {
-    krow = ATT_WARPS * PK + 16;  // padded position row of K (all heads of the group)
-    vrow = ATT_WARPS * PV + 16;
+  int krow, vrow, stage, bar, st0, lutk, lutv, pw, nrm, qt, total;
+  __host__ __device__ AttSmem(int D, int PK, int PV, int LK2, int LV2, int hw_max, int g) {
+    // padded position rows: K rows an odd number of 16-byte units apart mod 8
+    // (== 4), V rows a number of words == 4 mod 16, so the fragment loads of
+    // a warp fall in distinct banks
+    int u = (hw_max * PK + 15) / 16;
+    while (u % 8 != 4) ++u;
+    krow = u * 16;
+    int w = (hw_max * PV + 3) / 4;
+    while (w % 16 != 4) ++w;
+    vrow = w * 4;
     stage = ATT_TILE * (krow + vrow);
     bar = 0;
-    qt = 128;
-    kst = qt + ATT_WARPS * g * D * 4;
-    vst = kst + ATT_TILE * krow;  // stage s: kst + s*stage (K rows), then V rows
-    pw = kst + ATT_STAGES * stage;
-    lutk = pw + ATT_WARPS * ATT_TILE * ATT_MAXG * 4;
-    lutv = lutk + LK * 32 * 4;
-    total = lutv + LV * 32 * 4;
+    st0 = 128;
+    lutk = st0 + ATT_STAGES * stage;
+    lutv = lutk + LK2 * 32 * 4;
+    pw = lutv + LV2 * 32 * 4;                      // per warp: 2 blocks x 8 cols x 16 pos fp16
+    nrm = pw + ATT_WARPS * 2 * 8 * 16 * 2;          // per warp: K and V norms of the tile
+    qt = nrm + ATT_WARPS * 2 * ATT_TILE * 4;        // rotated queries of the CTA (f32)
+    total = qt + hw_max * g * D * 4;
   }
 };
 
-TQ_DEV float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+TQ_DEV float warp_max8(float v) {  // max over the 8 lanes sharing lane & 3
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
 }
-TQ_DEV float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+TQ_DEV float warp_sum8(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  v += __shfl_xor_sync(0xffffffffu, v, 8);
+  return v + __shfl_xor_sync(0xffffffffu, v, 16);
 }
 
-// Extract `NB` bits at bit offset `off` of a little-endian word stream.
-template <int NB>
-TQ_DEV uint32_t bits_at(const uint32_t* w, int off) {
+// `NB` bits at bit offset `off` of a little-endian word stream.
+template <int NB, int N>
+TQ_DEV uint32_t bits_at(const uint32_t (&w)[N], int off) {
   uint32_t f = w[off >> 5] >> (off & 31);
   if ((off & 31) + NB > 32) f |= w[(off >> 5) + 1] << (32 - (off & 31));
   return f & ((1u << NB) - 1u);
 }
 
+// NBYTES bytes of shared memory starting at p (at least 2-byte aligned) as a
+// little-endian word stream w[0..].
+template <int NBYTES, int NW>
+TQ_DEV void load_bytes(uint32_t (&w)[NW], const uint8_t* p) {
+  if (NBYTES % 16 == 0) {
+#pragma unroll
+    for (int i = 0; i < NBYTES / 16; ++i) {
+      const uint4 r = reinterpret_cast<const uint4*>(p)[i];
+      w[4 * i] = r.x;
+      w[4 * i + 1] = r.y;
+      w[4 * i + 2] = r.z;
+      w[4 * i + 3] = r.w;
+    }
+  } else if (NBYTES % 8 == 0) {
+#pragma unroll
+    for (int i = 0; i < NBYTES / 8; ++i) {
+      const uint2 r = reinterpret_cast<const uint2*>(p)[i];
+      w[2 * i] = r.x;
+      w[2 * i + 1] = r.y;
+    }
+  } else if (NBYTES % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NBYTES / 4; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  } else {
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(p);
+    const uint32_t* base = reinterpret_cast<const uint32_t*>(addr & ~uintptr_t(3));
+    const uint32_t sh = (uint32_t)(addr & 3) * 8u;
+    uint32_t raw[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) raw[i] = base[i];
+#pragma unroll
+    for (int i = 0; i + 1 < NW; ++i) w[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
+    w[NW - 1] = raw[NW - 1] >> sh;
+  }
+}
+
+TQ_DEV uint32_t lds32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+  return r;
+}
+
+// D += A * B on the tensor cores: m16n8k16, fp16 operands, f32 accumulate.
+TQ_DEV void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+TQ_DEV uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <int D, int KB, int VB>
 __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const __grid_constant__ AttnArgs a) {
   using Cfg = AttCfg<D, KB, VB>;
-  constexpr int PK = Cfg::PK, PV = Cfg::PV, CPL = Cfg::CPL;
+  constexpr int PK = Cfg::PK, PV = Cfg::PV, KT = Cfg::KT, VT = Cfg::VT, NB = Cfg::NB;
+  constexpr int KF = Cfg::KF, VF = Cfg::VF;
   extern __shared__ __align__(128) uint8_t smem[];
-  const AttSmem L(D, PK, PV, Cfg::LK, Cfg::LV, a.g);
+  const AttSmem L(D, PK, PV, Cfg::LK2, Cfg::LV2, a.hw_max, a.g);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
   const int split = blockIdx.x, b = blockIdx.y;
-  const int hk0 = blockIdx.z * ATT_WARPS;
-  const int hw = min(ATT_WARPS, a.hkv - hk0);  // kv heads in this CTA
+  const int hk0 = blockIdx.z * a.hw_max;
+  const int hw = min(a.hw_max, a.hkv - hk0);  // kv heads in this CTA
   const int g = a.g;
+  const int hl = warp / a.nt, nt = warp % a.nt;  // this warp's kv head (local) and column tile
+  const bool head_ok = hl < hw;
+  const int hk = hk0 + hl;
 
   int64_t pos = a.positions[b];
   if (pos > a.s_max) {
-    if (threadIdx.x == 0 && split == 0) record_error(a.err, TQ_DEVERR_POS_RANGE);
+    if (threadIdx.x == 0 && split == 0 && blockIdx.z == 0) record_error(a.err, TQ_DEVERR_POS_RANGE);
     pos = a.s_max;
   }
   const int64_t s0 = (int64_t)split * a.chunk;
@@ -142,12 +235,21 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
   float* qt = reinterpret_cast<float*>(smem + L.qt);
-  float* pw = reinterpret_cast<float*>(smem + L.pw) + warp * ATT_TILE * ATT_MAXG;
+  __half* pwb = reinterpret_cast<__half*>(smem + L.pw) + warp * 2 * 8 * 16;
+  float* nks = reinterpret_cast<float*>(smem + L.nrm) + warp * 2 * ATT_TILE;
+  float* nvs = nks + ATT_TILE;
   {
-    float* lk = reinterpret_cast<float*>(smem + L.lutk);
-    for (int e = threadIdx.x; e < Cfg::LK * 32; e += blockDim.x) lk[e] = a.k_levels[e >> 5];
-    float* lv = reinterpret_cast<float*>(smem + L.lutv);
-    for (int e = threadIdx.x; e < Cfg::LV * 32; e += blockDim.x) lv[e] = a.v_levels[e >> 5];
+    // two-code tables: entry f = code_lo | code_hi << bits -> fp16 pair (c[lo], c[hi])
+    uint32_t* lk = reinterpret_cast<uint32_t*>(smem + L.lutk);
+    for (int e = threadIdx.x; e < Cfg::LK2 * 32; e += blockDim.x) {
+      const int f = e >> 5;
+      lk[e] = pack_half2(a.k_levels[f & ((1 << KB) - 1)], a.k_levels[f >> KB]);
+    }
+    uint32_t* lv = reinterpret_cast<uint32_t*>(smem + L.lutv);
+    for (int e = threadIdx.x; e < Cfg::LV2 * 32; e += blockDim.x) {
+      const int f = e >> 5;
+      lv[e] = pack_half2(a.v_levels[f & ((1 << VB) - 1)], a.v_levels[f >> VB]);
+    }
   }
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -156,7 +258,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
   }
   __syncthreads();
 
-  // producer: warp 0 issues one K row copy and one V row copy per position
+  // producer: warp 0 issues one K and one V row copy per position of a tile
   const uint32_t krow_bytes = (uint32_t)(hw * PK), vrow_bytes = (uint32_t)(hw * PV);
   auto issue = [&](int tile, int stage) {
     const int64_t t0 = s0 + (int64_t)tile * ATT_TILE;
@@ -166,7 +268,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     __syncwarp();
     if (lane < nv) {
       const int64_t row = ((int64_t)b * a.s_max + t0 + lane) * a.hkv + hk0;
-      uint8_t* st = smem + L.kst + stage * L.stage;
+      uint8_t* st = smem + L.st0 + stage * L.stage;
       bulk_g2s(smem_u32(st + lane * L.krow), a.k_packed + row * PK, krow_bytes, bar);
       bulk_g2s(smem_u32(st + ATT_TILE * L.krow + lane * L.vrow), a.v_packed + row * PV, vrow_bytes, bar);
     }
@@ -197,21 +299,48 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     }
     __syncthreads();
   }
-  for (int e = threadIdx.x; e < nq * D; e += blockDim.x) qt[e] *= a.q_scale;
-  __syncthreads();
 
-  const bool head_ok = warp < hw;
-  const int hk = hk0 + warp;
-  const float* qw = qt + warp * g * D;  // this warp's g query heads
+  // B fragments of the score MMA: column gq = (query head nt*4 + gq/2, hi or lo
+  // part), rows = dims pi(kb, k) = tq*D/4 + 4*kb + k' for the fragment's k
+  uint32_t bq[NB][2];
+  {
+    const int j = nt * 4 + (gq >> 1);
+    const bool lo = gq & 1;
+    const float* qrow = qt + (hl * g + (j < g ? j : 0)) * D;
+#pragma unroll
+    for (int kb = 0; kb < NB; ++kb) {
+#pragma unroll
+      for (int e2 = 0; e2 < 2; ++e2) {
+        const int d0 = tq * (D / 4) + 4 * kb + 2 * e2;
+        float v0 = 0.f, v1 = 0.f;
+        if (head_ok && j < g) {
+          v0 = qrow[d0] * a.q_scale;
+          v1 = qrow[d0 + 1] * a.q_scale;
+        }
+        if (lo) {
+          v0 -= __half2float(__float2half_rn(v0));
+          v1 -= __half2float(__float2half_rn(v1));
+        }
+        bq[kb][e2] = pack_half2(v0, v1);
+      }
+    }
+  }
+
   const uint32_t lutk_lane = smem_u32(smem + L.lutk) + lane * 4u;
   const uint32_t lutv_lane = smem_u32(smem + L.lutv) + lane * 4u;
-  float m[ATT_MAXG], l[ATT_MAXG], acc[ATT_MAXG][CPL];
+  float m_run = -INFINITY, l_run = 0.f;
+  float acc[NB][4];
 #pragma unroll
-  for (int j = 0; j < ATT_MAXG; ++j) {
-    m[j] = -INFINITY;
-    l[j] = 0.f;
+  for (int i = 0; i < NB; ++i)
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[j][c] = 0.f;
+    for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+
+  // norms of the first tile (lane = position), then prefetched one tile ahead
+  float nk_next = 0.f, nv_next = 0.f;
+  if (head_ok && ntiles > 0 && lane < min64(ATT_TILE, npos)) {
+    const int64_t row = ((int64_t)b * a.s_max + s0 + lane) * a.hkv + hk;
+    nk_next = __ldg(a.k_norms + row);
+    nv_next = __ldg(a.v_norms + row);
   }
 
   uint32_t parity = 0;
@@ -219,13 +348,22 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     const int stage = tile % ATT_STAGES;
     const int64_t t0 = s0 + (int64_t)tile * ATT_TILE;
     const int nv = (int)min64(ATT_TILE, s1 - t0);
+    nks[lane] = nk_next;
+    nvs[lane] = nv_next;
+    if (head_ok && tile + 1 < ntiles) {
+      const int64_t t1 = t0 + ATT_TILE;
+      if (lane < min64(ATT_TILE, s1 - t1)) {
+        const int64_t row = ((int64_t)b * a.s_max + t1 + lane) * a.hkv + hk;
+        nk_next = __ldg(a.k_norms + row);
+        nv_next = __ldg(a.v_norms + row);
+      }
+    }
     // all threads poll the barrier; the CTA acts on one agreed outcome
     const bool ok = __syncthreads_and(mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u,
                                                         a.wait_limit) ? 1 : 0) != 0;
     if (!ok) {
       if (threadIdx.x == 0) {
         record_error(a.err, TQ_DEVERR_TIMEOUT);
-        // drain the other stages already issued, bounded, then leave
         for (int s = 1; s < ATT_STAGES; ++s) {
           const int os = (stage + s) % ATT_STAGES;
           if (tile + s < ntiles) (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
@@ -234,100 +372,80 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
       return;
     }
     parity ^= 1u << stage;
-    const uint8_t* kst = smem + L.kst + stage * L.stage;
+    const uint8_t* kst = smem + L.st0 + stage * L.stage;
     const uint8_t* vst = kst + ATT_TILE * L.krow;
 
     if (head_ok) {
-      // ---- scores, lane = position
-      const bool valid = lane < nv;
-      float sc[ATT_MAXG];
+      // ---- scores on the tensor cores: 2 blocks of 16 positions
+      float sc[2][2];
 #pragma unroll
-      for (int j = 0; j < ATT_MAXG; ++j) sc[j] = 0.f;
-      float nk = 0.f, nvn = 0.f;
-      if (valid) {
-        const int64_t row = ((int64_t)b * a.s_max + t0 + lane) * a.hkv + hk;
-        nk = __ldg(a.k_norms + row);
-        nvn = __ldg(a.v_norms + row);
-        const uint32_t* kw = reinterpret_cast<const uint32_t*>(kst + lane * L.krow + warp * PK);
-        uint32_t words[PK / 4];
+      for (int mb16 = 0; mb16 < 2; ++mb16) {
+        const int r0 = mb16 * 16 + gq, r1 = r0 + 8;
+        uint32_t kw0[Cfg::KW], kw1[Cfg::KW];
+        load_bytes<KT>(kw0, kst + r0 * L.krow + hl * PK + tq * KT);
+        load_bytes<KT>(kw1, kst + r1 * L.krow + hl * PK + tq * KT);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int w = 0; w < PK / 4; ++w) words[w] = kw[w];
-        constexpr int CH = 32;  // coordinates per chunk held in registers
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += CH) {
-          float lv[CH];
-#pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            const uint32_t code = bits_at<KB>(words, (c0 + i) * KB);
-            float val;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(val) : "r"(code * 128u + lutk_lane));
-            lv[i] = val;
-          }
-#pragma unroll
-          for (int j = 0; j < ATT_MAXG; ++j) {
-            if (j < g) {
-              const float4* qv = reinterpret_cast<const float4*>(qw + j * D + c0);
-              float s = 0.f;
-#pragma unroll
-              for (int i4 = 0; i4 < CH / 4; ++i4) {
-                const float4 qq = qv[i4];
-                s = fmaf(qq.x, lv[4 * i4], s);
-                s = fmaf(qq.y, lv[4 * i4 + 1], s);
-                s = fmaf(qq.z, lv[4 * i4 + 2], s);
-                s = fmaf(qq.w, lv[4 * i4 + 3], s);
-              }
-              sc[j] += s;
-            }
-          }
+        for (int kb = 0; kb < NB; ++kb) {
+          const uint32_t a0 = lds32(bits_at<KF>(kw0, (2 * kb) * KF) * 128u + lutk_lane);
+          const uint32_t a1 = lds32(bits_at<KF>(kw1, (2 * kb) * KF) * 128u + lutk_lane);
+          const uint32_t a2 = lds32(bits_at<KF>(kw0, (2 * kb + 1) * KF) * 128u + lutk_lane);
+          const uint32_t a3 = lds32(bits_at<KF>(kw1, (2 * kb + 1) * KF) * 128u + lutk_lane);
+          mma16816(c, a0, a1, a2, a3, bq[kb][0], bq[kb][1]);
         }
+        sc[mb16][0] = (r0 < nv) ? (c[0] + c[1]) * nks[r0] : -INFINITY;
+        sc[mb16][1] = (r1 < nv) ? (c[2] + c[3]) * nks[r1] : -INFINITY;
       }
-      // ---- online softmax (log2 domain), per query head of the group
-      float alpha[ATT_MAXG];
+      // ---- online softmax (log2 domain) for query head nt*4 + tq
+      const float mx = warp_max8(fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])));
+      const float mn = fmaxf(m_run, mx);
+      float alpha = 1.f, p[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      if (mn != -INFINITY) {
+        alpha = exp2f(m_run - mn);
 #pragma unroll
-      for (int j = 0; j < ATT_MAXG; ++j) {
-        alpha[j] = 1.f;
-        if (j < g) {
-          const float s = valid ? sc[j] * nk : -INFINITY;
-          const float mx = warp_max(s);
-          const float mn = fmaxf(m[j], mx);
-          float p = 0.f;
-          if (mn != -INFINITY) {
-            alpha[j] = exp2f(m[j] - mn);
-            p = valid ? exp2f(s - mn) : 0.f;
-          }
-          l[j] = l[j] * alpha[j] + warp_sum(p);
-          m[j] = mn;
-          pw[lane * ATT_MAXG + j] = p * nvn;
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) p[i][r] = exp2f(sc[i][r] - mn);  // exp2(-inf) = 0
+      }
+      l_run = l_run * alpha + warp_sum8(p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+      m_run = mn;
+#pragma unroll
+      for (int i = 0; i < NB; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[i][c] *= alpha;
+      // p * n^V as fp16 hi + lo, stored column-major [block][col][position]
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int pr = gq + 8 * r;
+          const float pv = (i * 16 + pr < nv) ? p[i][r] * nvs[i * 16 + pr] : 0.f;
+          const __half hi = __float2half_rn(pv);
+          const __half lo = __float2half_rn(pv - __half2float(hi));
+          pwb[(i * 8 + 2 * tq) * 16 + pr] = hi;
+          pwb[(i * 8 + 2 * tq + 1) * 16 + pr] = lo;
         }
       }
       __syncwarp();
-      // ---- values, lane = block of CPL coordinates
+      // ---- values on the tensor cores: acc[dims x cols] += V^T[dims x 16 pos] * P'[16 pos x cols]
 #pragma unroll
-      for (int j = 0; j < ATT_MAXG; ++j)
+      for (int mb16 = 0; mb16 < 2; ++mb16) {
+        const uint32_t* pcol = reinterpret_cast<const uint32_t*>(pwb + (mb16 * 8 + gq) * 16);
+        const uint32_t bp0 = pcol[tq], bp1 = pcol[tq + 4];
+        uint32_t vw[4][Cfg::VW];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[j][c] *= alpha[j];
-      for (int t = 0; t < nv; ++t) {
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vst + t * L.vrow + warp * PV);
-        const int off = lane * CPL * VB;
-        uint32_t two[2];
-        two[0] = vw[off >> 5];
-        two[1] = ((off & 31) + CPL * VB > 32) ? vw[(off >> 5) + 1] : 0u;
-        float lvv[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const uint32_t code = bits_at<VB>(two, (off & 31) + c * VB);
-          float val;
-          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(val) : "r"(code * 128u + lutv_lane));
-          lvv[c] = val;
+        for (int j = 0; j < 4; ++j) {
+          const int r = mb16 * 16 + 2 * tq + (j & 1) + 8 * (j >> 1);
+          load_bytes<VT>(vw[j], vst + r * L.vrow + hl * PV + gq * VT);
         }
-        const float* pt = pw + t * ATT_MAXG;
 #pragma unroll
-        for (int j = 0; j < ATT_MAXG; ++j) {
-          if (j < g) {
-            const float pj = pt[j];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[j][c] = fmaf(pj, lvv[c], acc[j][c]);
-          }
+        for (int mb = 0; mb < NB; ++mb) {
+          const uint32_t l0 = lds32(bits_at<VF>(vw[0], mb * VF) * 128u + lutv_lane);
+          const uint32_t l1 = lds32(bits_at<VF>(vw[1], mb * VF) * 128u + lutv_lane);
+          const uint32_t l2 = lds32(bits_at<VF>(vw[2], mb * VF) * 128u + lutv_lane);
+          const uint32_t l3 = lds32(bits_at<VF>(vw[3], mb * VF) * 128u + lutv_lane);
+          mma16816(acc[mb], __byte_perm(l0, l1, 0x5410), __byte_perm(l0, l1, 0x7632), __byte_perm(l2, l3, 0x5410),
+                   __byte_perm(l2, l3, 0x7632), bp0, bp1);
         }
       }
     }
@@ -335,21 +453,20 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     if (warp == 0 && tile + ATT_STAGES < ntiles) issue(tile + ATT_STAGES, stage);
   }
 
-  // ---- partial results of this split
-  if (head_ok) {
+  // ---- partial results of this split: query head hk*g + nt*4 + tq
+  const int j = nt * 4 + tq;
+  if (head_ok && j < g) {
+    const int h = hk * g + j;
+    const int64_t idx = ((int64_t)b * a.hq + h) * a.n_split + split;
+    if (gq == 0) {
+      a.ws_m[idx] = m_run;
+      a.ws_l[idx] = l_run;
+    }
+    float* dst = a.ws_acc + idx * D + gq * (D / 8);
 #pragma unroll
-    for (int j = 0; j < ATT_MAXG; ++j) {
-      if (j < g) {
-        const int h = hk * g + j;
-        const int64_t idx = ((int64_t)b * a.hq + h) * a.n_split + split;
-        if (lane == 0) {
-          a.ws_m[idx] = m[j];
-          a.ws_l[idx] = l[j];
-        }
-        float* dst = a.ws_acc + idx * D + lane * CPL;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) dst[c] = acc[j][c];
-      }
+    for (int mb = 0; mb < NB; ++mb) {
+      dst[2 * mb] = acc[mb][0] + acc[mb][1];
+      dst[2 * mb + 1] = acc[mb][2] + acc[mb][3];
     }
   }
 }
@@ -397,11 +514,11 @@ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 template <int D, int KB, int VB>
 static cudaError_t launch_attend_t(const AttnArgs& a, cudaStream_t st, int dev) {
   using Cfg = AttCfg<D, KB, VB>;
-  const AttSmem L(D, Cfg::PK, Cfg::PV, Cfg::LK, Cfg::LV, a.g);
+  const AttSmem L(D, Cfg::PK, Cfg::PV, Cfg::LK2, Cfg::LV2, a.hw_max, a.g);
   cudaError_t e = cudaFuncSetAttribute(attend_partial_kernel<D, KB, VB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
-  const dim3 grid(a.n_split, a.B, (a.hkv + ATT_WARPS - 1) / ATT_WARPS);
+  const dim3 grid(a.n_split, a.B, (a.hkv + a.hw_max - 1) / a.hw_max);
   attend_partial_kernel<D, KB, VB><<<grid, ATT_WARPS * 32, L.total, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -432,6 +549,8 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
   // position rows of a kv-head group are copied with 1-D bulk copies: their
   // byte counts and offsets must be multiples of 16
   if ((pk % 16 && hkv % 2) || (pv % 16 && hkv % 2)) return TQ_ERR_UNSUPPORTED;
+  if ((pk * (hkv % 8)) % 16 || (pv * (hkv % 8)) % 16 || (pk * (hkv % 4)) % 16 || (pv * (hkv % 4)) % 16)
+    return TQ_ERR_UNSUPPORTED;
   AttnArgs a;
   for (int i = 0; i < TQ_MAX_D / 2; ++i) {
     a.k_sign_h2[i] = k->t.sign_h2[i];
@@ -453,6 +572,8 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
   a.hkv = hkv;
   a.g = g;
   a.s_max = s_max;
+  a.nt = g > 4 ? 2 : 1;
+  a.hw_max = ATT_WARPS / a.nt;
   attn_split(B, s_max, &a.n_split, &a.chunk);
   const size_t rows = (size_t)B * hq * a.n_split;
   if (ws_bytes < 2 * align16(rows * 4) + rows * (size_t)d * 4) return TQ_ERR_WORKSPACE;

@@ -93,46 +93,16 @@ TQ_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::c
 
 // ---------------------------------------------------------------- f32x2
 
-struct f2 {
-  float x, y;
-};
+// Packed two-wide f32 arithmetic of sm_100 (one instruction for both
+// lanes of the pair), each component rounded exactly like its scalar op.
+using f2 = float2;
 
-TQ_DEV uint64_t as_u64(f2 a) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
-  return r;
-}
-TQ_DEV f2 as_f2(uint64_t r) {
-  f2 a;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
-  return a;
-}
-TQ_DEV f2 add2(f2 a, f2 b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
-  return as_f2(r);
-}
-TQ_DEV f2 sub2(f2 a, f2 b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
-  return as_f2(r);
-}
-TQ_DEV f2 mul2(f2 a, f2 b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
-  return as_f2(r);
-}
-TQ_DEV f2 fma2(f2 a, f2 b, f2 c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
-  return as_f2(r);
-}
+TQ_DEV f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
+TQ_DEV f2 sub2(f2 a, f2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+TQ_DEV f2 mul2(f2 a, f2 b) { return __fmul2_rn(a, b); }
+TQ_DEV f2 fma2(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
 // Round toward -inf (used to take floor(q) through the 2^23 magic constant).
-TQ_DEV f2 add2_rm(f2 a, f2 b) {
-  uint64_t r;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
-  return as_f2(r);
-}
+TQ_DEV f2 add2_rm(f2 a, f2 b) { return __fadd2_rd(a, b); }
 
 // In-register Walsh-Hadamard butterflies over N pairs v[j] = (e_{2j}, e_{2j+1})
 // for the element strides 2, 4, ..., N (pair strides 1 .. N/2). The stride-1

@@ -9,13 +9,15 @@
 // only roundings are the product by N/d (a power-of-two scaling of N, exact)
 // in f32 and the final fp16 conversion.
 //
-// B200 mapping: one vector per lane (two lanes for d = 256). Each warp runs a
-// 3-stage pipeline of 1-D bulk copies (TMA) bringing its tile of packed rows
-// and norms into shared memory; a lane-replicated table indexed by two codes
-// returns (c[a] + c[b], c[a] - c[b]), i.e. the levels already through the
-// first butterfly; the other stages run in registers with f32x2 add/sub; the
-// fp16 rows are staged in padded shared rows and leave through per-row 1-D
-// bulk stores (TMA), so every DRAM write is a full line.
+// B200 mapping: every lane owns 64 coordinates (1, 2 or 4 lanes per vector),
+// 16 warps per SM. Each warp runs a 3-stage pipeline of 1-D bulk copies (TMA)
+// bringing its tile of packed rows and norms into shared memory (row layout
+// chosen so the 64/128-bit shared reads are conflict-free); a lane-replicated
+// table indexed by two codes returns (c[a] + c[b], c[a] - c[b]), the levels
+// already through the first butterfly; the other stages run in registers with
+// f32x2 add/sub and shuffles across the lanes of a vector; the fp16 rows are
+// staged in padded shared rows and leave through per-row 1-D bulk stores
+// (TMA), so every DRAM write is a full line.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -25,33 +27,42 @@
 
 namespace tq {
 
-constexpr int DEC_WARPS = 8;
+constexpr int DEC_WARPS = 16;
 constexpr int DEC_STAGES = 3;
+constexpr int DEC_C = 64;
 
 template <int D, int BITS>
 struct DecCfg {
-  static constexpr int LPV = D > 128 ? 2 : 1;
-  static constexpr int C = D / LPV;
+  static constexpr int C = DEC_C;
+  static constexpr int LPV = D / C;
   static constexpr int NP = C / 2;
   static constexpr int VPW = 32 / LPV;
   static constexpr int P = D * BITS / 8;
-  static constexpr int PL = P / LPV;       // packed bytes per lane
-  static constexpr int WL = PL / 4;        // packed words per lane
+  static constexpr int PL = C * BITS / 8;  // packed bytes per lane: 16, 24, 32
+  static constexpr int WL = PL / 4;
   static constexpr int E = 1 << (2 * BITS);  // pair-table entries
-  static constexpr int TILE_P = VPW * P;   // packed bytes per full tile
-  static constexpr int IN_STAGE = ((TILE_P + 15) / 16) * 16 + 32 * 4;  // packed + norms
-  static constexpr int OUT_ROW = 2 * C + 16;  // padded fp16 lane-row
+  static constexpr int TILE_P = 32 * PL;     // packed bytes of a full tile
+  // 32-byte lane rows (4 bits) are copied one per lane into 48-byte rows so
+  // the 128-bit reads are conflict-free; 16- and 24-byte rows are read
+  // conflict-free straight from the contiguous tile.
+  static constexpr bool ROWS = (PL == 32);
+  static constexpr int PROW = ROWS ? 48 : PL;
+  static constexpr int PACK_BYTES = 32 * PROW;
+  static constexpr int IN_STAGE = PACK_BYTES + VPW * 4;  // packed rows + norms
+  static constexpr int OUT_ROW = 2 * C + 16;              // padded fp16 lane-row
   static constexpr int OUT = 32 * OUT_ROW;
 };
 
 template <int D, int BITS>
 struct DecSmem {
   using Cfg = DecCfg<D, BITS>;
-  static constexpr int BAR = 0;
-  static constexpr int IN = 256;
-  static constexpr int OUT = IN + DEC_WARPS * DEC_STAGES * Cfg::IN_STAGE;
+  static constexpr int BAR = 0;     // warps x stages u64
+  static constexpr int MASK = 512;  // sign masks, up to 128 u32
+  static constexpr int IN = MASK + 512;
+  static constexpr int OUT = IN + DEC_WARPS * DEC_STAGES * ((Cfg::IN_STAGE + 15) / 16 * 16);
   static constexpr int LUT = OUT + DEC_WARPS * Cfg::OUT;
   static constexpr size_t BYTES = (size_t)LUT + (size_t)Cfg::E * 32 * 8;
+  static constexpr int STAGE = (Cfg::IN_STAGE + 15) / 16 * 16;
 };
 
 struct DecArgs {
@@ -76,7 +87,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   using Cfg = DecCfg<D, BITS>;
   using Sm = DecSmem<D, BITS>;
   constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, VPW = Cfg::VPW, WL = Cfg::WL;
-  constexpr int P = Cfg::P, E = Cfg::E;
+  constexpr int E = Cfg::E;
   constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -91,9 +102,11 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
       const int f = e >> 5;
       const float ca = T.levels[f & ((1 << BITS) - 1)];
       const float cb = T.levels[f >> BITS];
-      lut[e] = f2{ca + cb, ca - cb};
+      lut[e] = make_float2(ca + cb, ca - cb);
     }
   }
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem + Sm::MASK);
+  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) smask[i] = T.sign_h2[i];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::BAR) + warp * DEC_STAGES;
   if (lane == 0) {
 #pragma unroll
@@ -102,27 +115,33 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   }
   __syncthreads();
 
-  uint8_t* in0 = smem + Sm::IN + warp * DEC_STAGES * Cfg::IN_STAGE;
-  uint8_t* out_rows = smem + Sm::OUT + warp * Cfg::OUT;
+  uint8_t* in0 = smem + Sm::IN + warp * DEC_STAGES * Sm::STAGE;
+  uint8_t* orow = smem + Sm::OUT + warp * Cfg::OUT + lane * Cfg::OUT_ROW;
   const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
+  const int part = lane & (LPV - 1);
+  const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
 
   const int64_t n_tiles = (a.n + VPW - 1) / VPW;
   const int64_t gw = (int64_t)blockIdx.x * DEC_WARPS + warp;
   const int64_t n_warps = (int64_t)gridDim.x * DEC_WARPS;
-  constexpr int NORM_OFF = ((Cfg::TILE_P + 15) / 16) * 16;
+  constexpr int NORM_OFF = Cfg::PACK_BYTES;
 
   // Full tiles come through bulk copies; the last, partial tile (if any) is
   // read with plain loads (its byte count need not be a multiple of 16).
   auto full_tile = [&](int64_t tile) { return (tile + 1) * VPW <= a.n; };
-  auto issue = [&](int64_t tile, int stage) {
+  auto issue = [&](int64_t tile, int stage) {  // called by the whole warp
     if (!full_tile(tile)) return;
+    const uint32_t bar = smem_u32(&bars[stage]);
+    uint8_t* dst = in0 + stage * Sm::STAGE;
     if (lane == 0) {
-      const uint32_t bar = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(bar, (uint32_t)(Cfg::TILE_P + (a.norms_bulk ? VPW * 4 : 0)));
-      uint8_t* dst = in0 + stage * Cfg::IN_STAGE;
-      bulk_g2s(smem_u32(dst), a.packed + tile * Cfg::TILE_P, Cfg::TILE_P, bar);
       if (a.norms_bulk) bulk_g2s(smem_u32(dst + NORM_OFF), a.norms + tile * VPW, VPW * 4, bar);
+      if (!Cfg::ROWS) bulk_g2s(smem_u32(dst), a.packed + tile * Cfg::TILE_P, Cfg::TILE_P, bar);
     }
+    __syncwarp();
+    if (Cfg::ROWS)
+      bulk_g2s(smem_u32(dst + lane * Cfg::PROW), a.packed + tile * Cfg::TILE_P + (int64_t)lane * Cfg::PL, Cfg::PL,
+               bar);
   };
 
 #pragma unroll
@@ -131,7 +150,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     if (t < n_tiles) issue(t, s);
   }
 
-  const int half = lane & (LPV - 1);
   int stage = 0;
   uint32_t parity = 0;
   bool stored_once = false;
@@ -143,10 +161,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     uint32_t words[WL];
     float nrm = 0.f;
     if (full_tile(tile)) {
-      // every lane polls; the warp acts on one agreed outcome
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u,
-                                                             a.wait_limit));
-    if (!ok) {
+      const bool ok =
+          __all_sync(FULL, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.wait_limit));
+      if (!ok) {
         if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
 #pragma unroll
         for (int s = 1; s < DEC_STAGES; ++s) {
@@ -158,16 +175,31 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         return;
       }
       parity ^= 1u << stage;
-      const uint8_t* st = in0 + stage * Cfg::IN_STAGE;
-      const uint32_t* row = reinterpret_cast<const uint32_t*>(st + vl * P + half * Cfg::PL);
+      const uint8_t* st = in0 + stage * Sm::STAGE;
+      const uint8_t* row = st + lane * Cfg::PROW;
+      if (Cfg::PL % 16 == 0) {
 #pragma unroll
-      for (int w = 0; w < WL; ++w) words[w] = row[w];
+        for (int w = 0; w < WL / 4; ++w) {
+          const uint4 r = reinterpret_cast<const uint4*>(row)[w];
+          words[4 * w] = r.x;
+          words[4 * w + 1] = r.y;
+          words[4 * w + 2] = r.z;
+          words[4 * w + 3] = r.w;
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < WL / 2; ++w) {
+          const uint2 r = reinterpret_cast<const uint2*>(row)[w];
+          words[2 * w] = r.x;
+          words[2 * w + 1] = r.y;
+        }
+      }
       nrm = a.norms_bulk ? reinterpret_cast<const float*>(st + NORM_OFF)[vl] : __ldg(a.norms + v0 + vl);
     } else {
 #pragma unroll
       for (int w = 0; w < WL; ++w) words[w] = 0;
       if (active) {
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(a.packed + (v0 + vl) * P + half * Cfg::PL);
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(a.packed + v0 * Cfg::P) + lane * WL;
 #pragma unroll
         for (int w = 0; w < WL; ++w) words[w] = __ldg(row + w);
         nrm = __ldg(a.norms + v0 + vl);
@@ -192,42 +224,43 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
       v[j] = lds_f2(f * 256u + lut_lane);
     }
     wht_pairs<NP>(v);
-    if (LPV == 2) {
-      const f2 sg = half ? f2{-1.f, -1.f} : f2{1.f, 1.f};
+#pragma unroll
+    for (int m = 1; m < LPV; m <<= 1) {
+      const f2 sg = (part & m) ? make_float2(-1.f, -1.f) : make_float2(1.f, 1.f);
 #pragma unroll
       for (int k = 0; k < NP; ++k) {
         f2 o;
-        o.x = __shfl_xor_sync(FULL, v[k].x, 1);
-        o.y = __shfl_xor_sync(FULL, v[k].y, 1);
+        o.x = __shfl_xor_sync(FULL, v[k].x, m);
+        o.y = __shfl_xor_sync(FULL, v[k].y, m);
         v[k] = fma2(v[k], sg, o);
       }
     }
 
     // ---- scale by N/d, round to fp16, apply the signs, stage the row
     const float sc = nrm * (1.0f / (float)D);
-    const f2 sc2 = {sc, sc};
-    // the previous bulk store from this warp's staging rows must have read them
+    const f2 sc2 = make_float2(sc, sc);
+    // the previous bulk store from this lane's staging row must have read it
     if (stored_once) bulk_wait_read<0>();
-    __syncwarp();
-    uint8_t* orow = out_rows + lane * Cfg::OUT_ROW;
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
+      uint4 mk;
+      if (LPV == 1)
+        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
+      else
+        mk = my_masks[c];
+      const uint32_t m4[4] = {mk.x, mk.y, mk.z, mk.w};
       uint32_t h[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int k = 4 * c + q;
-        const f2 y = mul2(v[k], sc2);
+        const f2 y = mul2(v[4 * c + q], sc2);
         const __half2 hv = __floats2half2_rn(y.x, y.y);
-        uint32_t mask = T.sign_h2[k];
-        if (LPV == 2) mask = half ? T.sign_h2[NP + k] : T.sign_h2[k];
-        h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ mask;
+        h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ m4[q];
       }
       *reinterpret_cast<uint4*>(orow + 16 * c) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     fence_proxy_async_smem();
-    __syncwarp();
     if (active) {
-      __half* dst = a.x + (v0 + vl) * D + half * C;
+      __half* dst = a.x + (v0 + vl) * D + part * C;
       bulk_s2g(dst, smem_u32(orow), 2 * C);
       bulk_commit();
       stored_once = true;

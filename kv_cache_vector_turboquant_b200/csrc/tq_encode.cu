@@ -8,15 +8,16 @@
 // indices packed little-endian, b bits each.
 //
 // B200 mapping:
-//  * one vector per lane (d <= 128) or per lane pair (d = 256); a warp owns a
+//  * every lane owns 64 coordinates of one vector (1, 2 or 4 lanes per vector
+//    for d = 64, 128, 256), so a CTA of 16 warps fits one SM; a warp owns a
 //    tile of 32 lane-rows and runs its own 2-stage pipeline: each lane issues
-//    one 1-D bulk copy (TMA) of its row into a padded shared-memory row, so
-//    the 128-bit shared loads that follow are free of bank conflicts;
-//  * the sign flip is an XOR of fp16 sign bits with masks held in the kernel
-//    parameters (constant bank, warp-uniform: every lane holds the same
-//    coordinates of a different vector);
-//  * the Walsh-Hadamard transform runs in registers with packed f32x2
-//    add/sub (one cross-lane shuffle stage for d = 256);
+//    one 1-D bulk copy (TMA) of its 128 bytes into a shared row padded to 144
+//    bytes, so the 128-bit shared loads that follow hit distinct bank groups;
+//  * the sign flip is an XOR of fp16 sign bits (masks from the constant bank
+//    when all lanes hold the same coordinates, else from shared memory),
+//    fused with the first butterfly stage at the fp16 -> f32 conversion;
+//  * the other Walsh-Hadamard stages run in registers with packed f32x2
+//    add/sub, then one or two shuffle stages across the lanes of a vector;
 //  * nearest level: q = w * (1 / (delta N)) + offset is floored through the
 //    2^23 round-down trick into a cell of a lane-replicated shared table that
 //    holds the one boundary inside the cell; one compare gives the index;
@@ -34,22 +35,23 @@
 
 namespace tq {
 
-constexpr int ENC_WARPS = 8;
+constexpr int ENC_WARPS = 16;
 constexpr int ENC_STAGES = 2;
+constexpr int ENC_C = 64;  // coordinates per lane
 constexpr float MAGIC_2P23 = 8388608.0f;
 
 template <int D, int BITS>
 struct EncCfg {
-  static constexpr int LPV = D > 128 ? 2 : 1;  // lanes per vector
-  static constexpr int C = D / LPV;            // coordinates per lane
-  static constexpr int NP = C / 2;             // f32x2 pairs per lane
-  static constexpr int VPW = 32 / LPV;         // vectors per warp tile
-  static constexpr int P = D * BITS / 8;       // packed bytes per vector
-  static constexpr int WL = P / LPV / 4;       // packed 32-bit words per lane
-  static constexpr int IN_ROW = 2 * C + 16;    // bytes per padded input lane-row
-  static constexpr int OUT_ROW = WL + 1;       // words per padded output lane-row (odd)
+  static constexpr int C = ENC_C;
+  static constexpr int LPV = D / C;         // lanes per vector
+  static constexpr int NP = C / 2;          // f32x2 pairs per lane
+  static constexpr int VPW = 32 / LPV;      // vectors per warp tile
+  static constexpr int P = D * BITS / 8;    // packed bytes per vector
+  static constexpr int WL = C * BITS / 32;  // packed 32-bit words per lane
+  static constexpr int IN_ROW = 2 * C + 16;  // padded input lane-row: 9 x 16 B
+  static constexpr int OUT_ROW = WL + 1;     // padded output lane-row, odd words
   static constexpr int L = 1 << BITS;
-  static constexpr int GROUPS = C / 32;        // guard groups of 32 coordinates
+  static constexpr int GROUPS = C / 32;  // guard groups of 32 coordinates
   static constexpr int IN_STAGE = 32 * IN_ROW;
   static constexpr int OUT_WORDS = 32 * OUT_ROW;
 };
@@ -71,11 +73,12 @@ struct EncArgs {
 template <int D, int BITS>
 struct EncSmem {
   using Cfg = EncCfg<D, BITS>;
-  static constexpr int BAR = 0;                                          // ENC_WARPS*ENC_STAGES u64
-  static constexpr int SCR = 128;                                        // per warp C floats scratch
-  static constexpr int IN = SCR + ENC_WARPS * Cfg::C * 4;                // input stages
+  static constexpr int BAR = 0;                                            // warps x stages u64
+  static constexpr int MASK = 256;                                         // sign masks, LPV x 32 u32
+  static constexpr int SCR = MASK + 4 * 32 * 4;                            // per warp 32-float scratch
+  static constexpr int IN = SCR + ENC_WARPS * 32 * 4;                      // input stages
   static constexpr int OUT = IN + ENC_WARPS * ENC_STAGES * Cfg::IN_STAGE;  // output rows
-  static constexpr int LUT = OUT + ENC_WARPS * Cfg::OUT_WORDS * 4;         // cell table
+  static constexpr int LUT = OUT + ENC_WARPS * Cfg::OUT_WORDS * 4;          // cell table
   static size_t bytes(int cells) { return (size_t)LUT + (size_t)cells * 32 * 8; }
 };
 
@@ -85,18 +88,26 @@ TQ_DEV uint2 lds_u2(uint32_t addr) {
   return r;
 }
 
+// Pack code m (< 2^BITS) of coordinate i into the lane's word array.
+template <int BITS, int WL>
+TQ_DEV void put_code(uint32_t (&words)[WL], int i, uint32_t m) {
+  const int off = i * BITS;
+  words[off >> 5] |= m << (off & 31);
+  if ((off & 31) + BITS > 32) words[(off >> 5) + 1] |= m >> (32 - (off & 31));
+}
+
+
 template <int D, int BITS>
 __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     encode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ EncArgs a) {
   using Cfg = EncCfg<D, BITS>;
   using Sm = EncSmem<D, BITS>;
-  constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, VPW = Cfg::VPW, WL = Cfg::WL;
-  constexpr int L = Cfg::L;
+  constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, VPW = Cfg::VPW, WL = Cfg::WL, L = Cfg::L;
+  constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t FULL = 0xffffffffu;
 
   // ---- lane-replicated cell table: entry (cell, lane) = {boundary bits, count below}
   {
@@ -117,6 +128,8 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       lut[e] = make_uint2(__float_as_uint(thr), below);
     }
   }
+  uint32_t* smask = reinterpret_cast<uint32_t*>(smem + Sm::MASK);
+  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) smask[i] = T.sign_h2[i];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::BAR) + warp * ENC_STAGES;
   if (lane == 0) {
 #pragma unroll
@@ -127,17 +140,18 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
 
   uint8_t* in_stage0 = smem + Sm::IN + warp * ENC_STAGES * Cfg::IN_STAGE;
   uint32_t* out_rows = reinterpret_cast<uint32_t*>(smem + Sm::OUT) + warp * Cfg::OUT_WORDS;
-  float* scratch = reinterpret_cast<float*>(smem + Sm::SCR) + warp * C;
+  float* scratch = reinterpret_cast<float*>(smem + Sm::SCR) + warp * 32;
   const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
+  const int part = lane & (LPV - 1);  // which 64-coordinate part of its vector this lane holds
+  const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
 
   const int64_t n_tiles = (a.n + VPW - 1) / VPW;
   const int64_t gw = (int64_t)blockIdx.x * ENC_WARPS + warp;
   const int64_t n_warps = (int64_t)gridDim.x * ENC_WARPS;
 
-  auto issue = [&](int64_t tile, int stage) {
+  auto issue = [&](int64_t tile, int stage) {  // called by the whole warp
     const int64_t v0 = tile * VPW;
-    const int valid = (int)min64(VPW, a.n - v0);
-    const int valid_lanes = valid * LPV;
+    const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
     const uint32_t bar = smem_u32(&bars[stage]);
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(valid_lanes * 2 * C));
     __syncwarp();
@@ -156,7 +170,6 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
   const float Rscale = T.inv_delta;
   const float qoff = T.q_offset;
   const float gq = T.guard_q;
-  const int half = lane & (LPV - 1);  // which half of the vector (d = 256)
 
   int stage = 0;
   uint32_t parity = 0;  // bit s: parity of the next completion of stage s
@@ -164,12 +177,10 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     const int64_t v0 = tile * VPW;
     const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
     // every lane polls; the warp acts on one agreed outcome
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u,
-                                                             a.wait_limit));
+    const bool ok = __all_sync(FULL, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.wait_limit));
     if (!ok) {
       if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
-      // Give the copies already issued into the other stages a bounded time
-      // to land before the CTA leaves.
+      // give the copies already issued into the other stage a bounded time to land
 #pragma unroll
       for (int s = 1; s < ENC_STAGES; ++s) {
         const int os = (stage + s) % ENC_STAGES;
@@ -188,97 +199,89 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     for (int c = 0; c < C / 8; ++c) {
       uint4 r = make_uint4(0, 0, 0, 0);
       if (active) r = *reinterpret_cast<const uint4*>(my_row + 16 * c);
-      const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+      uint4 mk;
+      if (LPV == 1)
+        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
+      else
+        mk = my_masks[c];
+      const uint32_t w4[4] = {r.x ^ mk.x, r.y ^ mk.y, r.z ^ mk.z, r.w ^ mk.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int k = 4 * c + q;  // pair index within the lane
-        uint32_t mask = T.sign_h2[k];
-        if (LPV == 2) mask = half ? T.sign_h2[NP + k] : T.sign_h2[k];
-        const uint32_t hw = w4[q] ^ mask;
-        const float lo = __half2float(__ushort_as_half((unsigned short)(hw & 0xffffu)));
-        const float hi = __half2float(__ushort_as_half((unsigned short)(hw >> 16)));
-        v[k].x = lo + hi;
-        v[k].y = lo - hi;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[q]));
+        v[4 * c + q] = make_float2(f.x + f.y, f.x - f.y);
       }
     }
     // ---- sum of squares: (x0+x1)^2 + (x0-x1)^2 = 2 (x0^2 + x1^2); 8 chains
-    f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+    f2 acc[4];
 #pragma unroll
-    for (int k = 0; k < NP; ++k) acc[k & 3] = fma2(v[k], v[k], acc[k & 3]);
-    const f2 s01 = add2(acc[0], acc[1]);
-    const f2 s23 = add2(acc[2], acc[3]);
-    const f2 s4 = add2(s01, s23);
+    for (int j = 0; j < 4; ++j) acc[j] = mul2(v[j], v[j]);
+#pragma unroll
+    for (int k = 4; k < NP; ++k) acc[k & 3] = fma2(v[k], v[k], acc[k & 3]);
+    const f2 s4 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
     float sum2 = s4.x + s4.y;
-    if (LPV == 2) sum2 += __shfl_xor_sync(FULL, sum2, 1);
+#pragma unroll
+    for (int m = 1; m < LPV; m <<= 1) sum2 += __shfl_xor_sync(FULL, sum2, m);
     const float nrm = sqrtf(0.5f * sum2);
 
-    // ---- remaining Walsh-Hadamard stages
+    // ---- remaining Walsh-Hadamard stages: in registers, then across the lanes of the vector
     wht_pairs<NP>(v);
-    if (LPV == 2) {
-      const f2 sg = half ? f2{-1.f, -1.f} : f2{1.f, 1.f};
+#pragma unroll
+    for (int m = 1; m < LPV; m <<= 1) {
+      const f2 sg = (part & m) ? make_float2(-1.f, -1.f) : make_float2(1.f, 1.f);
 #pragma unroll
       for (int k = 0; k < NP; ++k) {
         f2 o;
-        o.x = __shfl_xor_sync(FULL, v[k].x, 1);
-        o.y = __shfl_xor_sync(FULL, v[k].y, 1);
+        o.x = __shfl_xor_sync(FULL, v[k].x, m);
+        o.y = __shfl_xor_sync(FULL, v[k].y, m);
         v[k] = fma2(v[k], sg, o);
       }
     }
 
     // ---- quantize + pack
-    const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite
+    const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite vector
     const float R = special ? 0.f : __fdiv_rn(Rscale, nrm);
     uint32_t words[WL];
 #pragma unroll
     for (int w = 0; w < WL; ++w) words[w] = 0;
     uint32_t gmask = 0;
     if (!special) {
-      const f2 R2 = {R, R}, Q2 = {qoff, qoff}, M2 = {MAGIC_2P23, MAGIC_2P23};
+      const f2 R2 = make_float2(R, R), Q2 = make_float2(qoff, qoff), M2 = make_float2(MAGIC_2P23, MAGIC_2P23);
 #pragma unroll
       for (int g = 0; g < Cfg::GROUPS; ++g) {
-        bool gflag = false;
+        float gmin = 3.0e38f;  // closest approach to a boundary in this group (q units)
 #pragma unroll
         for (int k = g * 16; k < g * 16 + 16; ++k) {
           const f2 q2 = fma2(v[k], R2, Q2);
           const f2 qm = add2_rm(q2, M2);
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int i = 2 * k + e;
             const float q = e ? q2.y : q2.x;
             const uint32_t qb = __float_as_uint(e ? qm.y : qm.x);
             const uint2 ent = lds_u2(qb * 256u + lut_lane);
             const float dl = __uint_as_float(ent.x) - q;
-            const uint32_t m = ent.y + (__float_as_uint(dl) >> 31);
-            gflag |= fabsf(dl) < gq;
-            const int off = i * BITS;
-            words[off >> 5] |= m << (off & 31);
-            if ((off & 31) + BITS > 32) words[(off >> 5) + 1] |= m >> (32 - (off & 31));
+            gmin = fminf(gmin, fabsf(dl));
+            put_code<BITS>(words, 2 * k + e, ent.y + (__float_as_uint(dl) >> 31));
           }
         }
-        gmask |= gflag ? (1u << g) : 0u;
+        gmask |= (gmin < gq) ? (1u << g) : 0u;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < C; ++i) {
-        const int off = i * BITS;
-        const uint32_t m = L / 2;
-        words[off >> 5] |= m << (off & 31);
-        if ((off & 31) + BITS > 32) words[(off >> 5) + 1] |= m >> (32 - (off & 31));
-      }
+      for (int i = 0; i < C; ++i) put_code<BITS>(words, i, (uint32_t)(L / 2));
     }
     if (!active) gmask = 0;
 #pragma unroll
     for (int w = 0; w < WL; ++w) out_rows[lane * Cfg::OUT_ROW + w] = words[w];
 
-    // ---- exact recheck of coordinates inside the guard band (rare)
+    // ---- exact recheck of the coordinates inside the guard band (rare)
     uint32_t any = __ballot_sync(FULL, gmask != 0);
     while (any) {
       const int src = __ffs(any) - 1;
       any &= any - 1;
       uint32_t sg = __shfl_sync(FULL, gmask, src);
       const float srcR = __shfl_sync(FULL, R, src);
-      const int src_half = src & (LPV - 1);
-      const int vec_lane0 = src - src_half;
+      const int src_part = src & (LPV - 1);
+      const int vec_lane0 = src - src_part;
       while (sg) {
         const int g = __ffs(sg) - 1;
         sg &= sg - 1;
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
         __syncwarp();
         const float wj = scratch[lane];
         __syncwarp();
-        // same f32 arithmetic as the main pass -> the same flag
+        // the same f32 arithmetic as the main pass gives the same flags
         const float q = fmaf(wj, srcR, qoff);
         const uint32_t qb = __float_as_uint(__fadd_rd(q, MAGIC_2P23));
         const uint2 ent = lds_u2(qb * 256u + lut_lane);
@@ -306,29 +309,29 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
           const int j = __ffs(cm) - 1;
           cm &= cm - 1;
           const int i_local = g * 32 + j;
-          const int gi = src_half * C + i_local;  // coordinate index in the vector
-          // w_gi = sum_k s_k (-1)^popcount(gi & k) x_k, exact in fp64
-          double part = 0.0, sq = 0.0;
+          const int gi = src_part * C + i_local;  // coordinate index in the vector
+          // w_gi = sum_k s_k (-1)^popcount(gi & k) x_k: exact in fp64 for fp16 x
+          double part_sum = 0.0, sq = 0.0;
 #pragma unroll
           for (int t = 0; t < D / 32; ++t) {
             const int kk = lane + 32 * t;
             const __half hx = reinterpret_cast<const __half*>(
                 in_stage0 + stage * Cfg::IN_STAGE + (vec_lane0 + kk / C) * Cfg::IN_ROW)[kk % C];
             const double xk = (double)__half2float(hx);
-            const uint32_t sbit = (T.sign_h2[kk >> 1] >> (15 + 16 * (kk & 1))) & 1u;
+            const uint32_t sbit = (smask[kk >> 1] >> (15 + 16 * (kk & 1))) & 1u;
             const uint32_t neg = sbit ^ (uint32_t)(__popc(gi & kk) & 1);
-            part += neg ? -xk : xk;
+            part_sum += neg ? -xk : xk;
             sq = fma(xk, xk, sq);
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
-            part += __shfl_xor_sync(FULL, part, o);
+            part_sum += __shfl_xor_sync(FULL, part_sum, o);
             sq += __shfl_xor_sync(FULL, sq, o);
           }
           const double n64 = sqrt(sq);
           uint32_t m = 0;
 #pragma unroll
-          for (int jj = 0; jj < L - 1; ++jj) m += (part >= (double)T.bounds[jj] * n64) ? 1u : 0u;
+          for (int jj = 0; jj < L - 1; ++jj) m += (part_sum >= (double)T.bounds[jj] * n64) ? 1u : 0u;
           if (lane == 0) {
             const int off = i_local * BITS;
             uint32_t* row = out_rows + src * Cfg::OUT_ROW;
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed) + v0 * (Cfg::P / 4);
       const int total = valid_lanes * WL;
       for (int w = lane; w < total; w += 32) dst[w] = out_rows[(w / WL) * Cfg::OUT_ROW + (w % WL)];
-      if (active && half == 0) a.norms[v0 + lane / LPV] = nrm;
+      if (active && part == 0) a.norms[v0 + lane / LPV] = nrm;
     } else if (active) {
       const int64_t r = v0 + lane / LPV;
       const int64_t seq = r / a.h;
@@ -357,11 +360,11 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       const int32_t s = a.slot[seq];
       if (s >= 0 && s < a.s_max) {
         const int64_t drow = (seq * a.s_max + s) * a.h + head;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + drow * Cfg::P) + half * WL;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + drow * Cfg::P) + part * WL;
 #pragma unroll
         for (int w = 0; w < WL; ++w) dst[w] = out_rows[lane * Cfg::OUT_ROW + w];
-        if (half == 0) a.norms[drow] = nrm;
-      } else if (half == 0) {
+        if (part == 0) a.norms[drow] = nrm;
+      } else if (part == 0) {
         record_error(a.err, TQ_DEVERR_SLOT_RANGE);
       }
     }
@@ -388,10 +391,9 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, const EncArgs& a, c
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  const int sms = tq_sm_count(dev);
   const int64_t tiles = (a.n + Cfg::VPW - 1) / Cfg::VPW;
   const int64_t ctas_needed = (tiles + ENC_WARPS - 1) / ENC_WARPS;
-  const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)sms);
+  const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)tq_sm_count(dev));
   encode_kernel<D, BITS><<<grid, ENC_WARPS * 32, smem, st>>>(T, a);
   return cudaGetLastError();
 }

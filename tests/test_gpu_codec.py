@@ -127,12 +127,15 @@ def test_llama_layer_full_size_sampled(K, W, bits):
         assert code_mismatches(gp, det, bits, 128) == 0
         assert_norms(gn, det)
         assert_decode_ulp(dec[rows.cuda()].cpu().numpy(), O.decode(gp, gn, bits, 42, 128))
-        # whole-tensor property: unit-direction distortion equals the sphere marginal
-        u = flat.float() / flat.float().norm(dim=1, keepdim=True)
-        uh = dec.float() / norms[:, None]
-        mse = ((u - uh) ** 2).sum(dim=1).mean().item()
-        want = O.sphere_marginal_mse(O.format_levels(bits), 128)
-        assert abs(mse - want) / want < 0.01, (mse, want)
+        # whole-tensor property for the isotropic tensor (V: iid N(0,1), so the
+        # unit direction is uniform on the sphere): the distortion equals the
+        # sphere-marginal value. K's fixed outlier channels break isotropy.
+        if x is v:
+            u = flat.float() / flat.float().norm(dim=1, keepdim=True)
+            uh = dec.float() / norms[:, None]
+            mse = ((u - uh) ** 2).sum(dim=1).mean().item()
+            want = O.sphere_marginal_mse(O.format_levels(bits), 128)
+            assert abs(mse - want) / want < 0.01, (mse, want)
         del packed, norms, dec
     assert K.tq_device_error()[0] == K.TQ_OK
 
