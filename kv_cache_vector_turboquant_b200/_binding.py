@@ -5,7 +5,7 @@ CUDA stream to a handle, calls the C entry point of the same name and turns a
 non-zero status into :class:`TQError`. All computation happens in the CUDA
 kernels of ``libtq.so``; there is no fallback path. Importing this module
 raises ``ImportError`` if the library has not been built
-(``python -m kv_cache_vector_turboquant_b200.build``).
+(``python kv_cache_vector_turboquant_b200/build.py``).
 """
 
 from __future__ import annotations
@@ -17,7 +17,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtq.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
         f"libtq.so not found at {_LIB_PATH}; build it with "
-        "`python -m kv_cache_vector_turboquant_b200.build`"
+        "`python kv_cache_vector_turboquant_b200/build.py`"
     )
 _lib = ctypes.CDLL(_LIB_PATH)
 

@@ -1,6 +1,7 @@
 """Build libtq.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m kv_cache_vector_turboquant_b200.build [--force] [-j N]``.
+Usage: ``python kv_cache_vector_turboquant_b200/build.py [--force] [-j N]`` (run as a
+script: importing the package would load the library being built).
 Objects go to ``_build/`` at the repository root; the shared library is
 written next to this file. CUDA runtime is linked statically so the library
 does not depend on the runtime version that torch ships.
