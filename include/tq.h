@@ -178,6 +178,35 @@ tq_status tq_attend_decode(const tq_ctx* k, const tq_ctx* v, const void* q_f16, 
                            void* workspace, size_t ws_bytes, tq_stream stream);
 
 /*
+ * No counterpart in the paper: an addition of this library.
+ *
+ * tq_attend_decode for callers that cannot allocate device memory -- for
+ * example a plugin inside a serving framework that owns every byte of device
+ * memory through its own pool, or a decode loop that must not risk a
+ * device-synchronising or failing cudaMalloc in the middle of a generation.
+ * Same arguments, layouts, alignment rules and results as tq_attend_decode,
+ * without the workspace: the split-S scratch is a fixed array of
+ * TQ_ATTEND_STATIC_SCRATCH_BYTES in device memory that belongs to the
+ * library (one per device that loads it, kept until the process exits). The
+ * call allocates nothing.
+ *  - Returns TQ_ERR_WORKSPACE, without enqueuing anything, when the scratch
+ *    this call needs, tq_attend_workspace_bytes(B, hq, head_dim, s_max), is
+ *    larger than TQ_ATTEND_STATIC_SCRATCH_BYTES.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (with the device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array, and the array keeps what
+ *    the last call left there (each call overwrites every entry it reads).
+ *    Calls that overlap on the GPU -- on different streams, or from host
+ *    threads that do not order their streams -- race on it.
+ */
+#define TQ_ATTEND_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+tq_status tq_attend_decode_static(const tq_ctx* k, const tq_ctx* v, const void* q_f16, int B, int hq, int hkv,
+                                  const void* k_packed, const float* k_norms, const void* v_packed,
+                                  const float* v_norms, int64_t s_max, const int32_t* positions, void* out_f16,
+                                  tq_stream stream);
+
+/*
  * Read and clear the device error word of the current device (a bitwise OR
  * of TQ_DEVERR_* set by kernels since the last call). Synchronises `stream`.
  * Returns TQ_ERR_TIMEOUT if TQ_DEVERR_TIMEOUT was set, TQ_ERR_DEVICE if

@@ -26,7 +26,9 @@ from ._binding import (  # noqa: F401
     TQ_OK,
     Ctx,
     TQError,
+    TQ_ATTEND_STATIC_SCRATCH_BYTES,
     tq_attend_decode,
+    tq_attend_decode_static,
     tq_attend_workspace_bytes,
     tq_create,
     tq_decode,

@@ -38,6 +38,8 @@ _PROTOS = {
     "tq_attend_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64]),
     "tq_attend_decode": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64,
                                   _vp, _vp, _vp, _c_size, _vp]),
+    "tq_attend_decode_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64,
+                                         _vp, _vp, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
 }
@@ -170,6 +172,18 @@ def tq_attend_decode(k: Ctx, v: Ctx, q, B: int, hq: int, hkv: int, k_packed, k_n
     _check(_lib.tq_attend_decode(k.handle, v.handle, _ptr(q), int(B), int(hq), int(hkv), _ptr(k_packed),
                                  _ptr(k_norms), _ptr(v_packed), _ptr(v_norms), int(s_max), _ptr(positions),
                                  _ptr(out), _ptr(workspace), int(ws_bytes), _stream(stream)), "tq_attend_decode")
+
+
+def tq_attend_decode_static(k: Ctx, v: Ctx, q, B: int, hq: int, hkv: int, k_packed, k_norms, v_packed, v_norms,
+                            s_max: int, positions, out, stream=None) -> None:
+    """tq_attend_decode without a workspace argument: the library's own fixed
+    device scratch is used, so the call allocates nothing."""
+    _check(_lib.tq_attend_decode_static(k.handle, v.handle, _ptr(q), int(B), int(hq), int(hkv), _ptr(k_packed),
+                                        _ptr(k_norms), _ptr(v_packed), _ptr(v_norms), int(s_max), _ptr(positions),
+                                        _ptr(out), _stream(stream)), "tq_attend_decode_static")
+
+
+TQ_ATTEND_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 def tq_device_error(stream=None) -> tuple[int, int]:
