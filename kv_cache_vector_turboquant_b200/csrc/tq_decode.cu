@@ -11,13 +11,16 @@
 //
 // B200 mapping: every lane owns 64 coordinates (1, 2 or 4 lanes per vector),
 // 16 warps per SM. Each warp runs a 3-stage pipeline of 1-D bulk copies (TMA)
-// bringing its tile of packed rows and norms into shared memory (row layout
-// chosen so the 64/128-bit shared reads are conflict-free); a lane-replicated
-// table indexed by two codes returns (c[a] + c[b], c[a] - c[b]), the levels
-// already through the first butterfly; the other stages run in registers with
-// f32x2 add/sub and shuffles across the lanes of a vector; the fp16 rows are
-// staged in padded shared rows and leave through per-row 1-D bulk stores
-// (TMA), so every DRAM write is a full line.
+// bringing its tile of packed rows and norms into shared memory (one copy each
+// per tile); a lane-replicated table indexed by two codes returns
+// (c[a] + c[b], c[a] - c[b]), the levels already through the first
+// butterfly; the other stages run in registers with f32x2 add/sub and
+// shuffles across the lanes of a vector. The lane negates the levels of the
+// chunks j with popcount(j & s) odd (mirroring their codes, the codebook is
+// symmetric), which makes the transform deliver natural chunk c ^ s in
+// register slot c; so its 16-byte stores into the warp's 4 KB output tile are
+// free of bank conflicts while the tile itself is in natural order and leaves
+// through one 1-D bulk store (TMA) per tile.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -42,15 +45,9 @@ struct DecCfg {
   static constexpr int WL = PL / 4;
   static constexpr int E = 1 << (2 * BITS);  // pair-table entries
   static constexpr int TILE_P = 32 * PL;     // packed bytes of a full tile
-  // 32-byte lane rows (4 bits) are copied one per lane into 48-byte rows so
-  // the 128-bit reads are conflict-free; 16- and 24-byte rows are read
-  // conflict-free straight from the contiguous tile.
-  static constexpr bool ROWS = (PL == 32);
-  static constexpr int PROW = ROWS ? 48 : PL;
-  static constexpr int PACK_BYTES = 32 * PROW;
+  static constexpr int PACK_BYTES = TILE_P;   // lane rows contiguous, as in memory
   static constexpr int IN_STAGE = PACK_BYTES + VPW * 4;  // packed rows + norms
-  static constexpr int OUT_ROW = 2 * C + 16;              // padded fp16 lane-row
-  static constexpr int OUT = 32 * OUT_ROW;
+  static constexpr int OUT = 32 * 2 * C;                  // the warp's output tile (4 KB)
 };
 
 template <int D, int BITS>
@@ -116,10 +113,29 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   __syncthreads();
 
   uint8_t* in0 = smem + Sm::IN + warp * DEC_STAGES * Sm::STAGE;
-  uint8_t* orow = smem + Sm::OUT + warp * Cfg::OUT + lane * Cfg::OUT_ROW;
+  uint8_t* otile = smem + Sm::OUT + warp * Cfg::OUT;
+  uint8_t* orow = otile + lane * 2 * C;
   const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
   const int part = lane & (LPV - 1);
   const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
+  // chunk swizzle (shared by the lanes of a vector) and the code bits to
+  // mirror so that register slot c receives natural output chunk c ^ swz
+  const uint32_t swz = (uint32_t)(lane / LPV) & 7u;
+  uint32_t flipw[WL];
+#pragma unroll
+  for (int w = 0; w < WL; ++w) flipw[w] = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (__popc((uint32_t)j & swz) & 1) {
+#pragma unroll
+      for (int i = 8 * j; i < 8 * j + 8; ++i) {
+        const int off = i * BITS;
+        const uint32_t m = (1u << BITS) - 1u;
+        flipw[off >> 5] |= m << (off & 31);
+        if ((off & 31) + BITS > 32) flipw[(off >> 5) + 1] |= m >> (32 - (off & 31));
+      }
+    }
+  }
 
   const int64_t n_tiles = (a.n + VPW - 1) / VPW;
   const int64_t gw = (int64_t)blockIdx.x * DEC_WARPS + warp;
@@ -136,12 +152,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(bar, (uint32_t)(Cfg::TILE_P + (a.norms_bulk ? VPW * 4 : 0)));
       if (a.norms_bulk) bulk_g2s(smem_u32(dst + NORM_OFF), a.norms + tile * VPW, VPW * 4, bar);
-      if (!Cfg::ROWS) bulk_g2s(smem_u32(dst), a.packed + tile * Cfg::TILE_P, Cfg::TILE_P, bar);
+      bulk_g2s(smem_u32(dst), a.packed + tile * Cfg::TILE_P, Cfg::TILE_P, bar);
     }
     __syncwarp();
-    if (Cfg::ROWS)
-      bulk_g2s(smem_u32(dst + lane * Cfg::PROW), a.packed + tile * Cfg::TILE_P + (int64_t)lane * Cfg::PL, Cfg::PL,
-               bar);
   };
 
 #pragma unroll
@@ -171,12 +184,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
           if (tile + s * n_warps < n_tiles && full_tile(tile + s * n_warps))
             (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
         }
-        bulk_wait_all<0>();
+        if (lane == 0) bulk_wait_all<0>();
         return;
       }
       parity ^= 1u << stage;
       const uint8_t* st = in0 + stage * Sm::STAGE;
-      const uint8_t* row = st + lane * Cfg::PROW;
+      const uint8_t* row = st + lane * Cfg::PL;
       if (Cfg::PL % 16 == 0) {
 #pragma unroll
         for (int w = 0; w < WL / 4; ++w) {
@@ -205,6 +218,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         nrm = __ldg(a.norms + v0 + vl);
       }
     }
+#pragma unroll
+    for (int w = 0; w < WL; ++w) words[w] ^= flipw[w];
     __syncwarp();
     // the stage has been read into registers: refill it
     {
@@ -236,18 +251,16 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
       }
     }
 
-    // ---- scale by N/d, round to fp16, apply the signs, stage the row
+    // ---- scale by N/d, round to fp16, apply the signs, stage the tile
     const float sc = nrm * (1.0f / (float)D);
     const f2 sc2 = make_float2(sc, sc);
-    // the previous bulk store from this lane's staging row must have read it
-    if (stored_once) bulk_wait_read<0>();
+    // the previous tile's bulk store must have finished reading the buffer
+    if (lane == 0 && stored_once) bulk_wait_read<0>();
+    __syncwarp();
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
-      uint4 mk;
-      if (LPV == 1)
-        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
-      else
-        mk = my_masks[c];
+      const uint32_t ch = (uint32_t)c ^ swz;  // natural chunk held in slot c
+      const uint4 mk = my_masks[ch];
       const uint32_t m4[4] = {mk.x, mk.y, mk.z, mk.w};
       uint32_t h[4];
 #pragma unroll
@@ -256,18 +269,18 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         const __half2 hv = __floats2half2_rn(y.x, y.y);
         h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ m4[q];
       }
-      *reinterpret_cast<uint4*>(orow + 16 * c) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4*>(orow + 16 * ch) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     fence_proxy_async_smem();
-    if (active) {
-      __half* dst = a.x + (v0 + vl) * D + part * C;
-      bulk_s2g(dst, smem_u32(orow), 2 * C);
+    __syncwarp();
+    if (lane == 0) {
+      bulk_s2g(a.x + v0 * D, smem_u32(otile), (uint32_t)(valid_lanes * 2 * C));
       bulk_commit();
       stored_once = true;
     }
     if (++stage == DEC_STAGES) stage = 0;
   }
-  bulk_wait_all<0>();
+  if (lane == 0) bulk_wait_all<0>();
 }
 
 template <int D, int BITS>

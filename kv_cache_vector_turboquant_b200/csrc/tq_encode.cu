@@ -10,12 +10,17 @@
 // B200 mapping:
 //  * every lane owns 64 coordinates of one vector (1, 2 or 4 lanes per vector
 //    for d = 64, 128, 256), so a CTA of 16 warps fits one SM; a warp owns a
-//    tile of 32 lane-rows and runs its own 2-stage pipeline: each lane issues
-//    one 1-D bulk copy (TMA) of its 128 bytes into a shared row padded to 144
-//    bytes, so the 128-bit shared loads that follow hit distinct bank groups;
-//  * the sign flip is an XOR of fp16 sign bits (masks from the constant bank
-//    when all lanes hold the same coordinates, else from shared memory),
-//    fused with the first butterfly stage at the fp16 -> f32 conversion;
+//    tile of 32 lane-rows (4 KB, contiguous in memory) and runs its own
+//    2-stage pipeline of one 1-D bulk copy (TMA) per tile;
+//  * a lane reads its 16-byte chunk c ^ s into register slot c (s = a few bits
+//    of its vector index), which spreads a quarter-warp's 128-bit shared loads
+//    over distinct bank groups. Permuting the input of a Walsh-Hadamard
+//    transform by XOR with s only multiplies output i by (-1)^popcount(i & s),
+//    so the transform runs unchanged and the affected codes are mirrored
+//    (code -> 2^b - 1 - code, the codebook is symmetric) by one XOR per word;
+//  * the sign flip is an XOR of fp16 sign bits (masks from shared memory, in
+//    the lane's chunk order), fused with the first butterfly stage at the
+//    fp16 -> f32 conversion;
 //  * the other Walsh-Hadamard stages run in registers with packed f32x2
 //    add/sub, then one or two shuffle stages across the lanes of a vector;
 //  * nearest level: q = w * (1 / (delta N)) + offset is floored through the
@@ -48,7 +53,7 @@ struct EncCfg {
   static constexpr int VPW = 32 / LPV;      // vectors per warp tile
   static constexpr int P = D * BITS / 8;    // packed bytes per vector
   static constexpr int WL = C * BITS / 32;  // packed 32-bit words per lane
-  static constexpr int IN_ROW = 2 * C + 16;  // padded input lane-row: 9 x 16 B
+  static constexpr int IN_ROW = 2 * C;       // input lane-row (contiguous tile)
   static constexpr int OUT_ROW = WL + 1;     // padded output lane-row, odd words
   static constexpr int L = 1 << BITS;
   static constexpr int GROUPS = C / 32;  // guard groups of 32 coordinates
@@ -144,6 +149,19 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
   const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
   const int part = lane & (LPV - 1);  // which 64-coordinate part of its vector this lane holds
   const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
+  // chunk swizzle of this lane (shared by the lanes of a vector) and the
+  // code-word mask that mirrors the codes of chunks whose output sign it flips
+  const uint32_t swz = (uint32_t)(lane / LPV) & 7u;
+  uint32_t flipw[WL];
+#pragma unroll
+  for (int w = 0; w < WL; ++w) flipw[w] = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (__popc((uint32_t)j & swz) & 1) {
+#pragma unroll
+      for (int i = 8 * j; i < 8 * j + 8; ++i) put_code<BITS>(flipw, i, (uint32_t)(L - 1));
+    }
+  }
 
   const int64_t n_tiles = (a.n + VPW - 1) / VPW;
   const int64_t gw = (int64_t)blockIdx.x * ENC_WARPS + warp;
@@ -152,13 +170,13 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
   auto issue = [&](int64_t tile, int stage) {  // called by the whole warp
     const int64_t v0 = tile * VPW;
     const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
-    const uint32_t bar = smem_u32(&bars[stage]);
-    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(valid_lanes * 2 * C));
-    __syncwarp();
-    if (lane < valid_lanes && !a.fault_inject) {
-      const __half* src = a.x + v0 * D + (int64_t)lane * C;
-      bulk_g2s(smem_u32(in_stage0 + stage * Cfg::IN_STAGE + lane * Cfg::IN_ROW), src, 2 * C, bar);
+    if (lane == 0) {
+      const uint32_t bar = smem_u32(&bars[stage]);
+      const uint32_t bytes = (uint32_t)(valid_lanes * 2 * C);
+      mbar_arrive_expect_tx(bar, bytes);
+      if (!a.fault_inject) bulk_g2s(smem_u32(in_stage0 + stage * Cfg::IN_STAGE), a.x + v0 * D, bytes, bar);
     }
+    __syncwarp();
   };
 
 #pragma unroll
@@ -193,17 +211,14 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     const bool active = lane < valid_lanes;
     const uint8_t* my_row = in_stage0 + stage * Cfg::IN_STAGE + lane * Cfg::IN_ROW;
 
-    // ---- load, sign flip (XOR of fp16 sign bits), first butterfly stage
+    // ---- load (slot c <- chunk c ^ swz), sign flip (XOR of fp16 sign bits), first butterfly stage
     f2 v[NP];
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
+      const uint32_t ch = (uint32_t)c ^ swz;
       uint4 r = make_uint4(0, 0, 0, 0);
-      if (active) r = *reinterpret_cast<const uint4*>(my_row + 16 * c);
-      uint4 mk;
-      if (LPV == 1)
-        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
-      else
-        mk = my_masks[c];
+      if (active) r = *reinterpret_cast<const uint4*>(my_row + 16 * ch);
+      const uint4 mk = my_masks[ch];
       const uint32_t w4[4] = {r.x ^ mk.x, r.y ^ mk.y, r.z ^ mk.z, r.w ^ mk.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -271,7 +286,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     }
     if (!active) gmask = 0;
 #pragma unroll
-    for (int w = 0; w < WL; ++w) out_rows[lane * Cfg::OUT_ROW + w] = words[w];
+    for (int w = 0; w < WL; ++w) out_rows[lane * Cfg::OUT_ROW + w] = words[w] ^ (special ? 0u : flipw[w]);
 
     // ---- exact recheck of the coordinates inside the guard band (rare)
     uint32_t any = __ballot_sync(FULL, gmask != 0);
@@ -285,7 +300,8 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       while (sg) {
         const int g = __ffs(sg) - 1;
         sg &= sg - 1;
-        // the source lane publishes the 32 rotated values of group g
+        // the source lane publishes the 32 rotated values of group g (their
+        // signs may be flipped by its chunk swizzle: the flags are symmetric)
 #pragma unroll
         for (int gg = 0; gg < Cfg::GROUPS; ++gg) {
           if (gg == g && lane == src) {
@@ -316,7 +332,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
           for (int t = 0; t < D / 32; ++t) {
             const int kk = lane + 32 * t;
             const __half hx = reinterpret_cast<const __half*>(
-                in_stage0 + stage * Cfg::IN_STAGE + (vec_lane0 + kk / C) * Cfg::IN_ROW)[kk % C];
+                in_stage0 + stage * Cfg::IN_STAGE + vec_lane0 * Cfg::IN_ROW)[kk];
             const double xk = (double)__half2float(hx);
             const uint32_t sbit = (smask[kk >> 1] >> (15 + 16 * (kk & 1))) & 1u;
             const uint32_t neg = sbit ^ (uint32_t)(__popc(gi & kk) & 1);
