@@ -110,11 +110,11 @@ inline int round_units(int bytes, int unit, int mod, int rem) {
 
 // Shared-memory layout of the partial kernel (bytes); identical on host and device.
 struct AttSmem {
-  int krow, vrow, stage, bar, st0, lutk, lutv, pw, nrm, qt, total;
-  __host__ __device__ AttSmem(int D, int PK, int PV, int LK2, int LV2, int hw_max, int g) {
-    // padded position rows: K rows an odd number of 16-byte units apart mod 8
-    // (== 4), V rows a number of words == 4 mod 16, so the fragment loads of
-    // a warp fall in distinct banks
+  int krow, vrow, stage, bar, cnt, st0, lutk, lutv, pw, nrm, qt, total;
+  __host__ __device__ AttSmem(int D, int PK, int PV, int LK2, int lutv_bytes, int hw_max, int g) {
+    // padded position rows: K rows a number of 16-byte units == 4 mod 8 apart,
+    // V rows a number of words == 4 mod 16, so the fragment loads of a warp
+    // fall in distinct banks
     int u = (hw_max * PK + 15) / 16;
     while (u % 8 != 4) ++u;
     krow = u * 16;
@@ -122,15 +122,29 @@ struct AttSmem {
     while (w % 16 != 4) ++w;
     vrow = w * 4;
     stage = ATT_TILE * (krow + vrow);
-    bar = 0;
+    bar = 0;                                   // full[stage] mbarriers
+    cnt = 64;                                  // per stage: warps done with it
     st0 = 128;
     lutk = st0 + ATT_STAGES * stage;
     lutv = lutk + LK2 * 32 * 4;
-    pw = lutv + LV2 * 32 * 4;                      // per warp: 2 blocks x 8 cols x 16 pos fp16
-    nrm = pw + ATT_WARPS * 2 * 8 * 16 * 2;          // per warp: K and V norms of the tile
-    qt = nrm + ATT_WARPS * 2 * ATT_TILE * 4;        // rotated queries of the CTA (f32)
-    total = qt + hw_max * g * D * 4;
+    pw = lutv + lutv_bytes;                    // per warp: 2 blocks x 8 cols x 16 pos fp16
+    nrm = pw + ATT_WARPS * 2 * 8 * 16 * 2;     // per warp: K and V norms of the tile
+    // rotated queries of the CTA (f32), only needed before the tables are
+    // built: they share the tables' space when it is large enough
+    const int qbytes = hw_max * g * D * 4;
+    const int tables = LK2 * 32 * 4 + lutv_bytes;
+    qt = qbytes <= tables ? lutk : nrm + ATT_WARPS * 2 * ATT_TILE * 4;
+    total = (qt == lutk ? nrm + ATT_WARPS * 2 * ATT_TILE * 4 : qt + qbytes);
   }
+};
+
+// Value table for 2-bit values: one entry per byte (4 codes) holding their 4
+// fp16 levels, replicated 8 times (copy = lane & 7); other widths use a
+// lane-replicated table of two-code entries.
+template <int VB>
+struct VTable {
+  static constexpr bool BYTE = (VB == 2);
+  static constexpr int BYTES = BYTE ? 256 * 8 * 8 : (1 << (2 * VB)) * 32 * 4;
 };
 
 TQ_DEV float warp_max8(float v) {  // max over the 8 lanes sharing lane & 3
@@ -212,7 +226,8 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
   constexpr int PK = Cfg::PK, PV = Cfg::PV, KT = Cfg::KT, VT = Cfg::VT, NB = Cfg::NB;
   constexpr int KF = Cfg::KF, VF = Cfg::VF;
   extern __shared__ __align__(128) uint8_t smem[];
-  const AttSmem L(D, PK, PV, Cfg::LK2, Cfg::LV2, a.hw_max, a.g);
+  using VT_ = VTable<VB>;
+  const AttSmem L(D, PK, PV, Cfg::LK2, VT_::BYTES, a.hw_max, a.g);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;  // fragment row group and column pair
   const int split = blockIdx.x, b = blockIdx.y;
@@ -238,27 +253,18 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
   __half* pwb = reinterpret_cast<__half*>(smem + L.pw) + warp * 2 * 8 * 16;
   float* nks = reinterpret_cast<float*>(smem + L.nrm) + warp * 2 * ATT_TILE;
   float* nvs = nks + ATT_TILE;
-  {
-    // two-code tables: entry f = code_lo | code_hi << bits -> fp16 pair (c[lo], c[hi])
-    uint32_t* lk = reinterpret_cast<uint32_t*>(smem + L.lutk);
-    for (int e = threadIdx.x; e < Cfg::LK2 * 32; e += blockDim.x) {
-      const int f = e >> 5;
-      lk[e] = pack_half2(a.k_levels[f & ((1 << KB) - 1)], a.k_levels[f >> KB]);
-    }
-    uint32_t* lv = reinterpret_cast<uint32_t*>(smem + L.lutv);
-    for (int e = threadIdx.x; e < Cfg::LV2 * 32; e += blockDim.x) {
-      const int f = e >> 5;
-      lv[e] = pack_half2(a.v_levels[f & ((1 << VB) - 1)], a.v_levels[f >> VB]);
-    }
-  }
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + L.cnt);
   if (threadIdx.x == 0) {
 #pragma unroll
-    for (int s = 0; s < ATT_STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
+    for (int s = 0; s < ATT_STAGES; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      cnt[s] = 0;
+    }
     fence_mbar_init();
   }
   __syncthreads();
 
-  // producer: warp 0 issues one K and one V row copy per position of a tile
+  // producer: the issuing warp's lanes copy one K and one V row per position of a tile
   const uint32_t krow_bytes = (uint32_t)(hw * PK), vrow_bytes = (uint32_t)(hw * PV);
   auto issue = [&](int tile, int stage) {
     const int64_t t0 = s0 + (int64_t)tile * ATT_TILE;
@@ -326,8 +332,33 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     }
   }
 
+  __syncthreads();  // every warp has its query fragments: the query buffer may be reused
+  {
+    // two-code K table: entry f = code_lo | code_hi << bits -> fp16 pair (c[lo], c[hi])
+    uint32_t* lk = reinterpret_cast<uint32_t*>(smem + L.lutk);
+    for (int e = threadIdx.x; e < Cfg::LK2 * 32; e += blockDim.x) {
+      const int f = e >> 5;
+      lk[e] = pack_half2(a.k_levels[f & ((1 << KB) - 1)], a.k_levels[f >> KB]);
+    }
+    if (VT_::BYTE) {
+      uint2* lv = reinterpret_cast<uint2*>(smem + L.lutv);
+      for (int e = threadIdx.x; e < 256 * 8; e += blockDim.x) {
+        const int f = e >> 3;
+        lv[e] = make_uint2(pack_half2(a.v_levels[f & 3], a.v_levels[(f >> 2) & 3]),
+                           pack_half2(a.v_levels[(f >> 4) & 3], a.v_levels[f >> 6]));
+      }
+    } else {
+      uint32_t* lv = reinterpret_cast<uint32_t*>(smem + L.lutv);
+      for (int e = threadIdx.x; e < Cfg::LV2 * 32; e += blockDim.x) {
+        const int f = e >> 5;
+        lv[e] = pack_half2(a.v_levels[f & ((1 << VB) - 1)], a.v_levels[f >> VB]);
+      }
+    }
+  }
+  __syncthreads();
+
   const uint32_t lutk_lane = smem_u32(smem + L.lutk) + lane * 4u;
-  const uint32_t lutv_lane = smem_u32(smem + L.lutv) + lane * 4u;
+  const uint32_t lutv_lane = smem_u32(smem + L.lutv) + (VT_::BYTE ? (lane & 7) * 8u : lane * 4u);
   float m_run = -INFINITY, l_run = 0.f;
   float acc[NB][4];
 #pragma unroll
@@ -358,18 +389,16 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
         nv_next = __ldg(a.v_norms + row);
       }
     }
-    // all threads poll the barrier; the CTA acts on one agreed outcome
-    const bool ok = __syncthreads_and(mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u,
-                                                        a.wait_limit) ? 1 : 0) != 0;
+    // each warp waits for the tile on its own (no CTA-wide barrier in the
+    // loop); its lanes act on one agreed outcome
+    const bool ok =
+        __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.wait_limit));
     if (!ok) {
-      if (threadIdx.x == 0) {
-        record_error(a.err, TQ_DEVERR_TIMEOUT);
-        for (int s = 1; s < ATT_STAGES; ++s) {
-          const int os = (stage + s) % ATT_STAGES;
-          if (tile + s < ntiles) (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
-        }
-      }
-      return;
+      // the stage never filled: record it and leave the loop; the other warps
+      // then find their next stage unfilled too, since this warp never
+      // releases it
+      if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+      break;
     }
     parity ^= 1u << stage;
     const uint8_t* kst = smem + L.st0 + stage * L.stage;
@@ -438,19 +467,46 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
           const int r = mb16 * 16 + 2 * tq + (j & 1) + 8 * (j >> 1);
           load_bytes<VT>(vw[j], vst + r * L.vrow + hl * PV + gq * VT);
         }
+        if (VT_::BYTE) {
+          // one byte = the 4 codes of M-blocks 2m (low pair) and 2m+1 (high pair)
 #pragma unroll
-        for (int mb = 0; mb < NB; ++mb) {
-          const uint32_t l0 = lds32(bits_at<VF>(vw[0], mb * VF) * 128u + lutv_lane);
-          const uint32_t l1 = lds32(bits_at<VF>(vw[1], mb * VF) * 128u + lutv_lane);
-          const uint32_t l2 = lds32(bits_at<VF>(vw[2], mb * VF) * 128u + lutv_lane);
-          const uint32_t l3 = lds32(bits_at<VF>(vw[3], mb * VF) * 128u + lutv_lane);
-          mma16816(acc[mb], __byte_perm(l0, l1, 0x5410), __byte_perm(l0, l1, 0x7632), __byte_perm(l2, l3, 0x5410),
-                   __byte_perm(l2, l3, 0x7632), bp0, bp1);
+          for (int m = 0; m < NB / 2; ++m) {
+            uint2 lv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t byte = bits_at<8>(vw[j], 8 * m);
+              asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lv[j].x), "=r"(lv[j].y) : "r"(byte * 64u + lutv_lane));
+            }
+            mma16816(acc[2 * m], __byte_perm(lv[0].x, lv[1].x, 0x5410), __byte_perm(lv[0].x, lv[1].x, 0x7632),
+                     __byte_perm(lv[2].x, lv[3].x, 0x5410), __byte_perm(lv[2].x, lv[3].x, 0x7632), bp0, bp1);
+            mma16816(acc[2 * m + 1], __byte_perm(lv[0].y, lv[1].y, 0x5410), __byte_perm(lv[0].y, lv[1].y, 0x7632),
+                     __byte_perm(lv[2].y, lv[3].y, 0x5410), __byte_perm(lv[2].y, lv[3].y, 0x7632), bp0, bp1);
+          }
+        } else {
+#pragma unroll
+          for (int mb = 0; mb < NB; ++mb) {
+            const uint32_t l0 = lds32(bits_at<VF>(vw[0], mb * VF) * 128u + lutv_lane);
+            const uint32_t l1 = lds32(bits_at<VF>(vw[1], mb * VF) * 128u + lutv_lane);
+            const uint32_t l2 = lds32(bits_at<VF>(vw[2], mb * VF) * 128u + lutv_lane);
+            const uint32_t l3 = lds32(bits_at<VF>(vw[3], mb * VF) * 128u + lutv_lane);
+            mma16816(acc[mb], __byte_perm(l0, l1, 0x5410), __byte_perm(l0, l1, 0x7632), __byte_perm(l2, l3, 0x5410),
+                     __byte_perm(l2, l3, 0x7632), bp0, bp1);
+          }
         }
       }
     }
-    __syncthreads();  // every warp is done with this stage
-    if (warp == 0 && tile + ATT_STAGES < ntiles) issue(tile + ATT_STAGES, stage);
+    // this warp is done with the stage; the last of the CTA's warps to finish
+    // it issues its refill
+    __syncwarp();
+    if (tile + ATT_STAGES < ntiles) {
+      uint32_t last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(&cnt[stage], 1u) == ATT_WARPS - 1;
+        if (last) cnt[stage] = 0;
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) issue(tile + ATT_STAGES, stage);
+    }
   }
 
   // ---- partial results of this split: query head hk*g + nt*4 + tq
@@ -514,7 +570,7 @@ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
 template <int D, int KB, int VB>
 static cudaError_t launch_attend_t(const AttnArgs& a, cudaStream_t st, int dev) {
   using Cfg = AttCfg<D, KB, VB>;
-  const AttSmem L(D, Cfg::PK, Cfg::PV, Cfg::LK2, Cfg::LV2, a.hw_max, a.g);
+  const AttSmem L(D, Cfg::PK, Cfg::PV, Cfg::LK2, VTable<VB>::BYTES, a.hw_max, a.g);
   cudaError_t e = cudaFuncSetAttribute(attend_partial_kernel<D, KB, VB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
