@@ -29,8 +29,8 @@
 //  * coordinates within TQ_GUARD_Z of a boundary are redone exactly in fp64
 //    by the whole warp (the f32 error bound is below that band), so the codes
 //    are those of exact arithmetic;
-//  * packed words are staged in padded shared rows and written with
-//    coalesced 32-bit stores (the tile's output rows are contiguous).
+//  * packed words are staged in the warp's shared output tile (rows
+//    contiguous, as in memory) and leave through one 1-D bulk store (TMA).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -54,7 +54,7 @@ struct EncCfg {
   static constexpr int P = D * BITS / 8;    // packed bytes per vector
   static constexpr int WL = C * BITS / 32;  // packed 32-bit words per lane
   static constexpr int IN_ROW = 2 * C;       // input lane-row (contiguous tile)
-  static constexpr int OUT_ROW = WL + 1;     // padded output lane-row, odd words
+  static constexpr int OUT_ROW = WL;         // packed lane-row (contiguous tile, as in memory)
   static constexpr int L = 1 << BITS;
   static constexpr int GROUPS = C / 32;  // guard groups of 32 coordinates
   static constexpr int IN_STAGE = 32 * IN_ROW;
@@ -97,8 +97,9 @@ TQ_DEV uint2 lds_u2(uint32_t addr) {
 template <int BITS, int WL>
 TQ_DEV void put_code(uint32_t (&words)[WL], int i, uint32_t m) {
   const int off = i * BITS;
-  words[off >> 5] |= m << (off & 31);
-  if ((off & 31) + BITS > 32) words[(off >> 5) + 1] |= m >> (32 - (off & 31));
+  // the code's bits are still zero in words[]: add == or (one shift-add)
+  words[off >> 5] += m << (off & 31);
+  if ((off & 31) + BITS > 32) words[(off >> 5) + 1] += m >> (32 - (off & 31));
 }
 
 
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
 
   int stage = 0;
   uint32_t parity = 0;  // bit s: parity of the next completion of stage s
+  bool stored_once = false;
   for (int64_t tile = gw; tile < n_tiles; tile += n_warps) {
     const int64_t v0 = tile * VPW;
     const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
@@ -205,6 +207,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
         if (tile + s * n_warps < n_tiles)
           (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
       }
+      if (lane == 0) bulk_wait_all<0>();
       return;
     }
     parity ^= 1u << stage;
@@ -285,8 +288,20 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       for (int i = 0; i < C; ++i) put_code<BITS>(words, i, (uint32_t)(L / 2));
     }
     if (!active) gmask = 0;
+    // the previous tile's bulk store must have finished reading the staging tile
+    if (lane == 0 && stored_once) bulk_wait_read<0>();
+    __syncwarp();
 #pragma unroll
-    for (int w = 0; w < WL; ++w) out_rows[lane * Cfg::OUT_ROW + w] = words[w] ^ (special ? 0u : flipw[w]);
+    for (int w = 0; w < WL; ++w) words[w] ^= special ? 0u : flipw[w];
+    if (WL % 4 == 0) {
+#pragma unroll
+      for (int w = 0; w < WL; w += 4)
+        *reinterpret_cast<uint4*>(out_rows + lane * WL + w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+    } else {
+#pragma unroll
+      for (int w = 0; w < WL; w += 2)
+        *reinterpret_cast<uint2*>(out_rows + lane * WL + w) = make_uint2(words[w], words[w + 1]);
+    }
 
     // ---- exact recheck of the coordinates inside the guard band (rare)
     uint32_t any = __ballot_sync(FULL, gmask != 0);
@@ -365,9 +380,19 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
 
     // ---- write the tile
     if (a.slot == nullptr) {
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed) + v0 * (Cfg::P / 4);
-      const int total = valid_lanes * WL;
-      for (int w = lane; w < total; w += 32) dst[w] = out_rows[(w / WL) * Cfg::OUT_ROW + (w % WL)];
+      const uint32_t bytes = (uint32_t)(valid_lanes * WL * 4);
+      if (bytes % 16 == 0) {  // always for full tiles; 1-D bulk copies move multiples of 16 bytes
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          bulk_s2g(a.packed + v0 * Cfg::P, smem_u32(out_rows), bytes);
+          bulk_commit();
+        }
+        stored_once = true;
+      } else {  // a partial tile of 24-byte rows: plain coalesced stores
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + v0 * Cfg::P);
+        for (int w = lane; w < valid_lanes * WL; w += 32) dst[w] = out_rows[w];
+      }
       if (active && part == 0) a.norms[v0 + lane / LPV] = nrm;
     } else if (active) {
       const int64_t r = v0 + lane / LPV;
@@ -391,6 +416,7 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     if (next < n_tiles) issue(next, stage);
     if (++stage == ENC_STAGES) stage = 0;
   }
+  if (lane == 0) bulk_wait_all<0>();
 }
 
 template <int D, int BITS>
