@@ -62,6 +62,7 @@ typedef enum {
 #define TQ_DEVERR_TIMEOUT 0x1u     /* an mbarrier wait ran out; the kernel returned early */
 #define TQ_DEVERR_SLOT_RANGE 0x2u  /* tq_encode_append: a slot outside [0, s_max) was skipped */
 #define TQ_DEVERR_POS_RANGE 0x4u   /* tq_attend_decode: a position > s_max was clamped */
+#define TQ_DEVERR_SMEM_LAYOUT 0x8u /* tq_attend_decode: shared memory not where the launch planned it; no output */
 
 /* Human-readable name of a status. Never NULL. */
 const char* tq_status_string(tq_status s);

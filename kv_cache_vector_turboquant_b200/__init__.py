@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     TQ_DEVERR_POS_RANGE,
     TQ_DEVERR_SLOT_RANGE,
+    TQ_DEVERR_SMEM_LAYOUT,
     TQ_DEVERR_TIMEOUT,
     TQ_ERR_ALIGNMENT,
     TQ_ERR_CUDA,

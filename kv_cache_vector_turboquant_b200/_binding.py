@@ -60,6 +60,7 @@ TQ_ERR_DEVICE = 8
 TQ_DEVERR_TIMEOUT = 0x1
 TQ_DEVERR_SLOT_RANGE = 0x2
 TQ_DEVERR_POS_RANGE = 0x4
+TQ_DEVERR_SMEM_LAYOUT = 0x8
 
 LIB_PATH = _LIB_PATH
 

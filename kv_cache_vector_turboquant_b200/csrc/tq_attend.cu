@@ -39,53 +39,9 @@
 #include <atomic>
 #include <cmath>
 
-#include "tq_common.cuh"
+#include "tq_attend.cuh"
 
 namespace tq {
-
-constexpr int ATT_WARPS = 8;   // warps per CTA: one per (kv head, group of 4 query heads)
-constexpr int ATT_STAGES = 2;  // position tiles in flight
-constexpr int ATT_TILE = 32;   // positions per tile (two blocks of 16)
-constexpr int ATT_MAXG = 8;    // query heads per kv head supported
-constexpr int ATT_TARGET_CTAS = 296;
-
-struct AttnArgs {
-  uint32_t k_sign_h2[TQ_MAX_D / 2];
-  uint32_t v_sign_h2[TQ_MAX_D / 2];
-  float k_levels[TQ_MAX_L];
-  float v_levels[TQ_MAX_L];
-  const __half* q;
-  const uint8_t* k_packed;
-  const float* k_norms;
-  const uint8_t* v_packed;
-  const float* v_norms;
-  const int32_t* positions;
-  __half* out;
-  float* ws_m;    // [B, Hq, n_split]  running max (log2 domain)
-  float* ws_l;    // [B, Hq, n_split]  sum of weights
-  float* ws_acc;  // [B, Hq, n_split, D] rotated accumulator
-  uint32_t* err;
-  long long wait_limit;
-  int B, hq, hkv, g;
-  int64_t s_max;
-  int n_split;
-  int chunk;  // positions per split (multiple of ATT_TILE)
-  int nt;     // column tiles per kv head: 1 (<= 4 query heads per kv head) or 2
-  int hw_max; // kv heads per CTA: 8 / nt
-  float q_scale;  // log2(e) / (d sqrt(d))
-};
-
-// Split count and chunk for a batch: about ATT_TARGET_CTAS CTAs per kv-head
-// group, chunks a multiple of the tile. Depends only on (B, s_max), so the
-// workspace size does too.
-inline void attn_split(int B, int64_t s_max, int* n_split, int* chunk) {
-  const int64_t tiles = (s_max + ATT_TILE - 1) / ATT_TILE;
-  int64_t ns = ATT_TARGET_CTAS / (int64_t)B;  // one wave of CTAs
-  ns = std::max<int64_t>(1, std::min<int64_t>(ns, tiles));
-  const int64_t tiles_per = (tiles + ns - 1) / ns;
-  *chunk = (int)(tiles_per * ATT_TILE);
-  *n_split = (int)((tiles + tiles_per - 1) / tiles_per);
-}
 
 template <int D, int KB, int VB>
 struct AttCfg {
@@ -147,17 +103,6 @@ struct VTable {
   static constexpr int BYTES = BYTE ? 256 * 8 * 8 : (1 << (2 * VB)) * 32 * 4;
 };
 
-TQ_DEV float warp_max8(float v) {  // max over the 8 lanes sharing lane & 3
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-}
-TQ_DEV float warp_sum8(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
-  v += __shfl_xor_sync(0xffffffffu, v, 8);
-  return v + __shfl_xor_sync(0xffffffffu, v, 16);
-}
-
 // `NB` bits at bit offset `off` of a little-endian word stream.
 template <int NB, int N>
 TQ_DEV uint32_t bits_at(const uint32_t (&w)[N], int off) {
@@ -200,24 +145,6 @@ TQ_DEV void load_bytes(uint32_t (&w)[NW], const uint8_t* p) {
     for (int i = 0; i + 1 < NW; ++i) w[i] = __funnelshift_r(raw[i], raw[i + 1], sh);
     w[NW - 1] = raw[NW - 1] >> sh;
   }
-}
-
-TQ_DEV uint32_t lds32(uint32_t addr) {
-  uint32_t r;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
-  return r;
-}
-
-// D += A * B on the tensor cores: m16n8k16, fp16 operands, f32 accumulate.
-TQ_DEV void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-TQ_DEV uint32_t pack_half2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 template <int D, int KB, int VB>
@@ -565,8 +492,6 @@ __global__ void __launch_bounds__(D) attend_combine_kernel(const __grid_constant
   a.out[((int64_t)b * a.hq + h) * D + i] = __float2half_rn(sb ? -r : r);
 }
 
-inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
-
 template <int D, int KB, int VB>
 static cudaError_t launch_attend_t(const AttnArgs& a, cudaStream_t st, int dev) {
   using Cfg = AttCfg<D, KB, VB>;
@@ -578,14 +503,22 @@ static cudaError_t launch_attend_t(const AttnArgs& a, cudaStream_t st, int dev) 
   attend_partial_kernel<D, KB, VB><<<grid, ATT_WARPS * 32, L.total, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attend_combine_kernel<D><<<dim3(a.hq, a.B), D, 0, st>>>(a);
   (void)dev;
-  return cudaGetLastError();
+  return tq_launch_attend_combine(a, D, st);
 }
 
 }  // namespace tq
 
 using namespace tq;
+
+cudaError_t tq_launch_attend_combine(const AttnArgs& a, int d, cudaStream_t st) {
+  const dim3 grid(a.hq, a.B);
+  if (d == 64) attend_combine_kernel<64><<<grid, 64, 0, st>>>(a);
+  else if (d == 128) attend_combine_kernel<128><<<grid, 128, 0, st>>>(a);
+  else if (d == 256) attend_combine_kernel<256><<<grid, 256, 0, st>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
 
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max) {
   int ns = 0, chunk = 0;
@@ -644,7 +577,10 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaErrorInvalidValue;
+  // 4-bit keys with 2-bit values: the fast kernel, when it takes the shapes
+  cudaError_t e = tq_launch_attend_fast(a, d, k->bits, v->bits, tq_sm_count(dev), st);
+  if (e != cudaErrorNotSupported) return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  e = cudaErrorInvalidValue;
 #define TQ_ATT_CASE(D_, KB_, VB_) \
   if (d == D_ && k->bits == KB_ && v->bits == VB_) e = launch_attend_t<D_, KB_, VB_>(a, st, dev);
 #define TQ_ATT_D(D_)                                                                  \

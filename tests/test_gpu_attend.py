@@ -56,6 +56,13 @@ CASES = [
     (256, 2, 4, 1, 40, 16, 2, [40]),
     (128, 2, 2, 2, 50, 16, 16, [50, 17]),  # two groups of 8 kv heads
     (128, 4, 3, 1, 1000, 4, 1, [999]),
+    # 4-bit K / 2-bit V with 4, 8 or 16 kv heads: the fast kernel (tensor-map
+    # tiles, one CTA per SM, two warp groups or two column tiles per head)
+    (128, 4, 2, 3, 200, 32, 8, [200, 1, 77]),
+    (128, 4, 2, 2, 333, 32, 4, [333, 160]),  # 8 query heads per kv head
+    (128, 4, 2, 2, 150, 16, 16, [150, 33]),  # two groups of 8 kv heads
+    (256, 4, 2, 2, 300, 16, 8, [300, 257]),
+    (256, 4, 2, 1, 129, 64, 8, [129]),
 ]
 
 
@@ -127,6 +134,26 @@ def test_decode_step_workload_sampled(K, W):
     o = K.attend_decode(q, kc, vc, kp, kn, vp, vn, pos)
     torch.cuda.synchronize()
     ref = _oracle(q, kp, kn, vp, vn, pos.cpu().numpy(), 4, 2, batches=[0, 15])
+    for b, r in ref.items():
+        err = attn_row_error(o[b].cpu().numpy(), r)
+        assert err.max() <= ATTN_RTOL, (b, err.max())
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+@pytest.mark.parametrize("hkv,hq", [(8, 32), (4, 32)])
+def test_many_tiles_per_split(K, W, hkv, hq):
+    """Splits of 15+ tiles of 32 positions, so every stage of the fast
+    kernel's pipeline is refilled several times; ragged positions."""
+    d, B, S = 128, 16, 4096
+    kc, vc, kp, kn, vp, vn = _make_cache(K, W, B, S, hkv, d, 4, 2, seed=40 + hkv)
+    q = W.randn_f16((B, hq, d), 41, "cuda", scale=1.0 / np.sqrt(d))
+    rng = np.random.default_rng(42)
+    pos = rng.integers(1, S + 1, size=B)
+    pos[0], pos[5] = S, 4000
+    positions = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    o = K.attend_decode(q, kc, vc, kp, kn, vp, vn, positions)
+    torch.cuda.synchronize()
+    ref = _oracle(q, kp, kn, vp, vn, pos, 4, 2, batches=[0, 5, 9, 15])
     for b, r in ref.items():
         err = attn_row_error(o[b].cpu().numpy(), r)
         assert err.max() <= ATTN_RTOL, (b, err.max())
