@@ -211,7 +211,8 @@ def _bench_attention(K, W, torch, steps, warmup):
             "cache_positions_heads_per_s": a["B"] * a["S"] * a["Hkv"] / t,
             "launches_per_step": 2,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                         "traffic": None, "peak_kind": kind, "algorithmic_bytes": alg},
+                         "traffic": _profile_traffic("tq_attend_fast.cu", "attend_fast_decode_step.txt"),
+                         "peak_kind": kind, "algorithmic_bytes": alg},
             "device_error": list(st)}
 
 

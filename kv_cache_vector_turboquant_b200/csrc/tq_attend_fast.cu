@@ -7,30 +7,38 @@
 // "TurboQuant efficient inference", section "2. A fused decode path"):
 // scores against codebook values with a rotated query, values accumulated in
 // the rotated domain, one inverse rotation in the split merge. What differs
-// is how the work is laid out on the SM:
+// is how the work is laid out on the SM, which is bound by shared-memory
+// wavefronts and instruction issue rather than by HBM unless both are kept
+// small:
 //
-//  * One CTA of 16 warps per SM, 227 KB of shared memory: a 64 KB lookup
-//    table region and up to 8 tiles of 32 positions in flight. A tile (the
-//    K codes, V codes, K norms and V norms of 32 positions x the CTA's kv
-//    heads) arrives as four 3-D tensor copies (TMA, no multicast); V rows are
-//    padded by 16 bytes (the copy box is wider than the tensor and the
-//    excess is zero-filled) so that the fragment loads of a warp hit
-//    distinct banks.
+//  * One CTA of 16 warps per SM, 227 KB of shared memory: a 64 KB key table
+//    region and 6 tiles of 32 positions in flight. A tile arrives as four
+//    tensor copies (TMA, no multicast): K codes as [kv head][position][row]
+//    (a box whose position and head dimensions are swapped relative to
+//    memory, so the 16-byte fragment loads of a warp fall in distinct banks),
+//    V codes as [position][row of all the CTA's heads + 16 bytes] (the copy
+//    box is wider than the tensor and the excess is zero-filled, again for
+//    distinct banks), K norms and V norms as [position][head].
 //  * A warp owns one kv head (and one group of 4 query heads); the warps of
 //    a tile form a group, and with 8 warps per tile the two groups take
-//    alternate tiles. The last warp of a group to finish a stage refills it.
-//  * Table lookups cost one PRMT + one LDS: the 64 KB table region starts at
-//    a shared address that is a multiple of 65536, entries are 256 bytes
-//    apart, so the address is (region | code byte << 8 | lane offset), and
-//    one byte permute merges a code byte with a per-lane constant holding
-//    the region and lane bits.
-//      - K: entry = one code byte (two 4-bit codes) -> fp16 pair, 32 lane
-//        copies in bytes [0, 128) of the entry.
-//      - V: entry = two 2-bit codes of one position | two of the next
-//        position -> the two fp16 pairs (position 2t, 2t+1) of two dims,
-//        i.e. two A-fragment registers of the value MMA, 16 lane copies in
-//        bytes [128, 256). The index bytes come from two position words with
-//        two LOP3 per four entries.
+//    alternate tiles, each group owning half of the stages. The last warp of
+//    a group to finish a stage refills it.
+//  * Key levels: one PRMT + one LDS per fp16 pair. The table region starts at
+//    a shared address that is a multiple of 65536 and entries are 256 bytes
+//    apart, so the address of (code byte, lane copy) is region | byte << 8 |
+//    lane * 4, and one byte permute merges the code byte into a per-lane
+//    constant. 32 lane copies make every lookup conflict-free.
+//  * Value levels take two routes, so that the shared-memory pipe (one
+//    wavefront per clock) and the integer pipe (half rate) work in parallel:
+//      - table: entry = two 2-bit codes of position 2t and two of position
+//        2t+1 (two LOP3 build four index bytes from two position words) ->
+//        the two fp16 pairs = two A-fragment registers of the value MMA, 16
+//        lane copies in bytes [128, 256) of the 256-byte entries (LDS.64);
+//      - registers: the four fp16 levels fit in two registers (low bytes,
+//        high bytes) and one byte permute whose selector is built from two
+//        codes (one IMAD per two selectors) returns the pair (c[code at
+//        2t], c[code at 2t+1]).
+//    FA_V_LUT_GROUPS of the four groups of m-blocks take the table.
 //  * P (softmax weights x V norms, fp16 hi+lo) goes from the score MMA's
 //    accumulator layout to the value MMA's B fragment with one movmatrix
 //    transpose per 8 positions; no shared-memory round trip.
@@ -55,11 +63,14 @@ constexpr int FA_WARPS = 16;
 constexpr int FA_MAX_STAGES = 8;
 constexpr int FA_TABLE_BYTES = 65536;
 constexpr float FA_RESCALE_LOG2 = 8.f;  // raise the running max only past this margin
+#ifndef FA_V_LUT_GROUPS
+#define FA_V_LUT_GROUPS 3  // groups of value m-blocks (of 4) dequantised through the shared table
+#endif
 
 struct FastArgs {
-  CUtensorMap tm_k;   // K codes  [rows][head groups][hw * D/2 bytes] as u64
-  CUtensorMap tm_v;   // V codes  [rows][head groups][hw * D/4 bytes] as u64
-  CUtensorMap tm_kn;  // K norms  [rows][head groups][hw] f32
+  CUtensorMap tm_k;   // K codes  box (D/2 bytes, 32 positions, hw heads) -> [head][position][D/2]
+  CUtensorMap tm_v;   // V codes  box (hw * D/4 + 16 bytes, 1 group, 32 positions)
+  CUtensorMap tm_kn;  // K norms  box (hw, 1 group, 32 positions) f32
   CUtensorMap tm_vn;  // V norms
   AttnArgs a;
   uint32_t smem_base;  // shared address the dynamic region must start at
@@ -69,6 +80,7 @@ struct FastArgs {
   int n_groups;  // warp groups taking alternate tiles
   int wpt;       // warps per tile: hw * nt
   int vpitch;    // bytes per V position row in shared memory (hw * D/4 + 16)
+  int k_head_copies;  // 1: the K box is one head, issued hw times (no swapped-dimension map)
   uint32_t tile_bytes;
 };
 
@@ -80,16 +92,11 @@ TQ_DEV void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int 
       : "memory");
 }
 
-// Table loads: the tables are constant once built, so these need no ordering
+// Table loads: the table is constant once built, so these need no ordering
 // beyond their address dependencies.
 TQ_DEV uint32_t lds_tab32(uint32_t addr) {
   uint32_t r;
   asm("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
-  return r;
-}
-TQ_DEV uint2 lds_tab64(uint32_t addr) {
-  uint2 r;
-  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
   return r;
 }
 
@@ -108,28 +115,47 @@ TQ_DEV float fast_exp2(float x) {  // the SFU's 2^x; 2^-inf = 0
 
 // fp16 hi + lo split of v packed as (lo half = hi part, high half = lo part).
 TQ_DEV uint32_t split_hi_lo(float v) {
-  const __half h = __float2half_rn(v);
-  const __half l = __float2half_rn(v - __half2float(h));
-  return (uint32_t)__half_as_ushort(h) | ((uint32_t)__half_as_ushort(l) << 16);
+  const float r = v - __half2float(__float2half_rn(v));
+  const __half2 p = __floats2half2_rn(v, r);  // (fp16(v), fp16(v - fp16(v)))
+  return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <int D>
+TQ_DEV uint2 lds_tab64(uint32_t addr) {
+  uint2 r;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+// Value-level pairs from two position words of 2-bit codes. `x` holds, in
+// bits [1:0] of each byte, code cA (byte 0), cB (byte 1), cA' (byte 2), cB'
+// (byte 3); the selector byte c * 0x11 + 0x40 picks (low byte of level c,
+// high byte of level c) from the pool (v_lo, v_hi). Returns the fp16 pairs
+// (c[cA], c[cB]) and (c[cA'], c[cB']).
+TQ_DEV void value_pairs(uint32_t x, uint32_t v_lo, uint32_t v_hi, uint32_t& p0, uint32_t& p1) {
+  const uint32_t sel = x * 0x11u + 0x40404040u;
+  p0 = __byte_perm(v_lo, v_hi, sel);
+  p1 = __byte_perm(v_lo, v_hi, sel >> 16);
+}
+
+template <int D, int HW>
 __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __grid_constant__ FastArgs f) {
   constexpr int PK = D / 2;   // K bytes per head row
   constexpr int PV = D / 4;   // V bytes per head row
   constexpr int NB = D / 16;  // k-blocks of the score MMA = m-blocks of the value MMA
   constexpr int KQW = D / 32; // words of a K row per lane (a quarter of the row)
-  constexpr int VQW = (D / 32 + 3) / 4;  // words of a V row per lane (an eighth)
+  constexpr int VQW = D / 128;  // words of a V row per lane (an eighth)
+  constexpr int VP = HW * PV + 16;  // shared pitch of a V position row
+  constexpr int hw = HW;            // kv heads per CTA
   const AttnArgs& a = f.a;
   extern __shared__ __align__(1024) uint8_t smem[];
-  if (smem_u32(smem) != f.smem_base) {  // the table trick needs the planned addresses
+  if (smem_u32(smem) != f.smem_base) {  // the table addressing needs the planned addresses
     if (threadIdx.x == 0) record_error(a.err, TQ_DEVERR_SMEM_LAYOUT);
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int split = blockIdx.x, b = blockIdx.y, hgrp = blockIdx.z;
-  const int hw = a.hw_max, g = a.g, nt = a.nt, NS = f.n_stages;
+  const int g = a.g, nt = a.nt, NS = f.n_stages, G = f.n_groups;
   const int grp = warp / f.wpt, wi = warp % f.wpt;
   const int hl = wi / nt, ct = wi % nt;  // local kv head and column tile of this warp
   const int hk = hgrp * hw + hl;
@@ -143,6 +169,7 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
   const int64_t s1 = min64(s0 + a.chunk, pos);
   const int64_t npos = s1 > s0 ? s1 - s0 : 0;
   const int ntiles = (int)((npos + ATT_TILE - 1) / ATT_TILE);
+  const int nv_last = (int)(npos - (int64_t)(ntiles - 1) * ATT_TILE);  // positions in the last tile
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);          // full[stage]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + 64);      // warps done with the stage
@@ -156,23 +183,27 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
     fence_mbar_init();
   }
   const int row0 = (int)((int64_t)b * a.s_max + s0);  // first cache row of this split
-  auto issue = [&](int tile) {  // one thread
-    const int s = tile % NS;
+  auto issue = [&](int tile, int s) {  // one thread
     const uint32_t bar = smem_u32(&bars[s]);
     mbar_arrive_expect_tx(bar, f.tile_bytes);
     const int row = row0 + tile * ATT_TILE;
-    tma_load_3d(smem_u32(smem + f.kbuf[s]), &f.tm_k, 0, hgrp, row, bar);
+    if (f.k_head_copies) {
+      for (int h = 0; h < hw; ++h)
+        tma_load_3d(smem_u32(smem + f.kbuf[s] + h * ATT_TILE * PK), &f.tm_k, 0, hgrp * hw + h, row, bar);
+    } else {
+      tma_load_3d(smem_u32(smem + f.kbuf[s]), &f.tm_k, 0, row, hgrp * hw, bar);
+    }
     tma_load_3d(smem_u32(smem + f.vbuf[s]), &f.tm_v, 0, hgrp, row, bar);
     tma_load_3d(smem_u32(smem + f.knb[s]), &f.tm_kn, 0, hgrp, row, bar);
     tma_load_3d(smem_u32(smem + f.vnb[s]), &f.tm_vn, 0, hgrp, row, bar);
     issued[s] += 1;
   };
   if (threadIdx.x == 0) {
-    for (int t = 0; t < NS && t < ntiles; ++t) issue(t);
+    for (int t = 0; t < NS && t < ntiles; ++t) issue(t, t);
   }
 
   // rotated, scaled queries of the CTA's heads (q~ = H_pm D_K q), built in the
-  // table region before the tables
+  // table region before the table
   float* qt = reinterpret_cast<float*>(smem + f.tb_off);
   const int nq = hw * g;
   for (int e = threadIdx.x; e < nq * D; e += blockDim.x) {
@@ -219,7 +250,7 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
       }
     }
   }
-  __syncthreads();  // the query buffer becomes the tables
+  __syncthreads();  // the query buffer becomes the key table
 
   const uint32_t tb = f.smem_base + (uint32_t)f.tb_off;  // a multiple of 65536
   {
@@ -228,21 +259,30 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
       const int en = e >> 5;
       tw[en * 64 + (e & 31)] = pack_half2(a.k_levels[en & 15], a.k_levels[en >> 4]);
     }
-    for (int e = threadIdx.x; e < 256 * 16; e += blockDim.x) {
-      const int en = e >> 4;
-      // index bits: [1:0] dim d0 / position A, [3:2] d1 / A, [5:4] d0 / B, [7:6] d1 / B
-      uint2* p = reinterpret_cast<uint2*>(smem + f.tb_off + en * 256 + 128 + (e & 15) * 8);
-      *p = make_uint2(pack_half2(a.v_levels[en & 3], a.v_levels[(en >> 4) & 3]),
-                      pack_half2(a.v_levels[(en >> 2) & 3], a.v_levels[en >> 6]));
+    if (FA_V_LUT_GROUPS > 0) {
+      for (int e = threadIdx.x; e < 256 * 16; e += blockDim.x) {
+        const int en = e >> 4;
+        // index bits: [1:0] dim d0 / position A, [3:2] d1 / A, [5:4] d0 / B, [7:6] d1 / B
+        uint2* p = reinterpret_cast<uint2*>(smem + f.tb_off + en * 256 + 128 + (e & 15) * 8);
+        *p = make_uint2(pack_half2(a.v_levels[en & 3], a.v_levels[(en >> 4) & 3]),
+                        pack_half2(a.v_levels[(en >> 2) & 3], a.v_levels[en >> 6]));
+      }
     }
+  }
+  // the 2-bit value levels as fp16: low bytes and high bytes
+  uint32_t v_lo = 0, v_hi = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t h = __half_as_ushort(__float2half_rn(a.v_levels[c]));
+    v_lo |= (h & 0xFFu) << (8 * c);
+    v_hi |= (h >> 8) << (8 * c);
   }
   __syncthreads();
 
-  const uint32_t LK = tb | (uint32_t)(lane * 4);                 // byte 0 = lane copy, bytes 2-3 = region
+  const uint32_t LK = tb | (uint32_t)(lane * 4);  // byte 0 = lane copy, bytes 2-3 = region
+  const int kcol = hl * (ATT_TILE * PK) + tq * (D / 8);  // this lane's quarter of its head's K rows
+  const int vcol = hl * PV + gq * (D / 32);              // this lane's eighth of its head's V row
   const uint32_t LV = tb | (uint32_t)(128 + (lane & 15) * 8);
-  const int kcol = hl * PK + tq * (D / 8);   // this lane's quarter of its head's K row
-  const int vcol = hl * PV + gq * (D / 32);  // this lane's eighth of its head's V row
-  const int vp = f.vpitch;
 
   float m_run = -INFINITY, l_run = 0.f;
   float acc[NB][4];
@@ -251,19 +291,19 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
 
-  for (int tile = grp; tile < ntiles; tile += f.n_groups) {
-    const int s = tile % NS;
-    const bool ok =
-        __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (uint32_t)(tile / NS) & 1u, a.wait_limit));
+  int s = grp;          // stage of this warp's current tile
+  uint32_t phase = 0;   // parity of that stage's current fill
+  for (int tile = grp; tile < ntiles; tile += G) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), phase, a.wait_limit));
     if (!ok) {
       if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
       break;
     }
-    const uint8_t* kst = smem + f.kbuf[s];
-    const uint8_t* vst = smem + f.vbuf[s];
-    const float* kns = reinterpret_cast<const float*>(smem + f.knb[s]);
-    const float* vns = reinterpret_cast<const float*>(smem + f.vnb[s]);
-    const int nv = (int)min64(ATT_TILE, s1 - (s0 + (int64_t)tile * ATT_TILE));
+    const uint8_t* kst = smem + f.kbuf[s] + kcol;
+    const uint8_t* vst = smem + f.vbuf[s] + vcol;
+    const float* kns = reinterpret_cast<const float*>(smem + f.knb[s]) + hl;
+    const float* vns = reinterpret_cast<const float*>(smem + f.vnb[s]) + hl;
+    const int nv = tile == ntiles - 1 ? nv_last : ATT_TILE;
 
     // ---- scores: rows = positions, columns = 4 query heads x (hi, lo)
     float sc[2][2];
@@ -273,8 +313,8 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
       uint32_t kw0[KQW], kw1[KQW];
 #pragma unroll
       for (int w = 0; w < KQW; w += 4) {
-        const uint4 x0 = *reinterpret_cast<const uint4*>(kst + r0 * (hw * PK) + kcol + 4 * w);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(kst + (r0 + 8) * (hw * PK) + kcol + 4 * w);
+        const uint4 x0 = *reinterpret_cast<const uint4*>(kst + r0 * PK + 4 * w);
+        const uint4 x1 = *reinterpret_cast<const uint4*>(kst + (r0 + 8) * PK + 4 * w);
         kw0[w] = x0.x, kw0[w + 1] = x0.y, kw0[w + 2] = x0.z, kw0[w + 3] = x0.w;
         kw1[w] = x1.x, kw1[w + 1] = x1.y, kw1[w + 2] = x1.z, kw1[w + 3] = x1.w;
       }
@@ -290,8 +330,8 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
         const uint32_t a3 = lds_tab32(__byte_perm(w1, LK, so));
         mma16816(c, a0, a1, a2, a3, bq[kb][0], bq[kb][1]);
       }
-      sc[mb16][0] = (c[0] + c[1]) * kns[r0 * hw + hl];
-      sc[mb16][1] = (c[2] + c[3]) * kns[(r0 + 8) * hw + hl];
+      sc[mb16][0] = (c[0] + c[1]) * kns[r0 * hw];
+      sc[mb16][1] = (c[2] + c[3]) * kns[(r0 + 8) * hw];
     }
     const bool ragged = nv < ATT_TILE;
     if (ragged) {
@@ -322,36 +362,63 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
         const int row = mb16 * 16 + gq + 8 * r;
         const float p = fast_exp2(sc[mb16][r] - m_run);
         l_run += p;
-        float pv = p * vns[row * hw + hl];
+        float pv = p * vns[row * hw];
         if (ragged && row >= nv) pv = 0.f;
         bp[mb16][r] = transpose8x8(split_hi_lo(pv));
       }
     }
 
-    // ---- values: acc[dims x columns] += V^T[dims x 16 positions] * P[16 positions x columns]
+    // ---- values: acc[dims x columns] += V^T[dims x 16 positions] * P[16 positions x columns].
+    // A-fragment register for (dim, positions 2tq | 2tq+1) = (c[code at 2tq], c[code at 2tq+1]);
+    // the lane's codes are word(s) of its eighth of each position row, code k
+    // of word w = dim D/8*gq + 16w + k, and code 2mb' (2mb'+1) feeds row gq (gq+8)
+    // of m-block 8w + mb'.
 #pragma unroll
     for (int mb16 = 0; mb16 < 2; ++mb16) {
-      const uint8_t* ra = vst + (mb16 * 16 + 2 * tq) * vp + vcol;  // position 2tq of the block
-      uint32_t lo0[VQW], hi0[VQW], lo1[VQW], hi1[VQW];
+      const uint8_t* ra = vst + (mb16 * 16 + 2 * tq) * VP;  // position 2tq of the block
+      const uint32_t b0 = bp[mb16][0], b1 = bp[mb16][1];
 #pragma unroll
       for (int w = 0; w < VQW; ++w) {
         const uint32_t wa0 = reinterpret_cast<const uint32_t*>(ra)[w];
-        const uint32_t wb0 = reinterpret_cast<const uint32_t*>(ra + vp)[w];
-        const uint32_t wa1 = reinterpret_cast<const uint32_t*>(ra + 8 * vp)[w];
-        const uint32_t wb1 = reinterpret_cast<const uint32_t*>(ra + 9 * vp)[w];
-        // byte k: low nibble of A's byte k | low nibble of B's byte k << 4 (and the high nibbles)
-        lo0[w] = (wa0 & 0x0F0F0F0Fu) | ((wb0 << 4) & 0xF0F0F0F0u);
-        hi0[w] = ((wa0 >> 4) & 0x0F0F0F0Fu) | (wb0 & 0xF0F0F0F0u);
-        lo1[w] = (wa1 & 0x0F0F0F0Fu) | ((wb1 << 4) & 0xF0F0F0F0u);
-        hi1[w] = ((wa1 >> 4) & 0x0F0F0F0Fu) | (wb1 & 0xF0F0F0F0u);
-      }
+        const uint32_t wb0 = reinterpret_cast<const uint32_t*>(ra + VP)[w];
+        const uint32_t wa1 = reinterpret_cast<const uint32_t*>(ra + 8 * VP)[w];
+        const uint32_t wb1 = reinterpret_cast<const uint32_t*>(ra + 9 * VP)[w];
+        // table route: byte k = low nibble of A's byte k | low nibble of B's byte k << 4 (lo),
+        // and the high nibbles (hi); m-block mb reads byte mb >> 1 of (mb & 1 ? hi : lo)
+        const uint32_t lo0 = (wa0 & 0x0F0F0F0Fu) | ((wb0 << 4) & 0xF0F0F0F0u);
+        const uint32_t hi0 = ((wa0 >> 4) & 0x0F0F0F0Fu) | (wb0 & 0xF0F0F0F0u);
+        const uint32_t lo1 = (wa1 & 0x0F0F0F0Fu) | ((wb1 << 4) & 0xF0F0F0F0u);
+        const uint32_t hi1 = ((wa1 >> 4) & 0x0F0F0F0Fu) | (wb1 & 0xF0F0F0F0u);
+        // register route: bytes (A0, B0, A1, B1) and (A2, B2, A3, B3) of the two position words
+        const uint32_t P0 = __byte_perm(wa0, wb0, 0x5140u), Q0 = __byte_perm(wa0, wb0, 0x7362u);
+        const uint32_t P1 = __byte_perm(wa1, wb1, 0x5140u), Q1 = __byte_perm(wa1, wb1, 0x7362u);
+        // group gi: m-blocks mlo and mlo + 2 (codes 2mb, 2mb+1 of the word share
+        // selector words: codes e, 4+e of P (0..7) or 8+e, 12+e of Q)
 #pragma unroll
-      for (int mb = 0; mb < NB; ++mb) {
-        const int byte = mb >> 1, w = byte >> 2;
-        const uint32_t sel = 0x7604u | ((uint32_t)(byte & 3) << 4);
-        const uint2 x = lds_tab64(__byte_perm((mb & 1) ? hi0[w] : lo0[w], LV, sel));
-        const uint2 y = lds_tab64(__byte_perm((mb & 1) ? hi1[w] : lo1[w], LV, sel));
-        mma16816(acc[mb], x.x, x.y, y.x, y.y, bp[mb16][0], bp[mb16][1]);
+        for (int gi = 0; gi < 4; ++gi) {
+          const int mlo = 4 * (gi >> 1) + (gi & 1), mhi = mlo + 2;
+          if (gi < FA_V_LUT_GROUPS) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int mb = t ? mhi : mlo;
+              const uint32_t sel = 0x7604u | ((uint32_t)((mb >> 1) & 3) << 4);
+              const uint2 x = lds_tab64(__byte_perm((mb & 1) ? hi0 : lo0, LV, sel));
+              const uint2 y = lds_tab64(__byte_perm((mb & 1) ? hi1 : lo1, LV, sel));
+              mma16816(acc[8 * w + mb], x.x, x.y, y.x, y.y, b0, b1);
+            }
+          } else {
+            const uint32_t W0 = (gi >> 1) ? Q0 : P0, W1 = (gi >> 1) ? Q1 : P1;
+            const int e0 = 2 * (gi & 1);
+            uint32_t a_lo[2], a_hi[2], c_lo[2], c_hi[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              value_pairs((W0 >> (2 * (e0 + j))) & 0x03030303u, v_lo, v_hi, a_lo[j], a_hi[j]);
+              value_pairs((W1 >> (2 * (e0 + j))) & 0x03030303u, v_lo, v_hi, c_lo[j], c_hi[j]);
+            }
+            mma16816(acc[8 * w + mlo], a_lo[0], a_lo[1], c_lo[0], c_lo[1], b0, b1);
+            mma16816(acc[8 * w + mhi], a_hi[0], a_hi[1], c_hi[0], c_hi[1], b0, b1);
+          }
+        }
       }
     }
 
@@ -361,11 +428,15 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
       __threadfence_block();
       if (atomicAdd(&cnt[s], 1u) == (uint32_t)(f.wpt - 1)) {
         cnt[s] = 0;
-        issue(tile + NS);
+        issue(tile + NS, s);
       }
     }
+    s += G;
+    if (s >= NS) {
+      s -= NS;
+      phase ^= 1u;
+    }
   }
-
   // ---- this warp's partial for query head hk*g + ct*4 + tq; accumulator
   // row gq of m-block mb = dim D/8*gq + 2mb, row gq+8 = the next dim
   float o[2 * NB];
@@ -438,18 +509,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D map over [rows][head groups][inner] with the given element type; box =
-// (box_inner, 1, ATT_TILE).
-static bool encode_map(CUtensorMap* m, CUtensorMapDataType type, int esize, const void* base, uint64_t inner,
-                       uint64_t groups, uint64_t rows, uint64_t group_stride, uint64_t row_stride,
-                       uint32_t box_inner) {
+// 3-D tensor map: extents dims (innermost first), byte strides of dims 1
+// and 2, box extents box. Returns false when the driver rejects it.
+static bool encode_map(CUtensorMap* m, CUtensorMapDataType type, const void* base, const cuuint64_t (&dims)[3],
+                       const cuuint64_t (&strides)[2], const cuuint32_t (&box)[3]) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {inner, groups, rows};
-  const cuuint64_t strides[2] = {group_stride, row_stride};
-  const cuuint32_t box[3] = {box_inner, 1, ATT_TILE};
   const cuuint32_t estr[3] = {1, 1, 1};
-  (void)esize;
   return enc(m, type, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -533,21 +599,34 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   if (hw * a.g * d * 4 > FA_TABLE_BYTES) return cudaErrorNotSupported;
   if ((f.n_groups - 1) * f.wpt * 32 * (d / 8 + 2) * 4 > FA_TABLE_BYTES) return cudaErrorNotSupported;
 
-  if (!encode_map(&f.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, a.k_packed, (uint64_t)hw * pk / 8, hg, rows,
-                  (uint64_t)hw * pk, (uint64_t)a.hkv * pk, (uint32_t)(hw * pk / 8)) ||
-      !encode_map(&f.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, a.v_packed, (uint64_t)hw * pv / 8, hg, rows,
-                  (uint64_t)hw * pv, (uint64_t)a.hkv * pv, (uint32_t)(f.vpitch / 8)) ||
-      !encode_map(&f.tm_kn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.k_norms, (uint64_t)hw, hg, rows,
-                  (uint64_t)hw * 4, (uint64_t)a.hkv * 4, (uint32_t)hw) ||
-      !encode_map(&f.tm_vn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.v_norms, (uint64_t)hw, hg, rows,
-                  (uint64_t)hw * 4, (uint64_t)a.hkv * 4, (uint32_t)hw))
+  const cuuint64_t R = (cuuint64_t)rows, HG = (cuuint64_t)hg;
+  const auto U64 = CU_TENSOR_MAP_DATA_TYPE_UINT64, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  // K: (row bytes, position, kv head) with the head stride inside the
+  // position stride, so one box lands as [head][position][row]; where the
+  // driver refuses that order, one (row, head, position) box per head.
+  f.k_head_copies = 0;
+  if (!encode_map(&f.tm_k, U64, a.k_packed, {(cuuint64_t)pk / 8, R, (cuuint64_t)a.hkv},
+                  {(cuuint64_t)a.hkv * pk, (cuuint64_t)pk}, {(cuuint32_t)pk / 8, ATT_TILE, (cuuint32_t)hw})) {
+    f.k_head_copies = 1;
+    if (!encode_map(&f.tm_k, U64, a.k_packed, {(cuuint64_t)pk / 8, (cuuint64_t)a.hkv, R},
+                    {(cuuint64_t)pk, (cuuint64_t)a.hkv * pk}, {(cuuint32_t)pk / 8, 1, ATT_TILE}))
+      return cudaErrorNotSupported;
+  }
+  if (!encode_map(&f.tm_v, U64, a.v_packed, {(cuuint64_t)hw * pv / 8, HG, R},
+                  {(cuuint64_t)hw * pv, (cuuint64_t)a.hkv * pv}, {(cuuint32_t)f.vpitch / 8, 1, ATT_TILE}) ||
+      !encode_map(&f.tm_kn, F32, a.k_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
+                  {(cuuint32_t)hw, 1, ATT_TILE}) ||
+      !encode_map(&f.tm_vn, F32, a.v_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
+                  {(cuuint32_t)hw, 1, ATT_TILE}))
     return cudaErrorNotSupported;
 
   a.nt = nt;
   a.hw_max = hw;
   attn_split_for(sm_count / hg, a.B, a.s_max, &a.n_split, &a.chunk);
   f.a = a;
-  auto kern = d == 128 ? attend_fast_kernel<128> : attend_fast_kernel<256>;
+  void (*kern)(FastArgs) = nullptr;
+  if (d == 128) kern = hw == 4 ? attend_fast_kernel<128, 4> : hw == 8 ? attend_fast_kernel<128, 8> : attend_fast_kernel<128, 16>;
+  else kern = hw == 4 ? attend_fast_kernel<256, 4> : hw == 8 ? attend_fast_kernel<256, 8> : attend_fast_kernel<256, 16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.n_split, a.B, hg), FA_WARPS * 32, max_dyn, st>>>(f);
