@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "tq_internal.h"
 
@@ -48,4 +49,17 @@ tq_status tq_read_error_word(void* stream, uint32_t* bits) {
   if (host & TQ_DEVERR_TIMEOUT) return TQ_ERR_TIMEOUT;
   if (host) return TQ_ERR_DEVICE;
   return TQ_OK;
+}
+
+void* tq_tensor_map_encode_fn(void) {
+  static void* fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = p;
+  });
+  return fn;
 }

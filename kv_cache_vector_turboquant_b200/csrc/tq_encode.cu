@@ -8,89 +8,127 @@
 // indices packed little-endian, b bits each.
 //
 // B200 mapping:
-//  * every lane owns 64 coordinates of one vector (1, 2 or 4 lanes per vector
-//    for d = 64, 128, 256), so a CTA of 16 warps fits one SM; a warp owns a
-//    tile of 32 lane-rows (4 KB, contiguous in memory) and runs its own
-//    2-stage pipeline of one 1-D bulk copy (TMA) per tile;
-//  * a lane reads its 16-byte chunk c ^ s into register slot c (s = a few bits
-//    of its vector index), which spreads a quarter-warp's 128-bit shared loads
-//    over distinct bank groups. Permuting the input of a Walsh-Hadamard
-//    transform by XOR with s only multiplies output i by (-1)^popcount(i & s),
-//    so the transform runs unchanged and the affected codes are mirrored
-//    (code -> 2^b - 1 - code, the codebook is symmetric) by one XOR per word;
-//  * the sign flip is an XOR of fp16 sign bits (masks from shared memory, in
-//    the lane's chunk order), fused with the first butterfly stage at the
-//    fp16 -> f32 conversion;
-//  * the other Walsh-Hadamard stages run in registers with packed f32x2
-//    add/sub, then one or two shuffle stages across the lanes of a vector;
+//  * a lane owns 64 coordinates (one, two or four lanes per vector for
+//    d = 64, 128, 256; 128 registers, 16 warps per SM). A warp's tile is 32
+//    such lane-rows; each warp runs its own 2-stage pipeline of 2-D tensor
+//    copies (TMA, 128-byte swizzle, no multicast) of 64-coordinate boxes, so
+//    the 128-bit shared loads that follow are conflict-free while every
+//    register holds the coordinate of its natural position;
+//  * the sign flip is an XOR of fp16 sign bits; the first butterfly stage is
+//    fused with the fp16 -> f32 conversion (mixed-precision adds);
+//  * the Walsh-Hadamard stages run in registers with packed f32x2 add/sub,
+//    then one or two shuffle stages across the lanes of a vector;
 //  * nearest level: q = w * (1 / (delta N)) + offset is floored through the
-//    2^23 round-down trick into a cell of a lane-replicated shared table that
-//    holds the one boundary inside the cell; one compare gives the index;
-//  * coordinates within TQ_GUARD_Z of a boundary are redone exactly in fp64
-//    by the whole warp (the f32 error bound is below that band), so the codes
-//    are those of exact arithmetic;
-//  * packed words are staged in the warp's shared output tile (rows
-//    contiguous, as in memory) and leave through one 1-D bulk store (TMA).
+//    2^23 round-down trick into a cell of a shared table (16 lane copies)
+//    that holds the one boundary inside the cell; one compare gives the index;
+//  * coordinates within the guard band of a boundary are redone exactly in
+//    fp64 by the whole warp (the f32 error bound is below the band), so the
+//    codes are those of exact arithmetic;
+//  * each lane stores its packed row with 128-bit stores (the 32 rows of a
+//    tile are contiguous in memory).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <atomic>
+#include <cstring>
 
 #include "tq_common.cuh"
 
 namespace tq {
 
-constexpr int ENC_WARPS = 16;
 constexpr int ENC_STAGES = 2;
-constexpr int ENC_C = 64;  // coordinates per lane
+constexpr int ENC_BOX_ROWS = 32;                                // lane-rows per tile
+constexpr int ENC_BOX_COLS = 64;                                // fp16 per box row: 128 bytes
+constexpr int ENC_BOX_BYTES = ENC_BOX_ROWS * ENC_BOX_COLS * 2;  // 4096
+constexpr int ENC_LUT_COPIES = 16;
 constexpr float MAGIC_2P23 = 8388608.0f;
+
+constexpr int ENC_CMAX = 64;  // coordinates per lane at most
 
 template <int D, int BITS>
 struct EncCfg {
-  static constexpr int C = ENC_C;
-  static constexpr int LPV = D / C;         // lanes per vector
-  static constexpr int NP = C / 2;          // f32x2 pairs per lane
-  static constexpr int VPW = 32 / LPV;      // vectors per warp tile
-  static constexpr int P = D * BITS / 8;    // packed bytes per vector
-  static constexpr int WL = C * BITS / 32;  // packed 32-bit words per lane
-  static constexpr int IN_ROW = 2 * C;       // input lane-row (contiguous tile)
-  static constexpr int OUT_ROW = WL;         // packed lane-row (contiguous tile, as in memory)
+  static constexpr int C = D < ENC_CMAX ? D : ENC_CMAX;  // coordinates per lane
+  static constexpr int LPV = D / C;            // lanes per vector
+  static constexpr int NP = C / 2;             // f32x2 pairs per lane
+  static constexpr int VPW = 32 / LPV;         // vectors per warp tile
+  static constexpr int P = D * BITS / 8;       // packed bytes per vector
+  static constexpr int PL = C * BITS / 8;      // packed bytes per lane-row
+  static constexpr int WL = C * BITS / 32;     // packed 32-bit words per lane
   static constexpr int L = 1 << BITS;
-  static constexpr int GROUPS = C / 32;  // guard groups of 32 coordinates
-  static constexpr int IN_STAGE = 32 * IN_ROW;
-  static constexpr int OUT_WORDS = 32 * OUT_ROW;
+  static constexpr int GROUPS = C / 32;        // guard groups of 32 coordinates
+  static constexpr int BOXES = C / ENC_BOX_COLS;
+  static constexpr int STAGE = BOXES * ENC_BOX_BYTES;
+  static constexpr int WARPS = C == 128 ? 8 : 16;
 };
 
 struct EncArgs {
-  const __half* x;
-  int64_t n;  // vectors
+  CUtensorMap tm_x;  // input as [n * lanes-per-vector rows, C] fp16, box 64 x 32, 128-byte swizzle
+  int64_t n;         // vectors
+  int64_t vec_base;  // index of vector 0 of this launch in the caller's tensor (append mode)
   uint8_t* packed;
   float* norms;
   const int32_t* slot;  // append mode when non-null
   int h;                // heads per sequence (append mode)
   int64_t s_max;        // cache positions per sequence (append mode)
   uint32_t* err;
-  int fault_inject;      // test hook: 1 = never issue the row copies
+  int fault_inject;      // test hook: 1 = never issue the tile copies
   long long wait_limit;  // bound on each mbarrier wait, SM cycles
 };
 
-// Shared memory layout (bytes), per CTA.
+// Shared memory, per CTA: fixed header, then (1024-byte aligned, for the
+// swizzle pattern) the warps' stage buffers, then the cell table.
 template <int D, int BITS>
 struct EncSmem {
   using Cfg = EncCfg<D, BITS>;
-  static constexpr int BAR = 0;                                            // warps x stages u64
-  static constexpr int MASK = 256;                                         // sign masks, LPV x 32 u32
-  static constexpr int SCR = MASK + 4 * 32 * 4;                            // per warp 32-float scratch
-  static constexpr int IN = SCR + ENC_WARPS * 32 * 4;                      // input stages
-  static constexpr int OUT = IN + ENC_WARPS * ENC_STAGES * Cfg::IN_STAGE;  // output rows
-  static constexpr int LUT = OUT + ENC_WARPS * Cfg::OUT_WORDS * 4;          // cell table
-  static size_t bytes(int cells) { return (size_t)LUT + (size_t)cells * 32 * 8; }
+  static constexpr int BAR = 0;                    // warps x stages u64
+  static constexpr int BND = 256;                  // boundaries in z units, f32
+  static constexpr int MASK = 320;                 // sign masks, D/2 u32
+  static constexpr int SCR = 1024;                 // per warp 32-float scratch
+  static constexpr int HEADER = SCR + 16 * 32 * 4;  // 3072
+  static constexpr int IN_BYTES = Cfg::WARPS * ENC_STAGES * Cfg::STAGE;
+  static size_t bytes(int cells) {
+    return (size_t)HEADER + 1024 + IN_BYTES + (size_t)cells * ENC_LUT_COPIES * 8;
+  }
 };
 
 TQ_DEV uint2 lds_u2(uint32_t addr) {
   uint2 r;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
   return r;
+}
+
+TQ_DEV uint4 lds_u4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
+}
+
+TQ_DEV uint16_t lds_u16(uint32_t addr) {
+  uint16_t r;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
+  return r;
+}
+
+TQ_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// (x0 + x1, x0 - x1) in f32 for the fp16 pair (x0, x1) in the low and high
+// halves of h2: one conversion and two mixed-precision (f16 op f32) adds of
+// sm_100, each rounded once, as the plain f32 sum and difference are.
+TQ_DEV f2 first_butterfly(uint32_t h2) {
+  const uint16_t x0 = (uint16_t)(h2 & 0xffffu), x1 = (uint16_t)(h2 >> 16);
+  float a1, s, d;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(a1) : "h"(x1));
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(s) : "h"(x0), "f"(a1));
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(x0), "f"(a1));
+  return make_float2(s, d);
 }
 
 // Pack code m (< 2^BITS) of coordinate i into the lane's word array.
@@ -102,27 +140,108 @@ TQ_DEV void put_code(uint32_t (&words)[WL], int i, uint32_t m) {
   if ((off & 31) + BITS > 32) words[(off >> 5) + 1] += m >> (32 - (off & 31));
 }
 
+// Replace code i (runtime index) by m in the lane's word array.
+template <int BITS, int WL>
+TQ_DEV void set_code(uint32_t (&words)[WL], int i, uint32_t m) {
+  const int off = i * BITS, w0 = off >> 5, sh = off & 31;
+  const uint32_t msk = (1u << BITS) - 1u;
+#pragma unroll
+  for (int w = 0; w < WL; ++w) {
+    if (w == w0) words[w] = (words[w] & ~(msk << sh)) | (m << sh);
+    if (w == w0 + 1 && sh + BITS > 32) words[w] = (words[w] & ~(msk >> (32 - sh))) | (m >> (32 - sh));
+  }
+}
+
+// Shared address of coordinate k (0 <= k < C) of lane-row r in a stage
+// written by the swizzled tensor copies: box k/64, 16-byte chunk
+// ((k/8) % 8) ^ (r % 8) of the row's 128 bytes.
+TQ_DEV uint32_t swz_addr(uint32_t stage_addr, int r, int k) {
+  return stage_addr + (uint32_t)(k >> 6) * ENC_BOX_BYTES + (uint32_t)r * 128u +
+         ((uint32_t)(((k >> 3) & 7) ^ (r & 7)) << 4) + (uint32_t)(k & 7) * 2u;
+}
+
+// Exact codes of the coordinates of one guard group of the source lane that
+// lie inside the guard band. On entry scratch[0..31] holds the group's 32
+// rotated f32 values (published by the source lane); on return scratch[j]
+// holds, as a uint32, the exact code of coordinate j for every bit j of the
+// returned mask. Called by the whole warp; rare, so kept out of line.
+template <int D, int BITS>
+__device__ __noinline__ uint32_t recheck_group(float* scratch, float srcR, float qoff, float gq, uint32_t lut_lane,
+                                               uint32_t st_addr, int row0, int gi0, const uint32_t* smask,
+                                               const float* sbound) {
+  constexpr int C = EncCfg<D, BITS>::C;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const float wj = scratch[lane];
+  // the same f32 arithmetic as the main pass gives the same flags and cells
+  const float q = fmaf(wj, srcR, qoff);
+  const uint32_t qb = __float_as_uint(__fadd_rd(q, MAGIC_2P23));
+  const uint2 ent = lds_u2(qb * 128u + lut_lane);
+  const float dlj = __uint_as_float(ent.x) - q;
+  const uint32_t cm = __ballot_sync(FULL, fabsf(dlj) < gq);
+  // N in fp64 from the fp16 inputs still in the stage
+  double sq = 0.0;
+#pragma unroll
+  for (int t = 0; t < D / 32; ++t) {
+    const int k = lane + 32 * t;
+    const double xk = (double)__half2float(__ushort_as_half(lds_u16(swz_addr(st_addr, row0 + k / C, k % C))));
+    sq = fma(xk, xk, sq);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(FULL, sq, o);
+  const double n64 = sqrt(sq);
+  uint32_t code = 0;
+  for (uint32_t c2 = cm; c2; c2 &= c2 - 1) {
+    const int j = __ffs(c2) - 1;
+    const int gi = gi0 + j;  // coordinate index in the vector
+    // w_gi = sum_k s_k (-1)^popcount(gi & k) x_k: exact in fp64 for fp16 x
+    double ps = 0.0;
+#pragma unroll
+    for (int t = 0; t < D / 32; ++t) {
+      const int k = lane + 32 * t;
+      const double xk = (double)__half2float(__ushort_as_half(lds_u16(swz_addr(st_addr, row0 + k / C, k % C))));
+      const uint32_t sbit = (smask[k >> 1] >> (15 + 16 * (k & 1))) & 1u;
+      const uint32_t neg = sbit ^ (uint32_t)(__popc(gi & k) & 1);
+      ps += neg ? -xk : xk;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(FULL, ps, o);
+    // the cell of coordinate j holds boundary number `below`; every other
+    // boundary is decided with a margin of 1/64 cell
+    const uint32_t below = __shfl_sync(FULL, ent.y, j);
+    const uint32_t m = below + ((ps >= (double)sbound[below] * n64) ? 1u : 0u);
+    if (lane == j) code = m;
+  }
+  __syncwarp();
+  reinterpret_cast<uint32_t*>(scratch)[lane] = code;
+  __syncwarp();
+  return cm;
+}
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(ENC_WARPS * 32, 1)
+__global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
     encode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ EncArgs a) {
   using Cfg = EncCfg<D, BITS>;
   using Sm = EncSmem<D, BITS>;
-  constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, VPW = Cfg::VPW, WL = Cfg::WL, L = Cfg::L;
+  constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, WL = Cfg::WL, L = Cfg::L;
+  constexpr int WARPS = Cfg::WARPS;
   constexpr uint32_t FULL = 0xffffffffu;
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t in_addr = (smem_base + Sm::HEADER + 1023u) & ~1023u;  // stages: 1024-byte aligned
+  const uint32_t lut_addr = in_addr + Sm::IN_BYTES;
 
-  // ---- lane-replicated cell table: entry (cell, lane) = {boundary bits, count below}
+  // ---- cell table: entry (cell, copy) = {boundary bits or 3e38 if none, count of boundaries below}
   {
-    uint2* lut = reinterpret_cast<uint2*>(smem + Sm::LUT);
+    uint2* lut = reinterpret_cast<uint2*>(smem + (lut_addr - smem_base));
     const int cells = T.lut_cells;
-    for (int e = threadIdx.x; e < cells * 32; e += blockDim.x) {
-      const int cell = e >> 5;
+    for (int e = threadIdx.x; e < cells * ENC_LUT_COPIES; e += blockDim.x) {
+      const int cell = e / ENC_LUT_COPIES;
       uint32_t below = 0;
-      float thr = 3.0e38f;  // no boundary in this cell
+      float thr = 3.0e38f;
 #pragma unroll
       for (int j = 0; j < L - 1; ++j) {
         const float t = T.tau[j];
@@ -134,6 +253,8 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       lut[e] = make_uint2(__float_as_uint(thr), below);
     }
   }
+  float* sbound = reinterpret_cast<float*>(smem + Sm::BND);
+  for (int j = threadIdx.x; j < L - 1; j += blockDim.x) sbound[j] = T.bounds[j];
   uint32_t* smask = reinterpret_cast<uint32_t*>(smem + Sm::MASK);
   for (int i = threadIdx.x; i < D / 2; i += blockDim.x) smask[i] = T.sign_h2[i];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::BAR) + warp * ENC_STAGES;
@@ -144,45 +265,38 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
   }
   __syncthreads();
 
-  uint8_t* in_stage0 = smem + Sm::IN + warp * ENC_STAGES * Cfg::IN_STAGE;
-  uint32_t* out_rows = reinterpret_cast<uint32_t*>(smem + Sm::OUT) + warp * Cfg::OUT_WORDS;
+  const uint32_t stage0 = in_addr + (uint32_t)(warp * ENC_STAGES * Cfg::STAGE);
   float* scratch = reinterpret_cast<float*>(smem + Sm::SCR) + warp * 32;
-  const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
-  const int part = lane & (LPV - 1);  // which 64-coordinate part of its vector this lane holds
-  const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
-  // chunk swizzle of this lane (shared by the lanes of a vector) and the
-  // code-word mask that mirrors the codes of chunks whose output sign it flips
-  const uint32_t swz = (uint32_t)(lane / LPV) & 7u;
-  uint32_t flipw[WL];
-#pragma unroll
-  for (int w = 0; w < WL; ++w) flipw[w] = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (__popc((uint32_t)j & swz) & 1) {
-#pragma unroll
-      for (int i = 8 * j; i < 8 * j + 8; ++i) put_code<BITS>(flipw, i, (uint32_t)(L - 1));
-    }
-  }
+  // (2^23 + cell) * 128 = 2^31 + cell * 128 (mod 2^32): the 2^31 is taken out here
+  const uint32_t lut_lane = lut_addr + (uint32_t)(lane & (ENC_LUT_COPIES - 1)) * 8u - 0x80000000u;
+  const int part = lane & (LPV - 1);  // which C-coordinate part of its vector this lane holds
+  const uint32_t sw = (uint32_t)lane & 7u;
+  const uint32_t row_off = (uint32_t)lane * 128u;
 
-  const int64_t n_tiles = (a.n + VPW - 1) / VPW;
-  const int64_t gw = (int64_t)blockIdx.x * ENC_WARPS + warp;
-  const int64_t n_warps = (int64_t)gridDim.x * ENC_WARPS;
+  // a launch covers fewer than 2^30 lane-rows: tile and row indices fit in int32
+  const int n_rows = (int)(a.n * LPV);
+  const int n_tiles = (n_rows + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
+  // warps numbered SM-minor, so a partial last round of tiles spreads over all SMs
+  const int gw = warp * (int)gridDim.x + (int)blockIdx.x;
+  const int n_warps = (int)gridDim.x * WARPS;
 
-  auto issue = [&](int64_t tile, int stage) {  // called by the whole warp
-    const int64_t v0 = tile * VPW;
-    const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
+  auto issue = [&](int tile, int stage) {  // called by the whole warp
     if (lane == 0) {
       const uint32_t bar = smem_u32(&bars[stage]);
-      const uint32_t bytes = (uint32_t)(valid_lanes * 2 * C);
-      mbar_arrive_expect_tx(bar, bytes);
-      if (!a.fault_inject) bulk_g2s(smem_u32(in_stage0 + stage * Cfg::IN_STAGE), a.x + v0 * D, bytes, bar);
+      mbar_arrive_expect_tx(bar, (uint32_t)Cfg::STAGE);  // full boxes: rows past the end are zero-filled
+      if (!a.fault_inject) {
+#pragma unroll
+        for (int b = 0; b < Cfg::BOXES; ++b)
+          tma_load_2d(stage0 + (uint32_t)(stage * Cfg::STAGE + b * ENC_BOX_BYTES), &a.tm_x, b * ENC_BOX_COLS,
+                      tile * ENC_BOX_ROWS, bar);
+      }
     }
     __syncwarp();
   };
 
 #pragma unroll
   for (int s = 0; s < ENC_STAGES; ++s) {
-    const int64_t t = gw + s * n_warps;
+    const int t = gw + s * n_warps;
     if (t < n_tiles) issue(t, s);
   }
 
@@ -192,49 +306,48 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
 
   int stage = 0;
   uint32_t parity = 0;  // bit s: parity of the next completion of stage s
-  bool stored_once = false;
-  for (int64_t tile = gw; tile < n_tiles; tile += n_warps) {
-    const int64_t v0 = tile * VPW;
-    const int valid_lanes = (int)min64(VPW, a.n - v0) * LPV;
+  for (int tile = gw; tile < n_tiles; tile += n_warps) {
+    const int r0 = tile * ENC_BOX_ROWS;  // first lane-row of the tile
+    const int valid_rows = min(ENC_BOX_ROWS, n_rows - r0);
     // every lane polls; the warp acts on one agreed outcome
     const bool ok = __all_sync(FULL, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.wait_limit));
     if (!ok) {
       if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
       // give the copies already issued into the other stage a bounded time to land
-#pragma unroll
-      for (int s = 1; s < ENC_STAGES; ++s) {
-        const int os = (stage + s) % ENC_STAGES;
-        if (tile + s * n_warps < n_tiles)
-          (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
-      }
-      if (lane == 0) bulk_wait_all<0>();
+      const int os = stage ^ 1;
+      if (tile + n_warps < n_tiles) (void)mbar_wait_bounded(smem_u32(&bars[os]), (parity >> os) & 1u, a.wait_limit);
       return;
     }
     parity ^= 1u << stage;
-    const bool active = lane < valid_lanes;
-    const uint8_t* my_row = in_stage0 + stage * Cfg::IN_STAGE + lane * Cfg::IN_ROW;
+    const bool active = lane < valid_rows;
+    const uint32_t st_addr = stage0 + (uint32_t)(stage * Cfg::STAGE);
+    const uint32_t my_row = st_addr + row_off;
 
-    // ---- load (slot c <- chunk c ^ swz), sign flip (XOR of fp16 sign bits), first butterfly stage
+    // ---- load, sign flip (XOR of fp16 sign bits), first butterfly stage
     f2 v[NP];
-#pragma unroll
-    for (int c = 0; c < C / 8; ++c) {
-      const uint32_t ch = (uint32_t)c ^ swz;
-      uint4 r = make_uint4(0, 0, 0, 0);
-      if (active) r = *reinterpret_cast<const uint4*>(my_row + 16 * ch);
-      const uint4 mk = my_masks[ch];
-      const uint32_t w4[4] = {r.x ^ mk.x, r.y ^ mk.y, r.z ^ mk.z, r.w ^ mk.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[q]));
-        v[4 * c + q] = make_float2(f.x + f.y, f.x - f.y);
-      }
-    }
-    // ---- sum of squares: (x0+x1)^2 + (x0-x1)^2 = 2 (x0^2 + x1^2); 8 chains
     f2 acc[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[j] = mul2(v[j], v[j]);
+    for (int b = 0; b < Cfg::BOXES; ++b) {
 #pragma unroll
-    for (int k = 4; k < NP; ++k) acc[k & 3] = fma2(v[k], v[k], acc[k & 3]);
+      for (int c = 0; c < 8; ++c) {
+        const uint4 r = lds_u4(my_row + (uint32_t)(b * ENC_BOX_BYTES) + ((c ^ sw) << 4));
+        const int k0 = b * 32 + c * 4;  // first pair of the chunk
+        uint4 mk;
+        if constexpr (LPV == 1) {
+          mk = make_uint4(T.sign_h2[k0], T.sign_h2[k0 + 1], T.sign_h2[k0 + 2], T.sign_h2[k0 + 3]);
+        } else {
+          mk = *reinterpret_cast<const uint4*>(smask + part * NP + k0);
+        }
+        const uint32_t w4[4] = {r.x ^ mk.x, r.y ^ mk.y, r.z ^ mk.z, r.w ^ mk.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          v[k0 + q] = first_butterfly(w4[q]);
+          // sum of squares as the pairs arrive: (x0+x1)^2 + (x0-x1)^2 = 2 (x0^2 + x1^2);
+          // 8 chains of at most 16 terms
+          acc[q] = (k0 == 0) ? mul2(v[q], v[q]) : fma2(v[k0 + q], v[k0 + q], acc[q]);
+        }
+      }
+    }
     const f2 s4 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
     float sum2 = s4.x + s4.y;
 #pragma unroll
@@ -255,155 +368,91 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
       }
     }
 
-    // ---- quantize + pack
+    // ---- quantize + pack, 32 coordinates (one guard group) at a time; a
+    // group with a coordinate inside the guard band is redone at once, while
+    // its rotated values are still in registers
     const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite vector
     const float R = special ? 0.f : __fdiv_rn(Rscale, nrm);
     uint32_t words[WL];
 #pragma unroll
     for (int w = 0; w < WL; ++w) words[w] = 0;
-    uint32_t gmask = 0;
-    if (!special) {
-      const f2 R2 = make_float2(R, R), Q2 = make_float2(qoff, qoff), M2 = make_float2(MAGIC_2P23, MAGIC_2P23);
+    const f2 R2 = make_float2(R, R), Q2 = make_float2(qoff, qoff), M2 = make_float2(MAGIC_2P23, MAGIC_2P23);
 #pragma unroll
-      for (int g = 0; g < Cfg::GROUPS; ++g) {
-        float gmin = 3.0e38f;  // closest approach to a boundary in this group (q units)
+    for (int g = 0; g < Cfg::GROUPS; ++g) {
+      float gmin = 3.0e38f;  // closest approach to a boundary in this group (q units)
+      if (!special) {
 #pragma unroll
         for (int k = g * 16; k < g * 16 + 16; ++k) {
           const f2 q2 = fma2(v[k], R2, Q2);
-          const f2 qm = add2_rm(q2, M2);
+          const f2 qm = add2_rm(q2, M2);  // bits: 2^23 + floor(q)
+          float dl[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const float q = e ? q2.y : q2.x;
             const uint32_t qb = __float_as_uint(e ? qm.y : qm.x);
-            const uint2 ent = lds_u2(qb * 256u + lut_lane);
-            const float dl = __uint_as_float(ent.x) - q;
-            gmin = fminf(gmin, fabsf(dl));
-            put_code<BITS>(words, 2 * k + e, ent.y + (__float_as_uint(dl) >> 31));
+            const uint2 ent = lds_u2(qb * 128u + lut_lane);
+            dl[e] = __uint_as_float(ent.x) - q;
+            put_code<BITS>(words, 2 * k + e, ent.y + (__float_as_uint(dl[e]) >> 31));
           }
+          gmin = fminf(gmin, fminf(fabsf(dl[0]), fabsf(dl[1])));
         }
-        gmask |= (gmin < gq) ? (1u << g) : 0u;
+      } else {
+#pragma unroll
+        for (int i = g * 32; i < g * 32 + 32; ++i) put_code<BITS>(words, i, (uint32_t)(L / 2));
       }
-    } else {
+      // ---- exact recheck of the coordinates of this group inside the guard band (rare)
+      uint32_t any = __ballot_sync(FULL, active && gmin < gq);
+      while (any) {
+        const int src = __ffs(any) - 1;
+        any &= any - 1;
+        const float srcR = __shfl_sync(FULL, R, src);
+        const int src_part = src & (LPV - 1);
+        const int row0 = src - src_part;  // lane-row of part 0 of the source vector
+        // the source lane publishes the group's 32 rotated values
+        if (lane == src) {
 #pragma unroll
-      for (int i = 0; i < C; ++i) put_code<BITS>(words, i, (uint32_t)(L / 2));
-    }
-    if (!active) gmask = 0;
-    // the previous tile's bulk store must have finished reading the staging tile
-    if (lane == 0 && stored_once) bulk_wait_read<0>();
-    __syncwarp();
-#pragma unroll
-    for (int w = 0; w < WL; ++w) words[w] ^= special ? 0u : flipw[w];
-    if (WL % 4 == 0) {
-#pragma unroll
-      for (int w = 0; w < WL; w += 4)
-        *reinterpret_cast<uint4*>(out_rows + lane * WL + w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
-    } else {
-#pragma unroll
-      for (int w = 0; w < WL; w += 2)
-        *reinterpret_cast<uint2*>(out_rows + lane * WL + w) = make_uint2(words[w], words[w + 1]);
-    }
-
-    // ---- exact recheck of the coordinates inside the guard band (rare)
-    uint32_t any = __ballot_sync(FULL, gmask != 0);
-    while (any) {
-      const int src = __ffs(any) - 1;
-      any &= any - 1;
-      uint32_t sg = __shfl_sync(FULL, gmask, src);
-      const float srcR = __shfl_sync(FULL, R, src);
-      const int src_part = src & (LPV - 1);
-      const int vec_lane0 = src - src_part;
-      while (sg) {
-        const int g = __ffs(sg) - 1;
-        sg &= sg - 1;
-        // the source lane publishes the 32 rotated values of group g (their
-        // signs may be flipped by its chunk swizzle: the flags are symmetric)
-#pragma unroll
-        for (int gg = 0; gg < Cfg::GROUPS; ++gg) {
-          if (gg == g && lane == src) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              scratch[2 * k] = v[gg * 16 + k].x;
-              scratch[2 * k + 1] = v[gg * 16 + k].y;
-            }
+          for (int k = 0; k < 16; ++k) {
+            scratch[2 * k] = v[g * 16 + k].x;
+            scratch[2 * k + 1] = v[g * 16 + k].y;
           }
         }
         __syncwarp();
-        const float wj = scratch[lane];
-        __syncwarp();
-        // the same f32 arithmetic as the main pass gives the same flags
-        const float q = fmaf(wj, srcR, qoff);
-        const uint32_t qb = __float_as_uint(__fadd_rd(q, MAGIC_2P23));
-        const uint2 ent = lds_u2(qb * 256u + lut_lane);
-        const float dl = __uint_as_float(ent.x) - q;
-        uint32_t cm = __ballot_sync(FULL, fabsf(dl) < gq);
-        while (cm) {
-          const int j = __ffs(cm) - 1;
-          cm &= cm - 1;
-          const int i_local = g * 32 + j;
-          const int gi = src_part * C + i_local;  // coordinate index in the vector
-          // w_gi = sum_k s_k (-1)^popcount(gi & k) x_k: exact in fp64 for fp16 x
-          double part_sum = 0.0, sq = 0.0;
-#pragma unroll
-          for (int t = 0; t < D / 32; ++t) {
-            const int kk = lane + 32 * t;
-            const __half hx = reinterpret_cast<const __half*>(
-                in_stage0 + stage * Cfg::IN_STAGE + vec_lane0 * Cfg::IN_ROW)[kk];
-            const double xk = (double)__half2float(hx);
-            const uint32_t sbit = (smask[kk >> 1] >> (15 + 16 * (kk & 1))) & 1u;
-            const uint32_t neg = sbit ^ (uint32_t)(__popc(gi & kk) & 1);
-            part_sum += neg ? -xk : xk;
-            sq = fma(xk, xk, sq);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            part_sum += __shfl_xor_sync(FULL, part_sum, o);
-            sq += __shfl_xor_sync(FULL, sq, o);
-          }
-          const double n64 = sqrt(sq);
-          uint32_t m = 0;
-#pragma unroll
-          for (int jj = 0; jj < L - 1; ++jj) m += (part_sum >= (double)T.bounds[jj] * n64) ? 1u : 0u;
-          if (lane == 0) {
-            const int off = i_local * BITS;
-            uint32_t* row = out_rows + src * Cfg::OUT_ROW;
-            const uint32_t msk = (uint32_t)(L - 1);
-            row[off >> 5] = (row[off >> 5] & ~(msk << (off & 31))) | (m << (off & 31));
-            if ((off & 31) + BITS > 32) {
-              const int sh = 32 - (off & 31);
-              row[(off >> 5) + 1] = (row[(off >> 5) + 1] & ~(msk >> sh)) | (m >> sh);
-            }
+        const uint32_t cm = recheck_group<D, BITS>(scratch, srcR, qoff, gq, lut_lane, st_addr, row0,
+                                                   src_part * C + g * 32, smask, sbound);
+        if (lane == src) {
+          for (uint32_t c2 = cm; c2; c2 &= c2 - 1) {
+            const int j = __ffs(c2) - 1;
+            set_code<BITS>(words, g * 32 + j, reinterpret_cast<const uint32_t*>(scratch)[j]);
           }
         }
+        __syncwarp();
       }
     }
-    __syncwarp();
 
-    // ---- write the tile
+    // ---- write the tile: each lane its packed row (rows of a tile are contiguous)
     if (a.slot == nullptr) {
-      const uint32_t bytes = (uint32_t)(valid_lanes * WL * 4);
-      if (bytes % 16 == 0) {  // always for full tiles; 1-D bulk copies move multiples of 16 bytes
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          bulk_s2g(a.packed + v0 * Cfg::P, smem_u32(out_rows), bytes);
-          bulk_commit();
+      if (active) {
+        uint8_t* dst = a.packed + (int64_t)(r0 + lane) * Cfg::PL;
+        if constexpr (Cfg::PL % 16 == 0) {
+#pragma unroll
+          for (int w = 0; w < WL; w += 4)
+            *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+        } else {
+#pragma unroll
+          for (int w = 0; w < WL; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
         }
-        stored_once = true;
-      } else {  // a partial tile of 24-byte rows: plain coalesced stores
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + v0 * Cfg::P);
-        for (int w = lane; w < valid_lanes * WL; w += 32) dst[w] = out_rows[w];
+        if (part == 0) a.norms[(r0 + lane) / LPV] = nrm;
       }
-      if (active && part == 0) a.norms[v0 + lane / LPV] = nrm;
     } else if (active) {
-      const int64_t r = v0 + lane / LPV;
+      const int64_t r = a.vec_base + (r0 + lane) / LPV;
       const int64_t seq = r / a.h;
       const int head = (int)(r - seq * a.h);
       const int32_t s = a.slot[seq];
       if (s >= 0 && s < a.s_max) {
         const int64_t drow = (seq * a.s_max + s) * a.h + head;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + drow * Cfg::P) + part * WL;
+        uint8_t* dst = a.packed + drow * Cfg::P + part * Cfg::PL;
 #pragma unroll
-        for (int w = 0; w < WL; ++w) dst[w] = out_rows[lane * Cfg::OUT_ROW + w];
+        for (int w = 0; w < WL; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
         if (part == 0) a.norms[drow] = nrm;
       } else if (part == 0) {
         record_error(a.err, TQ_DEVERR_SLOT_RANGE);
@@ -412,15 +461,14 @@ __global__ void __launch_bounds__(ENC_WARPS * 32, 1)
     __syncwarp();
 
     // ---- refill this stage
-    const int64_t next = tile + ENC_STAGES * n_warps;
+    const int next = tile + ENC_STAGES * n_warps;
     if (next < n_tiles) issue(next, stage);
-    if (++stage == ENC_STAGES) stage = 0;
+    stage ^= 1;
   }
-  if (lane == 0) bulk_wait_all<0>();
 }
 
 template <int D, int BITS>
-static cudaError_t launch_encode_t(const tq_codec_tables& T, const EncArgs& a, cudaStream_t st) {
+static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const void* x, cudaStream_t st) {
   using Cfg = EncCfg<D, BITS>;
   const size_t smem = EncSmem<D, BITS>::bytes(T.lut_cells);
   int dev = 0;
@@ -433,11 +481,38 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, const EncArgs& a, c
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  const int64_t tiles = (a.n + Cfg::VPW - 1) / Cfg::VPW;
-  const int64_t ctas_needed = (tiles + ENC_WARPS - 1) / ENC_WARPS;
-  const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)tq_sm_count(dev));
-  encode_kernel<D, BITS><<<grid, ENC_WARPS * 32, smem, st>>>(T, a);
-  return cudaGetLastError();
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
+  if (!enc) return cudaErrorNotSupported;
+  // launches of at most 2^30 lane-rows keep the copy coordinates in int32
+  const int64_t max_vec = ((int64_t)1 << 30) / Cfg::LPV;
+  const int64_t n_total = a.n;
+  uint8_t* packed0 = a.packed;
+  float* norms0 = a.norms;
+  for (int64_t off = 0; off < n_total; off += max_vec) {
+    const int64_t n = std::min(max_vec, n_total - off);
+    a.n = n;
+    a.vec_base = off;
+    if (a.slot == nullptr) {
+      a.packed = packed0 + off * Cfg::P;
+      a.norms = norms0 + off;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)Cfg::C, (cuuint64_t)(n * Cfg::LPV)};
+    const cuuint64_t strides[1] = {(cuuint64_t)Cfg::C * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)ENC_BOX_COLS, (cuuint32_t)ENC_BOX_ROWS};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&a.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(static_cast<const void*>(static_cast<const __half*>(x) + off * D)), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+    const int64_t tiles = (n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
+    const int64_t ctas_needed = (tiles + Cfg::WARPS - 1) / Cfg::WARPS;
+    const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)tq_sm_count(dev));
+    encode_kernel<D, BITS><<<grid, Cfg::WARPS * 32, smem, st>>>(T, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tq
@@ -448,7 +523,7 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
                            const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject) {
   if (n == 0) return TQ_OK;
   EncArgs a;
-  a.x = static_cast<const __half*>(x);
+  memset(&a, 0, sizeof(a));
   a.n = n;
   a.packed = static_cast<uint8_t*>(packed);
   a.norms = norms;
@@ -463,7 +538,7 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
   cudaError_t e = cudaErrorInvalidValue;
   const tq_codec_tables& T = ctx->t;
 #define TQ_ENC_CASE(D_, B_) \
-  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_>(T, a, st);
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_>(T, a, x, st);
   TQ_ENC_CASE(64, 2) TQ_ENC_CASE(64, 3) TQ_ENC_CASE(64, 4)
   TQ_ENC_CASE(128, 2) TQ_ENC_CASE(128, 3) TQ_ENC_CASE(128, 4)
   TQ_ENC_CASE(256, 2) TQ_ENC_CASE(256, 3) TQ_ENC_CASE(256, 4)

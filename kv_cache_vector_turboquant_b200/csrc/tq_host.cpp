@@ -148,7 +148,7 @@ tq_status tq_create(int head_dim, int bits, uint64_t seed, tq_ctx** out) {
   t.inv_delta = (float)(1.0 / delta);
   t.q_offset = (float)(K + frac);
   t.lut_cells = 2 * K + 2;
-  t.guard_q = (float)(TQ_GUARD_Z / delta);
+  t.guard_q = (float)(tq_guard_z(head_dim) / delta);
   for (int j = 0; j < L - 1; ++j) t.tau[j] = (float)(t.bounds[j] / delta + (K + frac));
   *out = c;
   return TQ_OK;

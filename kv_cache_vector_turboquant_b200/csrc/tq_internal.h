@@ -40,10 +40,11 @@ struct tq_ctx {
 
 // Guard band of the encode quantizer in z units (N(0,1) scale). The f32 path
 // decides every coordinate whose scaled rotated value is farther than this
-// from a boundary; the f32 rounding error bound is below 1.1e-5 for
-// head_dim <= 256 (see the error analysis in the design notes), so those
-// decisions equal the exact ones. Closer coordinates are redone in fp64.
-#define TQ_GUARD_Z 2.0e-5
+// from a boundary; the f32 rounding error bound, u((log2 d + 1) sqrt(d) + 38)
+// with u = 2^-24, is 5.6e-6 at head_dim 64, 7.7e-6 at 128 and 1.1e-5 at 256,
+// below the band, so those decisions equal the exact ones. Closer
+// coordinates are redone in fp64.
+inline double tq_guard_z(int head_dim) { return head_dim <= 128 ? 1.0e-5 : 2.0e-5; }
 
 // Kernel launchers (defined in the .cu files). Arguments are validated by the
 // ABI layer before these are called.
@@ -56,6 +57,9 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
                            const float* v_norms, int64_t s_max, const int32_t* positions, void* out,
                            void* workspace, size_t ws_bytes, void* stream);
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max);
+
+// cuTensorMapEncodeTiled from the driver (cached; null if unavailable).
+void* tq_tensor_map_encode_fn(void);
 
 // Number of SMs of device `dev` (cached).
 int tq_sm_count(int dev);
