@@ -140,6 +140,64 @@ def test_llama_layer_full_size_sampled(K, W, bits):
     assert K.tq_device_error()[0] == K.TQ_OK
 
 
+@pytest.mark.parametrize("layer", [0, 41, 79])
+def test_long_context_layer_sampled(K, W, layer):
+    """Layers of the 80-layer long-context cache at 3 bits: K and V
+    [1, 131072, 8, 128] with log-normal per-channel scales, encoded whole on
+    the GPU; 4096 sampled rows per tensor against the oracle (codes, norms,
+    decode of the same bytes)."""
+    kx, vx = W.long_context_layer(layer)
+    tq = K.TurboQuant(128, 3)
+    g = torch.Generator().manual_seed(1000 + layer)
+    for x in (kx, vx):
+        flat = x.reshape(-1, 128)
+        packed, norms = tq.encode(flat)
+        dec = tq.decode(packed, norms)
+        torch.cuda.synchronize()
+        rows = torch.randperm(flat.shape[0], generator=g)[:4096].sort().values.cuda()
+        xs = flat[rows].cpu().numpy()
+        det = O.encode_detail(xs, 3, 42)
+        gp, gn = packed[rows].cpu().numpy(), norms[rows].cpu().numpy()
+        assert code_mismatches(gp, det, 3, 128) == 0
+        assert_norms(gn, det)
+        assert_decode_ulp(dec[rows].cpu().numpy(), O.decode(gp, gn, 3, 42, 128))
+        del packed, norms, dec
+    assert K.tq_device_error()[0] == K.TQ_OK
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_append_replayed_from_cuda_graph(K, W, d):
+    """The streaming append captured once in a CUDA graph (32 steps, K and V)
+    and replayed writes the same bytes as the eager calls."""
+    n_seq, h, s_max, steps, bits = 256, 8, 32, 32, 4
+    tq = K.TurboQuant(d, bits)
+    P = tq.packed_bytes
+    toks = W.append_stream(run=7 + d, steps=steps, n_seq=n_seq, H=h, d=d)
+    slots = torch.arange(steps, dtype=torch.int32, device="cuda")[:, None].expand(steps, n_seq).contiguous()
+    caches = [(torch.zeros(n_seq, s_max, h, P, dtype=torch.uint8, device="cuda"),
+               torch.zeros(n_seq, s_max, h, dtype=torch.float32, device="cuda")) for _ in range(2)]
+    tq.encode_append(toks[0], caches[0][0], caches[0][1], slots[0])  # one eager call before capture
+    torch.cuda.synchronize()
+    caches[0][0].zero_()
+    caches[0][1].zero_()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            for s in range(steps):
+                tq.encode_append(toks[s], caches[1][0], caches[1][1], slots[s])
+    torch.cuda.current_stream().wait_stream(stream)
+    graph.replay()
+    for s in range(steps):
+        tq.encode_append(toks[s], caches[0][0], caches[0][1], slots[s])
+    torch.cuda.synchronize()
+    assert torch.equal(caches[0][0], caches[1][0])
+    assert torch.equal(caches[0][1], caches[1][1])
+    assert K.tq_device_error()[0] == K.TQ_OK
+    del graph
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_append_matches_bulk_encode(K, W, d, bits):
