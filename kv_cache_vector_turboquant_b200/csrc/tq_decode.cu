@@ -15,16 +15,18 @@
 // per tile); a lane-replicated table indexed by two codes returns
 // (c[a] + c[b], c[a] - c[b]), the levels already through the first
 // butterfly; the other stages run in registers with f32x2 add/sub and
-// shuffles across the lanes of a vector. The lane negates the levels of the
-// chunks j with popcount(j & s) odd (mirroring their codes, the codebook is
-// symmetric), which makes the transform deliver natural chunk c ^ s in
-// register slot c; so its 16-byte stores into the warp's 4 KB output tile are
-// free of bank conflicts while the tile itself is in natural order and leaves
-// through one 1-D bulk store (TMA) per tile.
+// shuffles across the lanes of a vector. The fp16 rows are staged in the
+// warp's 4 KB output tile in the 128-byte swizzled layout (16-byte chunk c of
+// row r at position c ^ (r % 8): conflict-free stores of natural chunks) and
+// leave through one 2-D tensor store (TMA) per tile, which also clips a
+// partial last tile.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <atomic>
+#include <cstring>
 
 #include "tq_common.cuh"
 
@@ -50,19 +52,24 @@ struct DecCfg {
   static constexpr int OUT = 32 * 2 * C;                  // the warp's output tile (4 KB)
 };
 
+// Shared memory: header, input stages, then (1024-byte aligned, for the
+// swizzle pattern of the tensor store) the warps' output tiles and the pair
+// table. The dynamic window's base is only 16-byte aligned, so the kernel
+// rounds the output region up at run time (1 KB of slack is reserved).
 template <int D, int BITS>
 struct DecSmem {
   using Cfg = DecCfg<D, BITS>;
   static constexpr int BAR = 0;     // warps x stages u64
   static constexpr int MASK = 512;  // sign masks, up to 128 u32
   static constexpr int IN = MASK + 512;
-  static constexpr int OUT = IN + DEC_WARPS * DEC_STAGES * ((Cfg::IN_STAGE + 15) / 16 * 16);
-  static constexpr int LUT = OUT + DEC_WARPS * Cfg::OUT;
-  static constexpr size_t BYTES = (size_t)LUT + (size_t)Cfg::E * 32 * 8;
   static constexpr int STAGE = (Cfg::IN_STAGE + 15) / 16 * 16;
+  static constexpr int OUT = IN + DEC_WARPS * DEC_STAGES * STAGE;  // before rounding up to 1024
+  static constexpr int OUT_BYTES = DEC_WARPS * Cfg::OUT;
+  static constexpr size_t BYTES = (size_t)OUT + 1024 + OUT_BYTES + (size_t)Cfg::E * 32 * 8;
 };
 
 struct DecArgs {
+  CUtensorMap tm_x;  // output as [n * lanes-per-vector rows, 64] fp16, box 64 x 32, 128-byte swizzle
   const uint8_t* packed;
   const float* norms;
   int64_t n;
@@ -71,6 +78,13 @@ struct DecArgs {
   long long wait_limit;
   int norms_bulk;  // norms pointer 16-byte aligned: norms tiles come by bulk copy
 };
+
+TQ_DEV void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
 
 TQ_DEV f2 lds_f2(uint32_t addr) {
   f2 r;
@@ -90,11 +104,14 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t out_addr = (smem_base + Sm::OUT + 1023u) & ~1023u;
+  const uint32_t lut_addr = out_addr + Sm::OUT_BYTES;
 
   // pair table: entry (f, lane) with f = code_a | code_b << BITS holds
   // (c[a] + c[b], c[a] - c[b]) -- exact in f32 (2^-14 grid).
   {
-    f2* lut = reinterpret_cast<f2*>(smem + Sm::LUT);
+    f2* lut = reinterpret_cast<f2*>(smem + (lut_addr - smem_base));
     for (int e = threadIdx.x; e < E * 32; e += blockDim.x) {
       const int f = e >> 5;
       const float ca = T.levels[f & ((1 << BITS) - 1)];
@@ -113,29 +130,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   __syncthreads();
 
   uint8_t* in0 = smem + Sm::IN + warp * DEC_STAGES * Sm::STAGE;
-  uint8_t* otile = smem + Sm::OUT + warp * Cfg::OUT;
-  uint8_t* orow = otile + lane * 2 * C;
-  const uint32_t lut_lane = smem_u32(smem + Sm::LUT) + lane * 8u;
+  const uint32_t otile = out_addr + (uint32_t)(warp * Cfg::OUT);
+  uint8_t* orow = smem + (otile - smem_base) + lane * 2 * C;
+  const uint32_t sw = (uint32_t)lane & 7u;  // swizzle of this lane's output row
+  const uint32_t lut_lane = lut_addr + lane * 8u;
   const int part = lane & (LPV - 1);
   const uint4* my_masks = reinterpret_cast<const uint4*>(smask + part * NP);
-  // chunk swizzle (shared by the lanes of a vector) and the code bits to
-  // mirror so that register slot c receives natural output chunk c ^ swz
-  const uint32_t swz = (uint32_t)(lane / LPV) & 7u;
-  uint32_t flipw[WL];
-#pragma unroll
-  for (int w = 0; w < WL; ++w) flipw[w] = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (__popc((uint32_t)j & swz) & 1) {
-#pragma unroll
-      for (int i = 8 * j; i < 8 * j + 8; ++i) {
-        const int off = i * BITS;
-        const uint32_t m = (1u << BITS) - 1u;
-        flipw[off >> 5] |= m << (off & 31);
-        if ((off & 31) + BITS > 32) flipw[(off >> 5) + 1] |= m >> (32 - (off & 31));
-      }
-    }
-  }
 
   const int64_t n_tiles = (a.n + VPW - 1) / VPW;
   const int64_t gw = (int64_t)blockIdx.x * DEC_WARPS + warp;
@@ -218,8 +218,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         nrm = __ldg(a.norms + v0 + vl);
       }
     }
-#pragma unroll
-    for (int w = 0; w < WL; ++w) words[w] ^= flipw[w];
     __syncwarp();
     // the stage has been read into registers: refill it
     {
@@ -259,8 +257,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
-      const uint32_t ch = (uint32_t)c ^ swz;  // natural chunk held in slot c
-      const uint4 mk = my_masks[ch];
+      uint4 mk;
+      if constexpr (LPV == 1) {
+        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
+      } else {
+        mk = my_masks[c];
+      }
       const uint32_t m4[4] = {mk.x, mk.y, mk.z, mk.w};
       uint32_t h[4];
 #pragma unroll
@@ -269,12 +271,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
         const __half2 hv = __floats2half2_rn(y.x, y.y);
         h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ m4[q];
       }
-      *reinterpret_cast<uint4*>(orow + 16 * ch) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4*>(orow + 16 * (c ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      bulk_s2g(a.x + v0 * D, smem_u32(otile), (uint32_t)(valid_lanes * 2 * C));
+      // rows past the end of a partial tile are clipped by the tensor store
+      tma_store_2d(&a.tm_x, 0, (int)(tile * 32), otile);
       bulk_commit();
       stored_once = true;
     }
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 }
 
 template <int D, int BITS>
-static cudaError_t launch_decode_t(const tq_codec_tables& T, const DecArgs& a, cudaStream_t st) {
+static cudaError_t launch_decode_t(const tq_codec_tables& T, DecArgs a, cudaStream_t st) {
   using Cfg = DecCfg<D, BITS>;
   constexpr size_t smem = DecSmem<D, BITS>::BYTES;
   int dev = 0;
@@ -297,11 +300,37 @@ static cudaError_t launch_decode_t(const tq_codec_tables& T, const DecArgs& a, c
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  const int64_t tiles = (a.n + Cfg::VPW - 1) / Cfg::VPW;
-  const int64_t ctas = (tiles + DEC_WARPS - 1) / DEC_WARPS;
-  const int grid = (int)std::min<int64_t>(ctas, (int64_t)tq_sm_count(dev));
-  decode_kernel<D, BITS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
-  return cudaGetLastError();
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
+  if (!enc) return cudaErrorNotSupported;
+  // launches of at most 2^30 lane-rows keep the store coordinates in int32
+  const int64_t max_vec = ((int64_t)1 << 30) / Cfg::LPV;
+  const int64_t n_total = a.n;
+  const uint8_t* packed0 = a.packed;
+  const float* norms0 = a.norms;
+  __half* x0 = a.x;
+  for (int64_t off = 0; off < n_total; off += max_vec) {
+    const int64_t n = std::min(max_vec, n_total - off);
+    a.n = n;
+    a.packed = packed0 + off * Cfg::P;
+    a.norms = norms0 + off;
+    a.x = x0 + off * D;
+    a.norms_bulk = (reinterpret_cast<uintptr_t>(a.norms) & 15u) == 0;
+    const cuuint64_t dims[2] = {(cuuint64_t)Cfg::C, (cuuint64_t)(n * Cfg::LPV)};
+    const cuuint64_t strides[1] = {(cuuint64_t)Cfg::C * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)Cfg::C, 32u};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&a.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<void*>(a.x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+    const int64_t tiles = (n + Cfg::VPW - 1) / Cfg::VPW;
+    const int64_t ctas = (tiles + DEC_WARPS - 1) / DEC_WARPS;
+    const int grid = (int)std::min<int64_t>(ctas, (int64_t)tq_sm_count(dev));
+    decode_kernel<D, BITS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tq
@@ -312,6 +341,7 @@ tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* n
                            void* stream) {
   if (n == 0) return TQ_OK;
   DecArgs a;
+  memset(&a, 0, sizeof(a));
   a.packed = static_cast<const uint8_t*>(packed);
   a.norms = norms;
   a.n = n;
@@ -319,7 +349,6 @@ tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* n
   a.err = tq_error_word();
   if (!a.err) return TQ_ERR_CUDA;
   a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
-  a.norms_bulk = (reinterpret_cast<uintptr_t>(norms) & 15u) == 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorInvalidValue;
 #define TQ_DEC_CASE(D_, B_) \
