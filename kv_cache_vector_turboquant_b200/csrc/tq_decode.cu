@@ -257,19 +257,22 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
-      uint4 mk;
-      if constexpr (LPV == 1) {
-        mk = make_uint4(T.sign_h2[4 * c], T.sign_h2[4 * c + 1], T.sign_h2[4 * c + 2], T.sign_h2[4 * c + 3]);
-      } else {
-        mk = my_masks[c];
-      }
-      const uint32_t m4[4] = {mk.x, mk.y, mk.z, mk.w};
       uint32_t h[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const f2 y = mul2(v[4 * c + q], sc2);
         const __half2 hv = __floats2half2_rn(y.x, y.y);
-        h[q] = *reinterpret_cast<const uint32_t*>(&hv) ^ m4[q];
+        h[q] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+      if constexpr (LPV <= 2) {  // masks from the constant bank
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          h[q] ^= T.sign_h2[4 * c + q];
+          if (LPV == 2 && part) h[q] ^= T.sign_h2_dx[4 * c + q];
+        }
+      } else {
+        const uint4 mk = my_masks[c];
+        h[0] ^= mk.x, h[1] ^= mk.y, h[2] ^= mk.z, h[3] ^= mk.w;
       }
       *reinterpret_cast<uint4*>(orow + 16 * (c ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
     }

@@ -332,13 +332,17 @@ __global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
       for (int c = 0; c < 8; ++c) {
         const uint4 r = lds_u4(my_row + (uint32_t)(b * ENC_BOX_BYTES) + ((c ^ sw) << 4));
         const int k0 = b * 32 + c * 4;  // first pair of the chunk
-        uint4 mk;
-        if constexpr (LPV == 1) {
-          mk = make_uint4(T.sign_h2[k0], T.sign_h2[k0 + 1], T.sign_h2[k0 + 2], T.sign_h2[k0 + 3]);
+        uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+        if constexpr (LPV <= 2) {  // masks from the constant bank
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            w4[q] ^= T.sign_h2[k0 + q];
+            if (LPV == 2 && part) w4[q] ^= T.sign_h2_dx[k0 + q];
+          }
         } else {
-          mk = *reinterpret_cast<const uint4*>(smask + part * NP + k0);
+          const uint4 mk = *reinterpret_cast<const uint4*>(smask + part * NP + k0);
+          w4[0] ^= mk.x, w4[1] ^= mk.y, w4[2] ^= mk.z, w4[3] ^= mk.w;
         }
-        const uint32_t w4[4] = {r.x ^ mk.x, r.y ^ mk.y, r.z ^ mk.z, r.w ^ mk.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           v[k0 + q] = first_butterfly(w4[q]);

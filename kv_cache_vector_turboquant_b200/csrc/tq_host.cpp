@@ -138,6 +138,7 @@ tq_status tq_create(int head_dim, int bits, uint64_t seed, tq_ctx** out) {
     const uint64_t a = splitmix64_next(state), b = splitmix64_next(state);
     t.sign_h2[i / 2] = ((a >> 63) ? 0x8000u : 0u) | ((b >> 63) ? 0x80000000u : 0u);
   }
+  for (int k = 0; k < 32 && k + 32 < head_dim / 2; ++k) t.sign_h2_dx[k] = t.sign_h2[k] ^ t.sign_h2[k + 32];
 
   double delta = 0.0, frac = 0.0;
   if (!choose_grid(t.bounds, L - 1, &delta, &frac)) {

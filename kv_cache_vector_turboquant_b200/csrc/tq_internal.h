@@ -16,6 +16,10 @@ struct tq_codec_tables {
   // XOR mask for the fp16 pair (2k, 2k+1): bit 15 set <=> coordinate 2k is
   // negated, bit 31 set <=> coordinate 2k+1 is negated.
   uint32_t sign_h2[TQ_MAX_D / 2];
+  // sign_h2[k] ^ sign_h2[k + 32], k < 32: the change of mask between the two
+  // 64-coordinate halves of a head_dim-128 vector (a lane holding the upper
+  // half applies it on top of the lower half's mask).
+  uint32_t sign_h2_dx[32];
   float levels[TQ_MAX_L];      // format levels c_k (2^-14 grid), ascending
   float bounds[TQ_MAX_L - 1];  // decision boundaries t_j in z units (2^-15 grid)
   // Encode quantizer lookup table, in "q units" q = z * inv_delta + q_offset:
