@@ -63,6 +63,7 @@ typedef enum {
 #define TQ_DEVERR_SLOT_RANGE 0x2u  /* tq_encode_append: a slot outside [0, s_max) was skipped */
 #define TQ_DEVERR_POS_RANGE 0x4u   /* tq_attend_decode: a position > s_max was clamped */
 #define TQ_DEVERR_SMEM_LAYOUT 0x8u /* tq_attend_decode: shared memory not where the launch planned it; no output */
+#define TQ_DEVERR_BLOCK_RANGE 0x10u /* tq_attend_decode_paged: a block number outside [0, num_blocks) was clamped */
 
 /* Human-readable name of a status. Never NULL. */
 const char* tq_status_string(tq_status s);
@@ -177,6 +178,33 @@ tq_status tq_attend_decode(const tq_ctx* k, const tq_ctx* v, const void* q_f16, 
                            const void* k_packed, const float* k_norms, const void* v_packed,
                            const float* v_norms, int64_t s_max, const int32_t* positions, void* out_f16,
                            void* workspace, size_t ws_bytes, tq_stream stream);
+
+/*
+ * tq_attend_decode over a paged cache ("aither-kvcache", sections "Paged KV
+ * cache" and "API Reference": TQPagedAttention's block_tables and
+ * context_lens): the cache is a pool of blocks of TQ_PAGE_BLOCK positions,
+ * and each sequence lists the blocks that hold its positions in order.
+ *   k_cache     device, [num_blocks, TQ_PAGE_BLOCK, hkv, Pk] uint8, 16-byte
+ *               aligned.
+ *   k_norms     device, [num_blocks, TQ_PAGE_BLOCK, hkv] float32. (v likewise)
+ *   block_tables device, [B, max_blocks] int32: entry j of row b is the
+ *               block holding positions [16 j, 16 j + 16) of sequence b.
+ *               Entries past the sequence's context are not read; an entry
+ *               outside [0, num_blocks) that is read is clamped and flagged
+ *               with TQ_DEVERR_BLOCK_RANGE.
+ *   context_lens device, [B] int32: valid positions per sequence, as
+ *               `positions` of tq_attend_decode with s_max = max_blocks * 16.
+ *   workspace   at least tq_attend_workspace_bytes(B, hq, d, max_blocks * 16).
+ * Other arguments, results and errors as tq_attend_decode; with an identity
+ * block table over a [B, S, hkv, P] cache (S a multiple of 16) the output is
+ * bit-identical to tq_attend_decode's.
+ */
+#define TQ_PAGE_BLOCK 16
+tq_status tq_attend_decode_paged(const tq_ctx* k, const tq_ctx* v, const void* q_f16, int B, int hq, int hkv,
+                                 const void* k_cache, const float* k_norms, const void* v_cache,
+                                 const float* v_norms, int64_t num_blocks, const int32_t* block_tables,
+                                 int max_blocks, const int32_t* context_lens, void* out_f16, void* workspace,
+                                 size_t ws_bytes, tq_stream stream);
 
 /*
  * No counterpart in the paper: an addition of this library.

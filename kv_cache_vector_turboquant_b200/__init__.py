@@ -12,6 +12,7 @@ from __future__ import annotations
 
 from ._binding import (  # noqa: F401
     LIB_PATH,
+    TQ_DEVERR_BLOCK_RANGE,
     TQ_DEVERR_POS_RANGE,
     TQ_DEVERR_SLOT_RANGE,
     TQ_DEVERR_SMEM_LAYOUT,
@@ -25,10 +26,12 @@ from ._binding import (  # noqa: F401
     TQ_ERR_UNSUPPORTED,
     TQ_ERR_WORKSPACE,
     TQ_OK,
+    TQ_PAGE_BLOCK,
     Ctx,
     TQError,
     TQ_ATTEND_STATIC_SCRATCH_BYTES,
     tq_attend_decode,
+    tq_attend_decode_paged,
     tq_attend_decode_static,
     tq_attend_workspace_bytes,
     tq_create,
@@ -116,4 +119,29 @@ def attend_decode(q, k_codec: TurboQuant, v_codec: TurboQuant, k_packed, k_norms
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     tq_attend_decode(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_packed, k_norms, v_packed, v_norms, s_max,
                      positions, out, workspace, workspace.numel(), stream)
+    return out
+
+
+def attend_decode_paged(q, k_codec: TurboQuant, v_codec: TurboQuant, k_cache, k_norms, v_cache, v_norms,
+                        block_tables, context_lens, out=None, workspace=None, stream=None):
+    """One decode step of attention over paged packed caches.
+
+    q [B, Hq, d] fp16; k_cache [num_blocks, 16, Hkv, Pk] uint8; k_norms
+    [num_blocks, 16, Hkv] f32; v likewise; block_tables [B, max_blocks] int32
+    (block of positions [16 j, 16 j + 16) of sequence b); context_lens [B]
+    int32. Returns o [B, Hq, d] fp16.
+    """
+    import torch
+
+    B, hq, d = q.shape
+    num_blocks, blk, hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    _require(blk == TQ_PAGE_BLOCK, f"cache blocks must hold {TQ_PAGE_BLOCK} positions")
+    max_blocks = block_tables.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = tq_attend_workspace_bytes(B, hq, d, max_blocks * TQ_PAGE_BLOCK)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    tq_attend_decode_paged(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_cache, k_norms, v_cache, v_norms, num_blocks,
+                           block_tables, max_blocks, context_lens, out, workspace, workspace.numel(), stream)
     return out

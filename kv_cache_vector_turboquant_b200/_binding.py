@@ -40,6 +40,8 @@ _PROTOS = {
                                   _vp, _vp, _vp, _c_size, _vp]),
     "tq_attend_decode_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64,
                                          _vp, _vp, _vp]),
+    "tq_attend_decode_paged": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64, _vp,
+                                        _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
 }
@@ -61,6 +63,8 @@ TQ_DEVERR_TIMEOUT = 0x1
 TQ_DEVERR_SLOT_RANGE = 0x2
 TQ_DEVERR_POS_RANGE = 0x4
 TQ_DEVERR_SMEM_LAYOUT = 0x8
+TQ_DEVERR_BLOCK_RANGE = 0x10
+TQ_PAGE_BLOCK = 16
 
 LIB_PATH = _LIB_PATH
 
@@ -173,6 +177,15 @@ def tq_attend_decode(k: Ctx, v: Ctx, q, B: int, hq: int, hkv: int, k_packed, k_n
     _check(_lib.tq_attend_decode(k.handle, v.handle, _ptr(q), int(B), int(hq), int(hkv), _ptr(k_packed),
                                  _ptr(k_norms), _ptr(v_packed), _ptr(v_norms), int(s_max), _ptr(positions),
                                  _ptr(out), _ptr(workspace), int(ws_bytes), _stream(stream)), "tq_attend_decode")
+
+
+def tq_attend_decode_paged(k: Ctx, v: Ctx, q, B: int, hq: int, hkv: int, k_cache, k_norms, v_cache, v_norms,
+                           num_blocks: int, block_tables, max_blocks: int, context_lens, out, workspace,
+                           ws_bytes: int, stream=None) -> None:
+    _check(_lib.tq_attend_decode_paged(k.handle, v.handle, _ptr(q), int(B), int(hq), int(hkv), _ptr(k_cache),
+                                       _ptr(k_norms), _ptr(v_cache), _ptr(v_norms), int(num_blocks),
+                                       _ptr(block_tables), int(max_blocks), _ptr(context_lens), _ptr(out),
+                                       _ptr(workspace), int(ws_bytes), _stream(stream)), "tq_attend_decode_paged")
 
 
 def tq_attend_decode_static(k: Ctx, v: Ctx, q, B: int, hq: int, hkv: int, k_packed, k_norms, v_packed, v_norms,

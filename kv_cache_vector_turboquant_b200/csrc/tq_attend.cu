@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)nv * (krow_bytes + vrow_bytes));
     __syncwarp();
     if (lane < nv) {
-      const int64_t row = ((int64_t)b * a.s_max + t0 + lane) * a.hkv + hk0;
+      const int64_t row = attn_pos_row(a, b, t0 + lane) * a.hkv + hk0;
       uint8_t* st = smem + L.st0 + stage * L.stage;
       bulk_g2s(smem_u32(st + lane * L.krow), a.k_packed + row * PK, krow_bytes, bar);
       bulk_g2s(smem_u32(st + ATT_TILE * L.krow + lane * L.vrow), a.v_packed + row * PV, vrow_bytes, bar);
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
   // norms of the first tile (lane = position), then prefetched one tile ahead
   float nk_next = 0.f, nv_next = 0.f;
   if (head_ok && ntiles > 0 && lane < min64(ATT_TILE, npos)) {
-    const int64_t row = ((int64_t)b * a.s_max + s0 + lane) * a.hkv + hk;
+    const int64_t row = attn_pos_row(a, b, s0 + lane) * a.hkv + hk;
     nk_next = __ldg(a.k_norms + row);
     nv_next = __ldg(a.v_norms + row);
   }
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
     if (head_ok && tile + 1 < ntiles) {
       const int64_t t1 = t0 + ATT_TILE;
       if (lane < min64(ATT_TILE, s1 - t1)) {
-        const int64_t row = ((int64_t)b * a.s_max + t1 + lane) * a.hkv + hk;
+        const int64_t row = attn_pos_row(a, b, t1 + lane) * a.hkv + hk;
         nk_next = __ldg(a.k_norms + row);
         nv_next = __ldg(a.v_norms + row);
       }
@@ -527,10 +527,11 @@ size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max
   return 2 * align16(rows * 4) + rows * (size_t)head_dim * 4;
 }
 
-tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
-                           const void* k_packed, const float* k_norms, const void* v_packed,
-                           const float* v_norms, int64_t s_max, const int32_t* positions, void* out,
-                           void* workspace, size_t ws_bytes, void* stream) {
+static tq_status launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
+                               const void* k_packed, const float* k_norms, const void* v_packed,
+                               const float* v_norms, int64_t s_max, const int32_t* positions,
+                               const int32_t* block_tables, int max_blocks, int64_t num_blocks, void* out,
+                               void* workspace, size_t ws_bytes, void* stream) {
   const int d = k->d;
   const int g = hq / hkv;
   if (g > ATT_MAXG) return TQ_ERR_UNSUPPORTED;
@@ -540,7 +541,7 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
   if ((pk % 16 && hkv % 2) || (pv % 16 && hkv % 2)) return TQ_ERR_UNSUPPORTED;
   if ((pk * (hkv % 8)) % 16 || (pv * (hkv % 8)) % 16 || (pk * (hkv % 4)) % 16 || (pv * (hkv % 4)) % 16)
     return TQ_ERR_UNSUPPORTED;
-  AttnArgs a;
+  AttnArgs a{};
   for (int i = 0; i < TQ_MAX_D / 2; ++i) {
     a.k_sign_h2[i] = k->t.sign_h2[i];
     a.v_sign_h2[i] = v->t.sign_h2[i];
@@ -555,6 +556,9 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
   a.v_packed = static_cast<const uint8_t*>(v_packed);
   a.v_norms = v_norms;
   a.positions = positions;
+  a.block_tables = block_tables;
+  a.max_blocks = max_blocks;
+  a.num_blocks = num_blocks;
   a.out = static_cast<__half*>(out);
   a.B = B;
   a.hq = hq;
@@ -591,4 +595,21 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
 #undef TQ_ATT_D
 #undef TQ_ATT_CASE
   return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
+                           const void* k_packed, const float* k_norms, const void* v_packed,
+                           const float* v_norms, int64_t s_max, const int32_t* positions, void* out,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  return launch_attend(k, v, q, B, hq, hkv, k_packed, k_norms, v_packed, v_norms, s_max, positions, nullptr, 0, 0,
+                       out, workspace, ws_bytes, stream);
+}
+
+tq_status tq_launch_attend_paged(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
+                                 const void* k_cache, const float* k_norms, const void* v_cache,
+                                 const float* v_norms, int64_t num_blocks, const int32_t* block_tables,
+                                 int max_blocks, const int32_t* context_lens, void* out, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return launch_attend(k, v, q, B, hq, hkv, k_cache, k_norms, v_cache, v_norms, (int64_t)max_blocks * ATT_BLOCK,
+                       context_lens, block_tables, max_blocks, num_blocks, out, workspace, ws_bytes, stream);
 }

@@ -30,6 +30,12 @@ struct AttnArgs {
   const uint8_t* v_packed;
   const float* v_norms;
   const int32_t* positions;
+  // paged caches (block_tables non-null): K/V rows of position s of sequence
+  // b are in block block_tables[b * max_blocks + s / 16], row s % 16, of a
+  // cache of num_blocks blocks of 16 positions
+  const int32_t* block_tables;
+  int max_blocks;
+  int64_t num_blocks;
   __half* out;
   float* ws_m;    // [B, Hq, n_split]  running max (log2 domain)
   float* ws_l;    // [B, Hq, n_split]  sum of weights
@@ -63,6 +69,20 @@ inline void attn_split(int B, int64_t s_max, int* n_split, int* chunk) {
 }
 
 inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+constexpr int ATT_BLOCK = 16;  // positions per block of a paged cache
+
+// Cache row (position row, all kv heads) of position s of sequence b. A block
+// number outside [0, num_blocks) is clamped and flagged.
+TQ_DEV int64_t attn_pos_row(const AttnArgs& a, int b, int64_t s) {
+  if (a.block_tables == nullptr) return (int64_t)b * a.s_max + s;
+  int64_t blk = __ldg(a.block_tables + (int64_t)b * a.max_blocks + (s / ATT_BLOCK));
+  if (blk < 0 || blk >= a.num_blocks) {
+    record_error(a.err, TQ_DEVERR_BLOCK_RANGE);
+    blk = blk < 0 ? 0 : a.num_blocks - 1;
+  }
+  return blk * ATT_BLOCK + (s % ATT_BLOCK);
+}
 
 TQ_DEV float warp_max8(float v) {  // max over the 8 lanes sharing lane & 3
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));

@@ -81,6 +81,7 @@ struct FastArgs {
   int wpt;       // warps per tile: hw * nt
   int vpitch;    // bytes per V position row in shared memory (hw * D/4 + 16)
   int k_head_copies;  // 1: the K box is one head, issued hw times (no swapped-dimension map)
+  int paged;          // 1: boxes of 16 positions, two per tile, rows from the block table
   uint32_t tile_bytes;
 };
 
@@ -182,10 +183,27 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
     }
     fence_mbar_init();
   }
-  const int row0 = (int)((int64_t)b * a.s_max + s0);  // first cache row of this split
+  const int row0 = f.paged ? 0 : (int)((int64_t)b * a.s_max + s0);  // first cache row of this split
   auto issue = [&](int tile, int s) {  // one thread
     const uint32_t bar = smem_u32(&bars[s]);
     mbar_arrive_expect_tx(bar, f.tile_bytes);
+    if (f.paged) {
+      // the tile's two blocks of 16 positions; a second block past the
+      // context re-reads the first (its positions are masked out)
+      const int64_t sa = s0 + (int64_t)tile * ATT_TILE;
+      const int ra = (int)attn_pos_row(a, b, sa);
+      const int rb = sa + ATT_BLOCK < pos ? (int)attn_pos_row(a, b, sa + ATT_BLOCK) : ra;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = h ? rb : ra;
+        tma_load_3d(smem_u32(smem + f.kbuf[s] + h * hw * ATT_BLOCK * PK), &f.tm_k, 0, row, hgrp * hw, bar);
+        tma_load_3d(smem_u32(smem + f.vbuf[s] + h * ATT_BLOCK * VP), &f.tm_v, 0, hgrp, row, bar);
+        tma_load_3d(smem_u32(smem + f.knb[s] + h * ATT_BLOCK * hw * 4), &f.tm_kn, 0, hgrp, row, bar);
+        tma_load_3d(smem_u32(smem + f.vnb[s] + h * ATT_BLOCK * hw * 4), &f.tm_vn, 0, hgrp, row, bar);
+      }
+      issued[s] += 1;
+      return;
+    }
     const int row = row0 + tile * ATT_TILE;
     if (f.k_head_copies) {
       for (int h = 0; h < hw; ++h)
@@ -280,7 +298,11 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
   __syncthreads();
 
   const uint32_t LK = tb | (uint32_t)(lane * 4);  // byte 0 = lane copy, bytes 2-3 = region
-  const int kcol = hl * (ATT_TILE * PK) + tq * (D / 8);  // this lane's quarter of its head's K rows
+  // K stage layout: [head][32 positions][row], or with paged boxes
+  // [16-position box][head][16 positions][row]
+  const int khs = f.paged ? ATT_BLOCK * PK : ATT_TILE * PK;     // head stride
+  const int kbs = f.paged ? hw * ATT_BLOCK * PK : ATT_BLOCK * PK;  // stride of positions 16..31
+  const int kcol = hl * khs + tq * (D / 8);  // this lane's quarter of its head's K rows
   const int vcol = hl * PV + gq * (D / 32);              // this lane's eighth of its head's V row
   const uint32_t LV = tb | (uint32_t)(128 + (lane & 15) * 8);
 
@@ -310,11 +332,12 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
 #pragma unroll
     for (int mb16 = 0; mb16 < 2; ++mb16) {
       const int r0 = mb16 * 16 + gq;
+      const uint8_t* krow = kst + mb16 * kbs + gq * PK;  // position r0 (r0 + 8 is 8 rows on)
       uint32_t kw0[KQW], kw1[KQW];
 #pragma unroll
       for (int w = 0; w < KQW; w += 4) {
-        const uint4 x0 = *reinterpret_cast<const uint4*>(kst + r0 * PK + 4 * w);
-        const uint4 x1 = *reinterpret_cast<const uint4*>(kst + (r0 + 8) * PK + 4 * w);
+        const uint4 x0 = *reinterpret_cast<const uint4*>(krow + 4 * w);
+        const uint4 x1 = *reinterpret_cast<const uint4*>(krow + 8 * PK + 4 * w);
         kw0[w] = x0.x, kw0[w + 1] = x0.y, kw0[w + 2] = x0.z, kw0[w + 3] = x0.w;
         kw1[w] = x1.x, kw1[w + 1] = x1.y, kw1[w + 2] = x1.z, kw1[w + 3] = x1.w;
       }
@@ -575,7 +598,8 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   if (hw == 0) return cudaErrorNotSupported;
   const int pk = d / 2, pv = d / 4;
   const int hg = a.hkv / hw;
-  const int64_t rows = (int64_t)a.B * a.s_max;
+  const bool paged = a.block_tables != nullptr;
+  const int64_t rows = paged ? a.num_blocks * ATT_BLOCK : (int64_t)a.B * a.s_max;
   if (rows + 2 * ATT_TILE >= ((int64_t)1 << 31)) return cudaErrorNotSupported;  // int32 coordinates
   for (const void* p : {(const void*)a.k_packed, (const void*)a.v_packed, (const void*)a.k_norms,
                         (const void*)a.v_norms})
@@ -600,24 +624,28 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   if ((f.n_groups - 1) * f.wpt * 32 * (d / 8 + 2) * 4 > FA_TABLE_BYTES) return cudaErrorNotSupported;
 
   const cuuint64_t R = (cuuint64_t)rows, HG = (cuuint64_t)hg;
+  // positions per box: a tile, or one block of a paged cache (two boxes per tile)
+  const cuuint32_t BP = paged ? (cuuint32_t)ATT_BLOCK : (cuuint32_t)ATT_TILE;
+  f.paged = paged ? 1 : 0;
   const auto U64 = CU_TENSOR_MAP_DATA_TYPE_UINT64, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   // K: (row bytes, position, kv head) with the head stride inside the
   // position stride, so one box lands as [head][position][row]; where the
   // driver refuses that order, one (row, head, position) box per head.
   f.k_head_copies = 0;
   if (!encode_map(&f.tm_k, U64, a.k_packed, {(cuuint64_t)pk / 8, R, (cuuint64_t)a.hkv},
-                  {(cuuint64_t)a.hkv * pk, (cuuint64_t)pk}, {(cuuint32_t)pk / 8, ATT_TILE, (cuuint32_t)hw})) {
+                  {(cuuint64_t)a.hkv * pk, (cuuint64_t)pk}, {(cuuint32_t)pk / 8, BP, (cuuint32_t)hw})) {
+    if (paged) return cudaErrorNotSupported;  // the generic kernel takes it
     f.k_head_copies = 1;
     if (!encode_map(&f.tm_k, U64, a.k_packed, {(cuuint64_t)pk / 8, (cuuint64_t)a.hkv, R},
                     {(cuuint64_t)pk, (cuuint64_t)a.hkv * pk}, {(cuuint32_t)pk / 8, 1, ATT_TILE}))
       return cudaErrorNotSupported;
   }
   if (!encode_map(&f.tm_v, U64, a.v_packed, {(cuuint64_t)hw * pv / 8, HG, R},
-                  {(cuuint64_t)hw * pv, (cuuint64_t)a.hkv * pv}, {(cuuint32_t)f.vpitch / 8, 1, ATT_TILE}) ||
+                  {(cuuint64_t)hw * pv, (cuuint64_t)a.hkv * pv}, {(cuuint32_t)f.vpitch / 8, 1, BP}) ||
       !encode_map(&f.tm_kn, F32, a.k_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
-                  {(cuuint32_t)hw, 1, ATT_TILE}) ||
+                  {(cuuint32_t)hw, 1, BP}) ||
       !encode_map(&f.tm_vn, F32, a.v_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
-                  {(cuuint32_t)hw, 1, ATT_TILE}))
+                  {(cuuint32_t)hw, 1, BP}))
     return cudaErrorNotSupported;
 
   a.nt = nt;

@@ -234,6 +234,31 @@ tq_status tq_attend_decode(const tq_ctx* k, const tq_ctx* v, const void* q_f16, 
                           out_f16, workspace, ws_bytes, stream);
 }
 
+tq_status tq_attend_decode_paged(const tq_ctx* k, const tq_ctx* v, const void* q_f16, int B, int hq, int hkv,
+                                 const void* k_cache, const float* k_norms, const void* v_cache,
+                                 const float* v_norms, int64_t num_blocks, const int32_t* block_tables,
+                                 int max_blocks, const int32_t* context_lens, void* out_f16, void* workspace,
+                                 size_t ws_bytes, tq_stream stream) {
+  if (!k || !v) return TQ_ERR_INVALID_ARG;
+  if (k->d != v->d) return TQ_ERR_INVALID_ARG;
+  if (B < 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || num_blocks <= 0 || max_blocks <= 0)
+    return TQ_ERR_INVALID_ARG;
+  if (num_blocks > ((int64_t)1 << 26)) return TQ_ERR_UNSUPPORTED;  // cache rows stay below 2^30
+  if (B == 0) return TQ_OK;
+  if (!q_f16 || !k_cache || !k_norms || !v_cache || !v_norms || !block_tables || !context_lens || !out_f16)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned(q_f16, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out_f16, 16) ||
+      !aligned(k_norms, 4) || !aligned(v_norms, 4) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return TQ_ERR_ALIGNMENT;
+  const int64_t s_max = (int64_t)max_blocks * TQ_PAGE_BLOCK;
+  const size_t need = tq_attend_workspace_bytes(B, hq, k->d, s_max);
+  if (need == 0) return TQ_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < need) return TQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return TQ_ERR_ALIGNMENT;
+  return tq_launch_attend_paged(k, v, q_f16, B, hq, hkv, k_cache, k_norms, v_cache, v_norms, num_blocks,
+                                block_tables, max_blocks, context_lens, out_f16, workspace, ws_bytes, stream);
+}
+
 tq_status tq_device_error(tq_stream stream, uint32_t* bits) { return tq_read_error_word(stream, bits); }
 
 // Test hook (declared in include/tq_test.h): run tq_encode with the row copies

@@ -60,6 +60,11 @@ tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int 
                            const void* k_packed, const float* k_norms, const void* v_packed,
                            const float* v_norms, int64_t s_max, const int32_t* positions, void* out,
                            void* workspace, size_t ws_bytes, void* stream);
+tq_status tq_launch_attend_paged(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,
+                                 const void* k_cache, const float* k_norms, const void* v_cache,
+                                 const float* v_norms, int64_t num_blocks, const int32_t* block_tables,
+                                 int max_blocks, const int32_t* context_lens, void* out, void* workspace,
+                                 size_t ws_bytes, void* stream);
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max);
 
 // cuTensorMapEncodeTiled from the driver (cached; null if unavailable).

@@ -66,6 +66,7 @@ __all__ = [
     "decode_f64",
     "decode",
     "attend_decode",
+    "attend_decode_paged",
     "sphere_marginal_mse",
 ]
 
@@ -376,6 +377,37 @@ def attend_decode(q_f16, k_packed, k_norms, v_packed, v_norms, positions,
             p = np.exp(s - s.max())
             p /= p.sum()
             out[b, h] = p @ V[:, kv, :]
+    return out
+
+
+def attend_decode_paged(q_f16, k_cache, k_norms, v_cache, v_norms, block_tables, context_lens,
+                        k_bits: int, v_bits: int, k_seed: int = 42, v_seed: int = 42,
+                        block_size: int = 16) -> np.ndarray:
+    """attend_decode over a paged cache ("aither-kvcache", section "Paged KV
+    cache": blocks of 16 positions, a block table per sequence).
+
+    k_cache: [num_blocks, block_size, Hkv, P]; k_norms: [num_blocks,
+    block_size, Hkv]; v likewise; block_tables: [B, max_blocks], entry j of
+    row b the block holding positions [block_size j, block_size (j + 1)) of
+    sequence b; context_lens: [B]. Gathers each sequence's positions in order
+    and applies attend_decode to them.
+    """
+    q = np.asarray(q_f16)
+    B = q.shape[0]
+    kc, vc = np.asarray(k_cache), np.asarray(v_cache)
+    kn, vn = np.asarray(k_norms), np.asarray(v_norms)
+    bt = np.asarray(block_tables)
+    out = np.zeros(q.shape, dtype=np.float64)
+    for b in range(B):
+        n = int(context_lens[b])
+        nb = -(-n // block_size)
+        blocks = [int(bt[b, j]) for j in range(nb)]
+        kb = np.concatenate([kc[j] for j in blocks], axis=0)[:n]
+        vb = np.concatenate([vc[j] for j in blocks], axis=0)[:n]
+        knb = np.concatenate([kn[j] for j in blocks], axis=0)[:n]
+        vnb = np.concatenate([vn[j] for j in blocks], axis=0)[:n]
+        out[b] = attend_decode(q[b:b + 1], kb[None], knb[None], vb[None], vnb[None], [n],
+                               k_bits, v_bits, k_seed, v_seed)[0]
     return out
 
 

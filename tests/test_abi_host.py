@@ -162,3 +162,31 @@ def test_attend_validation_and_workspace(K):
 def test_compression_ratio_matches_formula(K):
     for b, want in ((2, 256 / 36), (3, 256 / 52), (4, 256 / 68)):
         assert abs(K.TurboQuant(128, b).compression_ratio() - want) < 1e-12
+
+
+def test_attend_paged_validation(K):
+    """tq_attend_decode_paged: sizes, null pointers, workspace and alignment
+    are checked on the host before anything is enqueued."""
+    k4, v2 = K.tq_create(128, 4), K.tq_create(128, 2)
+    k64 = K.tq_create(64, 4)
+    A = 0x100000
+    fn = "tq_attend_decode_paged"
+
+    def args(kc=k4, vc=v2, B=2, hq=8, hkv=2, nblk=40, bt=A, maxb=8, lens=A, ws_ptr=A, ws_b=None):
+        if ws_b is None:
+            ws_b = K.tq_attend_workspace_bytes(B if B > 0 else 1, hq, 128, maxb * K.TQ_PAGE_BLOCK)
+        return (kc.handle, vc.handle, A, B, hq, hkv, A, A, A, A, nblk, bt, maxb, lens, A, ws_ptr, ws_b, None)
+
+    need = K.tq_attend_workspace_bytes(2, 8, 128, 8 * 16)
+    assert _raw(K, fn, *args(hkv=3)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(vc=k64)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(nblk=0)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(maxb=0)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(bt=None)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(lens=None)) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, *args(bt=A + 2)) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, fn, *args(ws_b=need - 4)) == K.TQ_ERR_WORKSPACE
+    assert _raw(K, fn, *args(ws_ptr=None)) == K.TQ_ERR_WORKSPACE
+    assert _raw(K, fn, *args(ws_ptr=A + 4)) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, fn, *args(nblk=(1 << 26) + 1)) == K.TQ_ERR_UNSUPPORTED
+    assert _raw(K, fn, *args(B=0)) == K.TQ_OK

@@ -158,3 +158,64 @@ def test_many_tiles_per_split(K, W, hkv, hq):
         err = attn_row_error(o[b].cpu().numpy(), r)
         assert err.max() <= ATTN_RTOL, (b, err.max())
     assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+PAGED_CASES = [
+    # d, kb, vb, B, S (multiple of 16), hq, hkv, context lengths
+    (128, 4, 2, 3, 256, 32, 8, [256, 1, 77]),   # fast kernel
+    (256, 4, 2, 2, 160, 16, 8, [160, 129]),     # fast kernel, head_dim 256
+    (128, 4, 2, 2, 96, 32, 4, [96, 40]),        # fast kernel, 8 query heads per kv head
+    (128, 3, 3, 2, 112, 32, 8, [112, 33]),      # generic kernel
+    (64, 2, 4, 2, 64, 8, 2, [17, 64]),          # generic kernel, head_dim 64
+]
+
+
+def _to_pages(t, perm):
+    """[B, S, ...] contiguous cache -> pool [B*S/16, 16, ...] with logical block
+    j of sequence b stored at physical block perm[b * S/16 + j]."""
+    B, S = t.shape[0], t.shape[1]
+    blocks = t.reshape(B * S // 16, 16, *t.shape[2:])
+    pool = torch.empty_like(blocks)
+    pool[perm] = blocks
+    return pool
+
+
+@pytest.mark.parametrize("d,kb,vb,B,S,hq,hkv,lens", PAGED_CASES)
+def test_paged_attention_matches_contiguous_and_oracle(K, W, d, kb, vb, B, S, hq, hkv, lens):
+    """Paged caches with the blocks scattered by a random permutation: output
+    bit-identical to tq_attend_decode on the contiguous cache (same tiles, same
+    arithmetic) and within the tolerance of the oracle's paged attention."""
+    kc, vc, kp, kn, vp, vn = _make_cache(K, W, B, S, hkv, d, kb, vb, seed=3 * d + kb + vb + S)
+    q = W.randn_f16((B, hq, d), 7 + B, "cuda", scale=1.0 / np.sqrt(d))
+    lens_t = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    nb = S // 16
+    perm = torch.randperm(B * nb, generator=torch.Generator().manual_seed(d + S)).cuda()
+    kpool, vpool = _to_pages(kp, perm), _to_pages(vp, perm)
+    knpool, vnpool = _to_pages(kn, perm), _to_pages(vn, perm)
+    bt = perm.reshape(B, nb).to(torch.int32)
+    # table entries past each context are never read: fill them with garbage
+    for b, n in enumerate(lens):
+        bt[b, (n + 15) // 16:] = -12345
+    o_paged = K.attend_decode_paged(q, kc, vc, kpool, knpool, vpool, vnpool, bt, lens_t)
+    o_contig = K.attend_decode(q, kc, vc, kp, kn, vp, vn, lens_t)
+    torch.cuda.synchronize()
+    assert torch.equal(o_paged, o_contig)
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    ref = O.attend_decode_paged(q.cpu().numpy(), kpool.cpu().numpy(), knpool.cpu().numpy(), vpool.cpu().numpy(),
+                                vnpool.cpu().numpy(), bt.cpu().numpy(), lens, kb, vb)
+    err = attn_row_error(o_paged.cpu().numpy().astype(np.float64), ref)
+    assert err.max() <= ATTN_RTOL, err.max()
+
+
+def test_paged_attention_out_of_range_block_is_clamped_and_flagged(K, W):
+    d, B, S, hq, hkv = 128, 1, 64, 32, 8
+    kc, vc, kp, kn, vp, vn = _make_cache(K, W, B, S, hkv, d, 4, 2, seed=5)
+    q = W.randn_f16((B, hq, d), 8, "cuda", scale=1.0 / np.sqrt(d))
+    bt = torch.tensor([[0, 1, 99, 3]], dtype=torch.int32, device="cuda")  # block 99 of 4
+    lens = torch.tensor([64], dtype=torch.int32, device="cuda")
+    o = K.attend_decode_paged(q, kc, vc, kp.reshape(4, 16, hkv, -1), kn.reshape(4, 16, hkv),
+                              vp.reshape(4, 16, hkv, -1), vn.reshape(4, 16, hkv), bt, lens)
+    torch.cuda.synchronize()
+    st, bits = K.tq_device_error()
+    assert st == K.TQ_ERR_DEVICE and bits == K.TQ_DEVERR_BLOCK_RANGE
+    assert torch.isfinite(o.float()).all()

@@ -348,3 +348,47 @@ def test_attention_single_position_and_equal_keys():
     o2 = O.attend_decode(q, kp2, kn2, vp, vn, np.array([S, 5]), 4, 2)
     assert np.abs(o2[0] - V[0, :, 0].mean(axis=0)[None, :]).max() < 1e-12
     assert np.abs(o2[1] - V[1, :5, 0].mean(axis=0)[None, :]).max() < 1e-12
+
+
+def test_paged_attention_matches_sdpa_on_gathered_rows():
+    """Paged cache ("aither-kvcache", section "Paged KV cache"): the oracle's
+    block-table gather against torch SDPA on rows picked by flat index
+    block_tables[b, s // 16] * 16 + s % 16."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, d, blk, nblocks, maxb = 3, 8, 2, 64, 16, 11, 4
+    pool_k = rng.standard_normal((nblocks * blk, Hkv, d)).astype(np.float16)
+    pool_v = rng.standard_normal((nblocks * blk, Hkv, d)).astype(np.float16)
+    kp, kn = O.encode(pool_k, 4, 42)
+    vp, vn = O.encode(pool_v, 2, 42)
+    kc, vc = kp.reshape(nblocks, blk, Hkv, -1), vp.reshape(nblocks, blk, Hkv, -1)
+    knc, vnc = kn.reshape(nblocks, blk, Hkv), vn.reshape(nblocks, blk, Hkv)
+    bt = np.stack([rng.permutation(nblocks)[:maxb] for _ in range(B)]).astype(np.int32)
+    lens = np.array([64, 17, 5])
+    q = (rng.standard_normal((B, Hq, d)) / math.sqrt(d)).astype(np.float16)
+    got = O.attend_decode_paged(q, kc, knc, vc, vnc, bt, lens, 4, 2)
+    K = torch.from_numpy(O.decode_f64(kp, kn, 4, 42, d))  # [rows, Hkv, d]
+    V = torch.from_numpy(O.decode_f64(vp, vn, 2, 42, d))
+    for b in range(B):
+        s = np.arange(lens[b])
+        rows = torch.from_numpy(bt[b, s // blk].astype(np.int64) * blk + s % blk)
+        kk = K[rows].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+        vv = V[rows].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+        qq = torch.from_numpy(q[b].astype(np.float64))[:, None, :]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv)[:, 0, :]
+        assert np.abs(got[b] - ref.numpy()).max() < 1e-12
+
+
+def test_paged_attention_with_identity_table_is_contiguous_attention():
+    rng = np.random.default_rng(10)
+    B, S, Hq, Hkv, d = 2, 48, 4, 2, 64
+    kp, kn, vp, vn = _small_cache(rng, B, S, Hkv, d, 3, 3)
+    q = rng.standard_normal((B, Hq, d)).astype(np.float16)
+    pos = np.array([48, 33])
+    want = O.attend_decode(q, kp, kn, vp, vn, pos, 3, 3)
+    nb = S // 16
+    kc = kp.reshape(B * nb, 16, Hkv, -1)
+    vc = vp.reshape(B * nb, 16, Hkv, -1)
+    knc, vnc = kn.reshape(B * nb, 16, Hkv), vn.reshape(B * nb, 16, Hkv)
+    bt = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    got = O.attend_decode_paged(q, kc, knc, vc, vnc, bt, pos, 3, 3)
+    assert np.array_equal(got, want)
