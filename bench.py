@@ -206,6 +206,7 @@ def _bench_attention(K, W, torch, steps, warmup):
     peak, kind = _peaks()
     ach = alg / t / 1e9
     st = K.tq_device_error()
+    paged = _bench_attention_paged(K, torch, a, q, kc, vc, kp, kn, vp, vn, pos, steps, warmup, alg)
     return {"workload": "decode_step: q [16,32,128] fp16, K 4-bit / V 2-bit packed caches [16,32768,8,*]",
             "tokens_per_s": a["B"] / t, "ms_per_step": t * 1e3, "ms_median": statistics.median(ms),
             "cache_positions_heads_per_s": a["B"] * a["S"] * a["Hkv"] / t,
@@ -213,6 +214,49 @@ def _bench_attention(K, W, torch, steps, warmup):
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                          "traffic": _profile_traffic("tq_attend_fast.cu", "attend_fast_decode_step.txt"),
                          "peak_kind": kind, "algorithmic_bytes": alg},
+            "device_error": list(st), "paged": paged}
+
+
+def _bench_attention_paged(K, torch, a, q, kc, vc, kp, kn, vp, vn, pos, steps, warmup, alg):
+    """The same decode step over a paged cache: the 16-position blocks of all
+    sequences scattered over the pool by a random permutation, read through
+    block tables [16, 2048]."""
+    B, S = a["B"], a["S"]
+    nb = S // 16
+    perm = torch.randperm(B * nb, generator=torch.Generator().manual_seed(3)).cuda()
+
+    def pages(t):
+        blocks = t.reshape(B * nb, 16, *t.shape[2:])
+        pool = torch.empty_like(blocks)
+        pool[perm] = blocks
+        return pool
+
+    kpool, knpool, vpool, vnpool = pages(kp), pages(kn), pages(vp), pages(vn)
+    bt = perm.reshape(B, nb).to(torch.int32)
+    out = torch.empty_like(q)
+    wsb = K.tq_attend_workspace_bytes(B, a["Hq"], a["d"], S)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+
+    def call():
+        K.tq_attend_decode_paged(kc.ctx, vc.ctx, q, B, a["Hq"], a["Hkv"], kpool, knpool, vpool, vnpool, B * nb, bt,
+                                 nb, pos, out, ws, wsb)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(_ev(torch), _ev(torch)) for _ in range(steps)]
+    for e0, e1 in evs:
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    t = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs) / 1e3
+    peak, kind = _peaks()
+    st = K.tq_device_error()
+    del kpool, knpool, vpool, vnpool
+    return {"workload": "decode_step over a paged cache: 16-position blocks scattered by a random permutation, "
+                        "block tables [16, 2048]",
+            "tokens_per_s": B / t, "ms_per_step": t * 1e3, "GBps": alg / t / 1e9, "frac": alg / t / 1e9 / peak,
             "device_error": list(st)}
 
 
