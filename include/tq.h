@@ -145,6 +145,26 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
                            float* cache_norms, int64_t s_max, const int32_t* slot, tq_stream stream);
 
 /*
+ * Encode-on-write into a paged cache ("aither-kvcache", section "Custom
+ * inference loop": encode where the K/V of new tokens are written; the
+ * slot-mapping form of serving engines): token t of x is encoded and written
+ * to slot slot_mapping[t] of a pool of num_slots slots.
+ *   x_f16        device, [n_tok, h, d] fp16, 16-byte aligned.
+ *   cache_packed device, [num_slots, h, P] uint8, 16-byte aligned; the pool
+ *                of tq_attend_decode_paged is [num_blocks, TQ_PAGE_BLOCK, h,
+ *                P], i.e. num_slots = num_blocks * TQ_PAGE_BLOCK with slot =
+ *                block * TQ_PAGE_BLOCK + offset.
+ *   cache_norms  device, [num_slots, h] float32.
+ *   slot_mapping device, [n_tok] int32. A negative slot (a padding token)
+ *                is skipped; a slot >= num_slots is skipped and flagged with
+ *                TQ_DEVERR_SLOT_RANGE.
+ * Rows of other slots are not touched. The codes written are bit-identical
+ * to tq_encode of the same rows.
+ */
+tq_status tq_encode_slots(const tq_ctx* ctx, const void* x_f16, int64_t n_tok, int h, void* cache_packed,
+                          float* cache_norms, int64_t num_slots, const int32_t* slot_mapping, tq_stream stream);
+
+/*
  * Workspace (device bytes) that tq_attend_decode needs for a batch of B
  * sequences, hq query heads, head_dim and caches of s_max positions: the
  * split-S partial results (running max, sum and rotated accumulator per

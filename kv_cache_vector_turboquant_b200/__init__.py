@@ -39,6 +39,7 @@ from ._binding import (  # noqa: F401
     tq_device_error,
     tq_encode,
     tq_encode_append,
+    tq_encode_slots,
     tq_get_tables,
     tq_status_string,
 )
@@ -98,6 +99,16 @@ class TurboQuant:
         _require(d == self.head_dim, "last dim must be head_dim")
         s_max = cache_packed.shape[1]
         tq_encode_append(self.ctx, x, n_seq, h, cache_packed, cache_norms, s_max, slot, stream)
+
+    def encode_slots(self, x, cache_packed, cache_norms, slot_mapping, stream=None):
+        """Encode-on-write: x [n_tok, h, d] into slot slot_mapping[t] of a pool
+        cache_packed [num_slots, h, P] (or a paged pool [num_blocks, 16, h, P]),
+        cache_norms likewise; negative slots are skipped."""
+        n_tok, h, d = x.shape
+        _require(d == self.head_dim, "last dim must be head_dim")
+        _require(cache_packed.shape[-2] == h and cache_packed.shape[-1] == self.packed_bytes, "cache layout")
+        num_slots = cache_packed.numel() // (h * self.packed_bytes)
+        tq_encode_slots(self.ctx, x, n_tok, h, cache_packed, cache_norms, num_slots, slot_mapping, stream)
 
 
 def attend_decode(q, k_codec: TurboQuant, v_codec: TurboQuant, k_packed, k_norms, v_packed, v_norms,

@@ -35,6 +35,7 @@ _PROTOS = {
     "tq_encode": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_decode": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_append": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
+    "tq_encode_slots": (_c_int, [_vp, _vp, _c_i64, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_attend_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64]),
     "tq_attend_decode": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64,
                                   _vp, _vp, _vp, _c_size, _vp]),
@@ -166,6 +167,12 @@ def tq_encode_append(ctx: Ctx, x, n_seq: int, h: int, cache_packed, cache_norms,
                      stream=None) -> None:
     _check(_lib.tq_encode_append(ctx.handle, _ptr(x), int(n_seq), int(h), _ptr(cache_packed), _ptr(cache_norms),
                                  int(s_max), _ptr(slot), _stream(stream)), "tq_encode_append")
+
+
+def tq_encode_slots(ctx: Ctx, x, n_tok: int, h: int, cache_packed, cache_norms, num_slots: int, slot_mapping,
+                    stream=None) -> None:
+    _check(_lib.tq_encode_slots(ctx.handle, _ptr(x), int(n_tok), int(h), _ptr(cache_packed), _ptr(cache_norms),
+                                int(num_slots), _ptr(slot_mapping), _stream(stream)), "tq_encode_slots")
 
 
 def tq_attend_workspace_bytes(B: int, hq: int, head_dim: int, s_max: int) -> int:

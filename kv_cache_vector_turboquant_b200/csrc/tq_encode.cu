@@ -69,9 +69,10 @@ struct EncArgs {
   int64_t vec_base;  // index of vector 0 of this launch in the caller's tensor (append mode)
   uint8_t* packed;
   float* norms;
-  const int32_t* slot;  // append mode when non-null
+  const int32_t* slot;  // append mode when non-null: a slot per sequence (slot_abs = 0) or per token (1)
   int h;                // heads per sequence (append mode)
-  int64_t s_max;        // cache positions per sequence (append mode)
+  int64_t s_max;        // cache positions per sequence (append mode) or slots of the pool (slot_abs)
+  int slot_abs;         // 1: row slot[token] of a pool of s_max rows; a negative slot is skipped silently
   uint32_t* err;
   int fault_inject;      // test hook: 1 = never issue the tile copies
   long long wait_limit;  // bound on each mbarrier wait, SM cycles
@@ -453,12 +454,12 @@ __global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
       const int head = (int)(r - seq * a.h);
       const int32_t s = a.slot[seq];
       if (s >= 0 && s < a.s_max) {
-        const int64_t drow = (seq * a.s_max + s) * a.h + head;
+        const int64_t drow = (a.slot_abs ? (int64_t)s : seq * a.s_max + s) * a.h + head;
         uint8_t* dst = a.packed + drow * Cfg::P + part * Cfg::PL;
 #pragma unroll
         for (int w = 0; w < WL; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
         if (part == 0) a.norms[drow] = nrm;
-      } else if (part == 0) {
+      } else if (part == 0 && !(a.slot_abs && s < 0)) {
         record_error(a.err, TQ_DEVERR_SLOT_RANGE);
       }
     }
@@ -524,7 +525,8 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
 using namespace tq;
 
 tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
-                           const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject) {
+                           const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject,
+                           int slot_abs) {
   if (n == 0) return TQ_OK;
   EncArgs a;
   memset(&a, 0, sizeof(a));
@@ -534,6 +536,7 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
   a.slot = slot;
   a.h = h;
   a.s_max = s_max;
+  a.slot_abs = slot_abs;
   a.err = tq_error_word();
   if (!a.err) return TQ_ERR_CUDA;
   a.fault_inject = fault_inject;

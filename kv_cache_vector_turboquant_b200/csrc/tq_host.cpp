@@ -208,6 +208,16 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
   return tq_launch_encode(ctx, x_f16, (int64_t)n_seq * h, cache_packed, cache_norms, slot, h, s_max, stream, 0);
 }
 
+tq_status tq_encode_slots(const tq_ctx* ctx, const void* x_f16, int64_t n_tok, int h, void* cache_packed,
+                          float* cache_norms, int64_t num_slots, const int32_t* slot_mapping, tq_stream stream) {
+  if (!ctx || n_tok < 0 || h <= 0 || num_slots <= 0) return TQ_ERR_INVALID_ARG;
+  if (n_tok == 0) return TQ_OK;
+  if (!x_f16 || !cache_packed || !cache_norms || !slot_mapping) return TQ_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(cache_packed, 16) || !aligned(cache_norms, 4) || !aligned(slot_mapping, 4))
+    return TQ_ERR_ALIGNMENT;
+  return tq_launch_encode(ctx, x_f16, n_tok * h, cache_packed, cache_norms, slot_mapping, h, num_slots, stream, 0, 1);
+}
+
 size_t tq_attend_workspace_bytes(int B, int hq, int head_dim, int64_t s_max) {
   if (B <= 0 || hq <= 0 || s_max <= 0 || !(head_dim == 64 || head_dim == 128 || head_dim == 256)) return 0;
   return tq_attend_workspace_bytes_impl(B, hq, head_dim, s_max);

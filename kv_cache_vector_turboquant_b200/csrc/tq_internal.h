@@ -53,7 +53,8 @@ inline double tq_guard_z(int head_dim) { return head_dim <= 128 ? 1.0e-5 : 2.0e-
 // Kernel launchers (defined in the .cu files). Arguments are validated by the
 // ABI layer before these are called.
 tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
-                           const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject);
+                           const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject,
+                           int slot_abs = 0);
 tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n,
                            void* x, void* stream);
 tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,

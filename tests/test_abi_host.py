@@ -190,3 +190,18 @@ def test_attend_paged_validation(K):
     assert _raw(K, fn, *args(ws_ptr=A + 4)) == K.TQ_ERR_ALIGNMENT
     assert _raw(K, fn, *args(nblk=(1 << 26) + 1)) == K.TQ_ERR_UNSUPPORTED
     assert _raw(K, fn, *args(B=0)) == K.TQ_OK
+
+
+def test_encode_slots_validation(K):
+    ctx = K.tq_create(128, 4)
+    h = ctx.handle
+    A = 0x100000
+    fn = "tq_encode_slots"
+    assert _raw(K, fn, None, A, 4, 8, A, A, 64, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, h, A, -1, 8, A, A, 64, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, h, A, 4, 0, A, A, 64, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, h, A, 4, 8, A, A, 0, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, h, A, 4, 8, A, A, 64, None, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, fn, h, A + 8, 4, 8, A, A, 64, A, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, fn, h, A, 4, 8, A, A + 2, 64, A, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, fn, h, A, 0, 8, A, A, 64, A, None) == K.TQ_OK

@@ -234,6 +234,46 @@ def test_append_matches_bulk_encode(K, W, d, bits):
     assert code_mismatches(bp.reshape(-1, P)[:2048].numpy(), det, bits, d) == 0
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_encode_slots_writes_bulk_codes_into_mapped_slots(K, W, d, bits):
+    """Encode-on-write into a paged pool [num_blocks, 16, h, P]: token t lands
+    in slot slot_mapping[t] bit-identical to a bulk encode of the same rows;
+    padding tokens (slot -1) and every other slot are left untouched."""
+    n_tok, h, num_blocks = 300, 8, 40
+    tq = K.TurboQuant(d, bits)
+    P = tq.packed_bytes
+    x = W.append_stream(run=100 + d + bits, steps=1, n_seq=n_tok, H=h, d=d)[0].contiguous()
+    g = torch.Generator().manual_seed(d * bits)
+    slots = torch.randperm(num_blocks * 16, generator=g)[:n_tok].to(torch.int32)
+    slots[::7] = -1  # padding tokens
+    pool = torch.full((num_blocks, 16, h, P), 0x5A, dtype=torch.uint8, device="cuda")
+    pnorm = torch.full((num_blocks, 16, h), -2.0, dtype=torch.float32, device="cuda")
+    tq.encode_slots(x, pool, pnorm, slots.cuda())
+    bp, bn = tq.encode(x.reshape(-1, d))
+    torch.cuda.synchronize()
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    flat, fnorm = pool.reshape(-1, h, P).cpu(), pnorm.reshape(-1, h).cpu()
+    bp, bn = bp.reshape(n_tok, h, P).cpu(), bn.reshape(n_tok, h).cpu()
+    used = slots >= 0
+    assert torch.equal(flat[slots[used].long()], bp[used])
+    assert torch.equal(fnorm[slots[used].long()], bn[used])
+    untouched = torch.ones(flat.shape[0], dtype=torch.bool)
+    untouched[slots[used].long()] = False
+    assert torch.all(flat[untouched] == 0x5A) and torch.all(fnorm[untouched] == -2.0)
+
+
+def test_encode_slots_out_of_range_is_flagged(K, W):
+    tq = K.TurboQuant(128, 4)
+    x = W.append_stream(run=3, steps=1, n_seq=4, H=8, d=128)[0].contiguous()
+    pool = torch.zeros(2, 16, 8, 64, dtype=torch.uint8, device="cuda")
+    pnorm = torch.zeros(2, 16, 8, dtype=torch.float32, device="cuda")
+    tq.encode_slots(x, pool, pnorm, torch.tensor([0, 31, 32, -1], dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    st, bits = K.tq_device_error()
+    assert st == K.TQ_ERR_DEVICE and bits == K.TQ_DEVERR_SLOT_RANGE
+
+
 def test_append_out_of_range_slot_is_skipped_and_flagged(K, W):
     tq = K.TurboQuant(128, 4)
     n_seq, h, s_max = 4, 8, 8
