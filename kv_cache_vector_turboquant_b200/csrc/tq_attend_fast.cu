@@ -82,6 +82,8 @@ struct FastArgs {
   int vpitch;    // bytes per V position row in shared memory (hw * D/4 + 16)
   int k_head_copies;  // 1: the K box is one head, issued hw times (no swapped-dimension map)
   int paged;          // 1: boxes of 16 positions, two per tile, rows from the block table
+  int pg_off;         // paged: shared copy of the split's first block rows (int32), at this offset
+  int pg_cap;         //        and this many entries (later blocks are read from the table)
   uint32_t tile_bytes;
 };
 
@@ -188,11 +190,15 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
     const uint32_t bar = smem_u32(&bars[s]);
     mbar_arrive_expect_tx(bar, f.tile_bytes);
     if (f.paged) {
-      // the tile's two blocks of 16 positions; a second block past the
-      // context re-reads the first (its positions are masked out)
+      // the tile's two blocks of 16 positions (rows of the split's first
+      // blocks from the shared copy); a second block past the context
+      // re-reads the first (its positions are masked out)
       const int64_t sa = s0 + (int64_t)tile * ATT_TILE;
-      const int ra = (int)attn_pos_row(a, b, sa);
-      const int rb = sa + ATT_BLOCK < pos ? (int)attn_pos_row(a, b, sa + ATT_BLOCK) : ra;
+      const int ja = 2 * tile;  // block index within the split
+      const int* pg = reinterpret_cast<const int*>(smem + f.pg_off);
+      const int ra = ja < f.pg_cap ? pg[ja] : (int)attn_pos_row(a, b, sa);
+      const int rb = sa + ATT_BLOCK < pos ? (ja + 1 < f.pg_cap ? pg[ja + 1] : (int)attn_pos_row(a, b, sa + ATT_BLOCK))
+                                          : ra;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = h ? rb : ra;
@@ -216,6 +222,12 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
     tma_load_3d(smem_u32(smem + f.vnb[s]), &f.tm_vn, 0, hgrp, row, bar);
     issued[s] += 1;
   };
+  if (f.paged) {  // the split's first block rows, before the first copies are issued
+    int* pg = reinterpret_cast<int*>(smem + f.pg_off);
+    const int nblk = (int)min64(f.pg_cap, (npos + ATT_BLOCK - 1) / ATT_BLOCK);
+    for (int j = threadIdx.x; j < nblk; j += blockDim.x) pg[j] = (int)attn_pos_row(a, b, s0 + (int64_t)j * ATT_BLOCK);
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
     for (int t = 0; t < NS && t < ntiles; ++t) issue(t, t);
   }
@@ -548,13 +560,13 @@ static bool encode_map(CUtensorMap* m, CUtensorMapDataType type, const void* bas
 // shared address that is a multiple of 65536, stage buffers (128-byte
 // aligned) in the space below and above the tables. The most stages that
 // fit, a multiple of the group count and at least two per group.
-static bool plan_smem(FastArgs& f, int base, int max_dyn, int kbytes, int vbytes, int nbytes) {
+static bool plan_smem(FastArgs& f, int base, int max_dyn, int kbytes, int vbytes, int nbytes, int hdr) {
   const int tb_abs = (base + FA_TABLE_BYTES - 1) & ~(FA_TABLE_BYTES - 1);
   const int tb_off = tb_abs - base;
-  if (tb_off < 128 || tb_off + FA_TABLE_BYTES > max_dyn) return false;
+  if (tb_off < hdr || tb_off + FA_TABLE_BYTES > max_dyn) return false;
   for (int ns = FA_MAX_STAGES; ns >= 2 * f.n_groups; --ns) {
     if (ns % f.n_groups) continue;
-    int lo[2] = {128, tb_off + FA_TABLE_BYTES}, hi[2] = {tb_off, max_dyn};
+    int lo[2] = {hdr, tb_off + FA_TABLE_BYTES}, hi[2] = {tb_off, max_dyn};
     auto take = [&](int bytes, int* out) {
       for (int r = 0; r < 2; ++r) {
         const int at = (lo[r] + 127) & ~127;
@@ -616,7 +628,11 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   f.n_groups = FA_WARPS / f.wpt;
   f.vpitch = hw * pv + 16;
   const int kbytes = ATT_TILE * hw * pk, vbytes = ATT_TILE * f.vpitch, nbytes = ATT_TILE * hw * 4;
-  if (!plan_smem(f, reserved, max_dyn, kbytes, vbytes, nbytes)) return cudaErrorNotSupported;
+  // paged: 2 KB after the 128-byte header hold the rows of the split's first
+  // 512 blocks, so the issuing thread reads them from shared memory
+  f.pg_off = 128;
+  f.pg_cap = paged ? 512 : 0;
+  if (!plan_smem(f, reserved, max_dyn, kbytes, vbytes, nbytes, 128 + 4 * f.pg_cap)) return cudaErrorNotSupported;
   f.smem_base = (uint32_t)reserved;
   f.tile_bytes = (uint32_t)(kbytes + vbytes + 2 * nbytes);
   // the rotated queries (before the tables) and the group merge (after) use the table region

@@ -60,7 +60,6 @@ struct EncCfg {
   static constexpr int GROUPS = C / 32;        // guard groups of 32 coordinates
   static constexpr int BOXES = C / ENC_BOX_COLS;
   static constexpr int STAGE = BOXES * ENC_BOX_BYTES;
-  static constexpr int WARPS = C == 128 ? 8 : 16;
 };
 
 struct EncArgs {
@@ -80,7 +79,7 @@ struct EncArgs {
 
 // Shared memory, per CTA: fixed header, then (1024-byte aligned, for the
 // swizzle pattern) the warps' stage buffers, then the cell table.
-template <int D, int BITS>
+template <int D, int BITS, int W>
 struct EncSmem {
   using Cfg = EncCfg<D, BITS>;
   static constexpr int BAR = 0;                    // warps x stages u64
@@ -88,7 +87,7 @@ struct EncSmem {
   static constexpr int MASK = 320;                 // sign masks, D/2 u32
   static constexpr int SCR = 1024;                 // per warp 32-float scratch
   static constexpr int HEADER = SCR + 16 * 32 * 4;  // 3072
-  static constexpr int IN_BYTES = Cfg::WARPS * ENC_STAGES * Cfg::STAGE;
+  static constexpr int IN_BYTES = W * ENC_STAGES * Cfg::STAGE;
   static size_t bytes(int cells) {
     return (size_t)HEADER + 1024 + IN_BYTES + (size_t)cells * ENC_LUT_COPIES * 8;
   }
@@ -219,13 +218,13 @@ __device__ __noinline__ uint32_t recheck_group(float* scratch, float srcR, float
   return cm;
 }
 
-template <int D, int BITS>
-__global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
+template <int D, int BITS, int W>
+__global__ void __launch_bounds__(W * 32, 1)
     encode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ EncArgs a) {
   using Cfg = EncCfg<D, BITS>;
-  using Sm = EncSmem<D, BITS>;
+  using Sm = EncSmem<D, BITS, W>;
   constexpr int C = Cfg::C, NP = Cfg::NP, LPV = Cfg::LPV, WL = Cfg::WL, L = Cfg::L;
-  constexpr int WARPS = Cfg::WARPS;
+  constexpr int WARPS = W;
   constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -235,23 +234,14 @@ __global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
   const uint32_t in_addr = (smem_base + Sm::HEADER + 1023u) & ~1023u;  // stages: 1024-byte aligned
   const uint32_t lut_addr = in_addr + Sm::IN_BYTES;
 
-  // ---- cell table: entry (cell, copy) = {boundary bits or 3e38 if none, count of boundaries below}
+  // ---- cell table (built on the host): entry (cell, copy) = {boundary bits
+  // or 3e38 if none, count of boundaries below}, 16 lane copies
   {
     uint2* lut = reinterpret_cast<uint2*>(smem + (lut_addr - smem_base));
-    const int cells = T.lut_cells;
-    for (int e = threadIdx.x; e < cells * ENC_LUT_COPIES; e += blockDim.x) {
+    const int entries = T.lut_cells * ENC_LUT_COPIES;
+    for (int e = threadIdx.x; e < entries; e += blockDim.x) {
       const int cell = e / ENC_LUT_COPIES;
-      uint32_t below = 0;
-      float thr = 3.0e38f;
-#pragma unroll
-      for (int j = 0; j < L - 1; ++j) {
-        const float t = T.tau[j];
-        if (t < (float)cell)
-          ++below;
-        else if (t < (float)(cell + 1))
-          thr = t;
-      }
-      lut[e] = make_uint2(__float_as_uint(thr), below);
+      lut[e] = make_uint2(T.cell[cell][0], T.cell[cell][1]);
     }
   }
   float* sbound = reinterpret_cast<float*>(smem + Sm::BND);
@@ -472,22 +462,36 @@ __global__ void __launch_bounds__(EncCfg<D, BITS>::WARPS * 32, 1)
   }
 }
 
+// Warps per CTA: 16 (one persistent CTA per SM) for bulk work; 2 when the
+// launch has at most two tiles per SM (a streaming append), so its few tiles
+// spread over the SMs instead of sharing a few of them.
+constexpr int ENC_WARPS_BULK = 16;
+constexpr int ENC_WARPS_SMALL = 2;
+
+template <int D, int BITS, int W>
+static cudaError_t configure_encode(size_t smem, int dev) {
+  static std::atomic<uint64_t> configured{0};  // one bit per device
+  const uint64_t bit = 1ull << (dev & 63);
+  if (configured.load() & bit) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(encode_kernel<D, BITS, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) configured.fetch_or(bit);
+  return e;
+}
+
 template <int D, int BITS>
 static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const void* x, cudaStream_t st) {
   using Cfg = EncCfg<D, BITS>;
-  const size_t smem = EncSmem<D, BITS>::bytes(T.lut_cells);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static std::atomic<uint64_t> configured{0};  // one bit per device
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(encode_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured.fetch_or(bit);
-  }
+  const size_t smem_bulk = EncSmem<D, BITS, ENC_WARPS_BULK>::bytes(T.lut_cells);
+  const size_t smem_small = EncSmem<D, BITS, ENC_WARPS_SMALL>::bytes(T.lut_cells);
+  if ((e = configure_encode<D, BITS, ENC_WARPS_BULK>(smem_bulk, dev)) != cudaSuccess) return e;
+  if ((e = configure_encode<D, BITS, ENC_WARPS_SMALL>(smem_small, dev)) != cudaSuccess) return e;
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
   if (!enc) return cudaErrorNotSupported;
+  const int sms = tq_sm_count(dev);
   // launches of at most 2^30 lane-rows keep the copy coordinates in int32
   const int64_t max_vec = ((int64_t)1 << 30) / Cfg::LPV;
   const int64_t n_total = a.n;
@@ -511,9 +515,14 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
     const int64_t tiles = (n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
-    const int64_t ctas_needed = (tiles + Cfg::WARPS - 1) / Cfg::WARPS;
-    const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)tq_sm_count(dev));
-    encode_kernel<D, BITS><<<grid, Cfg::WARPS * 32, smem, st>>>(T, a);
+    if (tiles <= (int64_t)ENC_WARPS_SMALL * sms) {
+      const int grid = (int)((tiles + ENC_WARPS_SMALL - 1) / ENC_WARPS_SMALL);
+      encode_kernel<D, BITS, ENC_WARPS_SMALL><<<grid, ENC_WARPS_SMALL * 32, smem_small, st>>>(T, a);
+    } else {
+      const int64_t ctas_needed = (tiles + ENC_WARPS_BULK - 1) / ENC_WARPS_BULK;
+      const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)sms);
+      encode_kernel<D, BITS, ENC_WARPS_BULK><<<grid, ENC_WARPS_BULK * 32, smem_bulk, st>>>(T, a);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -151,6 +151,24 @@ tq_status tq_create(int head_dim, int bits, uint64_t seed, tq_ctx** out) {
   t.lut_cells = 2 * K + 2;
   t.guard_q = (float)(tq_guard_z(head_dim) / delta);
   for (int j = 0; j < L - 1; ++j) t.tau[j] = (float)(t.bounds[j] / delta + (K + frac));
+  if (t.lut_cells > TQ_MAX_CELLS) {
+    delete c;
+    return TQ_ERR_UNSUPPORTED;
+  }
+  for (int cell = 0; cell < t.lut_cells; ++cell) {
+    uint32_t below = 0;
+    float thr = 3.0e38f;  // no boundary in this cell
+    for (int j = 0; j < L - 1; ++j) {
+      if (t.tau[j] < (float)cell)
+        ++below;
+      else if (t.tau[j] < (float)(cell + 1))
+        thr = t.tau[j];
+    }
+    uint32_t tb;
+    std::memcpy(&tb, &thr, 4);
+    t.cell[cell][0] = tb;
+    t.cell[cell][1] = below;
+  }
   *out = c;
   return TQ_OK;
 }

@@ -9,6 +9,7 @@
 
 #define TQ_MAX_D 256
 #define TQ_MAX_L 16
+#define TQ_MAX_CELLS 272
 
 // Codec tables, passed by value in every kernel launch (constant bank), so
 // warp-uniform lookups (sign masks, levels) cost no registers or loads.
@@ -30,6 +31,9 @@ struct tq_codec_tables {
   float inv_delta;          // 1/delta, a power of two
   float guard_q;            // half-width of the f64 recheck band, q units
   int lut_cells;            // number of cells (q in [0, lut_cells))
+  // per cell: {bits of the boundary inside it (3e38 if none), count of
+  // boundaries below the cell}; kernels replicate it into shared memory
+  uint32_t cell[TQ_MAX_CELLS][2];
   int d;
   int bits;
 };
