@@ -67,6 +67,10 @@ __all__ = [
     "decode",
     "attend_decode",
     "attend_decode_paged",
+    "encode_os_detail",
+    "encode_os",
+    "decode_os_f64",
+    "decode_os",
     "sphere_marginal_mse",
 ]
 
@@ -409,6 +413,81 @@ def attend_decode_paged(q_f16, k_cache, k_norms, v_cache, v_norms, block_tables,
         out[b] = attend_decode(q[b:b + 1], kb[None], knb[None], vb[None], vnb[None], [n],
                                k_bits, v_bits, k_seed, v_seed)[0]
     return out
+
+
+def _side_pack(mu16: np.ndarray, n16: np.ndarray) -> np.ndarray:
+    return (mu16.astype(np.float16).view(np.uint16).astype(np.uint32)
+            | (n16.astype(np.float16).view(np.uint16).astype(np.uint32) << 16))
+
+
+def _side_unpack(side: np.ndarray):
+    side = np.asarray(side, dtype=np.uint32).reshape(-1)
+    mu16 = (side & 0xFFFF).astype(np.uint16).view(np.float16)
+    n16 = (side >> 16).astype(np.uint16).view(np.float16)
+    return mu16, n16
+
+
+def encode_os_detail(x_f16: np.ndarray, bits: int, seed: int, side=None) -> dict:
+    """The offset + half-precision scale variant ("TurboQuant efficient
+    inference", section "1. The quantizer": remove a small per-vector offset,
+    rotate, round each coordinate to a level, keep one scale alongside, codes
+    packed two per byte at 4 bits, scales in half precision).
+
+    Reading: offset mu16 = fp16(mean(x)); y = x - mu16; scale n16 =
+    fp16(||y||); then the TurboQuant step on y with n16 in place of the norm:
+    z = (H_pm D y) / n16, index_i = #{j : z_i >= t_j}. Side data per vector:
+    uint32 = fp16 bits of mu16 | fp16 bits of n16 << 16.
+
+    ``side``: optional [n] uint32 to use instead of computing mu16 and n16
+    (to check codes given another implementation's side data).
+    """
+    x16 = np.asarray(x_f16)
+    if x16.dtype != np.float16:
+        raise TypeError("input must be float16")
+    d = x16.shape[-1]
+    x = _as_rows(x16, d).astype(np.float64)
+    if side is None:
+        mu16 = (x.sum(axis=1) / d).astype(np.float16)  # the fp16 sum is exact in fp64; /d exact
+        y = x - mu16.astype(np.float64)[:, None]        # exact: both fp16
+        nrm = np.sqrt((y * y).sum(axis=1))
+        with np.errstate(over="ignore"):
+            n16 = nrm.astype(np.float16)
+    else:
+        mu16, n16 = _side_unpack(side)
+        y = x - mu16.astype(np.float64)[:, None]
+        nrm = np.sqrt((y * y).sum(axis=1))
+    nq = n16.astype(np.float64)
+    s = sign_vector(seed, d)
+    w = (y * s[None, :]) @ hadamard_pm(d).T  # sums of +-y_k: exact in fp64
+    ok = (nq > 0.0) & np.isfinite(nq)
+    z = np.where(ok[:, None], w / np.where(ok, nq, 1.0)[:, None], 0.0)
+    idx = quantize(z, format_boundaries(format_levels(bits)))
+    return {"packed": pack_codes(idx, bits), "side": _side_pack(mu16, n16), "idx": idx, "z": z,
+            "mu16": mu16, "n16": n16, "norm64": nrm}
+
+
+def encode_os(x_f16: np.ndarray, bits: int, seed: int = 42):
+    """``[..., d]`` fp16 -> (``[..., d*b/8]`` uint8, ``[...]`` uint32 side data)."""
+    x16 = np.asarray(x_f16)
+    lead = x16.shape[:-1]
+    out = encode_os_detail(x16, bits, seed)
+    return out["packed"].reshape(*lead, packed_bytes(x16.shape[-1], bits)), out["side"].reshape(lead)
+
+
+def decode_os_f64(packed: np.ndarray, side: np.ndarray, bits: int, seed: int, d: int) -> np.ndarray:
+    """x_hat = mu16 + (n16 / d) D H_pm c[idx] in fp64, before the fp16 rounding."""
+    pk = np.asarray(packed)
+    lead = pk.shape[:-1]
+    idx = unpack_codes(pk.reshape(-1, pk.shape[-1]), bits, d)
+    c = format_levels(bits)[idx]
+    mu16, n16 = _side_unpack(side)
+    hc = c @ hadamard_pm(d).T * sign_vector(seed, d)[None, :]
+    out = mu16.astype(np.float64)[:, None] + (n16.astype(np.float64) / d)[:, None] * hc
+    return out.reshape(*lead, d)
+
+
+def decode_os(packed: np.ndarray, side: np.ndarray, bits: int, seed: int, d: int) -> np.ndarray:
+    return decode_os_f64(packed, side, bits, seed, d).astype(np.float16)
 
 
 # --------------------------------------------------------------------------

@@ -392,3 +392,69 @@ def test_paged_attention_with_identity_table_is_contiguous_attention():
     bt = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
     got = O.attend_decode_paged(q, kc, knc, vc, vnc, bt, pos, 3, 3)
     assert np.array_equal(got, want)
+
+
+# ---------------------------------------------- offset + half-precision scale
+
+def test_os_side_data_layout_and_constant_vectors():
+    """Side data = fp16 bits of the offset | fp16 bits of the scale << 16:
+    [1, 3, 1, 3, ...] has mean 2 and centred norm sqrt(64) = 8 (fp16 0x4000
+    and 0x4800). A constant vector has scale 0, codes 2^(b-1) and decodes to
+    itself exactly."""
+    d = 64
+    x = np.tile(np.array([1.0, 3.0], dtype=np.float16), d // 2)[None, :]
+    det = O.encode_os_detail(x, 4, 42)
+    assert int(det["side"][0]) == 0x4000 | (0x4800 << 16)
+    c = np.full((3, 128), [[-2.5], [0.0], [1000.0]], dtype=np.float16)
+    for bits in (2, 3, 4):
+        p, sd = O.encode_os(c, bits, 7)
+        assert np.all(O.unpack_codes(p, bits, 128) == 2 ** (bits - 1))
+        assert np.array_equal(O.decode_os(p, sd, bits, 7, 128), c)
+
+
+def test_os_codes_are_translation_invariant():
+    """Adding a constant c to a zero-mean integer vector (every value, the
+    mean c and the centred vector stay exact in fp16) leaves codes and scale
+    unchanged and makes the offset c."""
+    rng = np.random.default_rng(21)
+    h = rng.integers(-40, 40, size=(50, 64)).astype(np.float16)
+    x = np.concatenate([h, -h], axis=1)
+    a = O.encode_os_detail(x, 3, 42)
+    assert np.all(a["mu16"] == 0)
+    for c in (4.0, -16.0, 100.0):
+        b = O.encode_os_detail((x.astype(np.float64) + c).astype(np.float16), 3, 42)
+        assert np.all(b["mu16"].astype(np.float64) == c)
+        assert np.array_equal(a["idx"], b["idx"])
+        assert np.array_equal(a["n16"], b["n16"])
+
+
+def test_os_zero_mean_matches_turboquant_with_rounded_norm():
+    """For vectors with an exactly zero mean the offset is 0 and the codes are
+    the TurboQuant codes of the same vector with the norm rounded to fp16."""
+    rng = np.random.default_rng(22)
+    h = rng.standard_normal((200, 64)).astype(np.float16)
+    x = np.concatenate([h, -h], axis=1)  # mean exactly 0
+    os_ = O.encode_os_detail(x, 4, 42)
+    tq = O.encode_detail(x, 4, 42)
+    assert np.all(os_["mu16"] == 0)
+    z = tq["z"] * (tq["norm64"] / os_["n16"].astype(np.float64))[:, None]
+    assert np.array_equal(O.quantize(z, O.format_boundaries(O.format_levels(4))), os_["idx"])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_os_distortion_of_centred_gaussian_rows(bits):
+    """Gaussian rows with a random offset: the per-coordinate distortion of the
+    centred direction is the sphere-marginal value, as for TurboQuant (the fp16
+    scale moves it by < 1e-3 relative)."""
+    d = 128
+    rng = np.random.default_rng(30 + bits)
+    x = (rng.standard_normal((8000, d)) + rng.uniform(-3, 3, size=(8000, 1))).astype(np.float16)
+    det = O.encode_os_detail(x, bits, 42)
+    xh = O.decode_os_f64(det["packed"], det["side"], bits, 42, d)
+    mu = det["mu16"].astype(np.float64)[:, None]
+    y = x.astype(np.float64) - mu
+    yh = xh - mu
+    # ||y - yh||^2 / ||y||^2 = (n16 / ||y||)^2 * mean over coordinates of (z - c)^2
+    emp = (((y - yh) ** 2).sum(axis=1) / (y * y).sum(axis=1)).mean()
+    want = O.sphere_marginal_mse(O.format_levels(bits), d)
+    assert abs(emp - want) / want < 0.02, (emp, want)
