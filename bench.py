@@ -321,6 +321,40 @@ def _bench_append(K, W, torch, steps_per_run=1024):
     return res
 
 
+def _bench_offset_variant(K, W, torch, reps=10):
+    """The offset + fp16-scale variant (4 bits) on the llama layer's K and V
+    tensors, alternating, one launch per tensor: encode, then decode."""
+    k, v = W.llama_layer(device="cuda")
+    xs = [k.reshape(-1, D), v.reshape(-1, D)]
+    n = xs[0].shape[0]
+    c = K.TurboQuant(D, 4)
+    P = c.packed_bytes
+    pk = [torch.empty(n, P, dtype=torch.uint8, device="cuda") for _ in xs]
+    sd = [torch.empty(n, dtype=torch.int32, device="cuda") for _ in xs]
+    out = [torch.empty(n, D, dtype=torch.float16, device="cuda") for _ in xs]
+    for i in range(4):
+        K.tq_encode_os(c.ctx, xs[i % 2], n, pk[i % 2], sd[i % 2])
+        K.tq_decode_os(c.ctx, pk[i % 2], sd[i % 2], n, out[i % 2])
+    torch.cuda.synchronize()
+    res = {}
+    peak, kind = _peaks()
+    alg = n * (2 * D + P + 4)
+    for name, fn in (("encode", lambda i: K.tq_encode_os(c.ctx, xs[i % 2], n, pk[i % 2], sd[i % 2])),
+                     ("decode", lambda i: K.tq_decode_os(c.ctx, pk[i % 2], sd[i % 2], n, out[i % 2]))):
+        e0, e1 = _ev(torch), _ev(torch)
+        e0.record()
+        for i in range(reps):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / reps / 1e3
+        res[name] = {"us": t * 1e6, "GBps": alg / t / 1e9, "frac": alg / t / 1e9 / peak}
+    res["workload"] = "offset + fp16-scale variant, 4 bits, llama layer K/V [8,8192,8,128] (one tensor per launch)"
+    res["device_error"] = list(K.tq_device_error())
+    del k, v, xs, pk, sd, out
+    return res
+
+
 def _bench_long_context(K, W, torch, reps=2):
     """The 80-layer long-context cache at 3 bits: K and V [1, 131072, 8, 128]
     of every layer, all resident in HBM, encoded layer by layer (K then V) on
@@ -494,6 +528,7 @@ def run_ours(args, rank, world, local_rank):
         result["attn"] = _bench_attention(K, W, torch, max(args.steps, 5), max(args.warmup, 3))
         result["append"] = _bench_append(K, W, torch)
         result["long_context"] = _bench_long_context(K, W, torch)
+        result["offset_variant"] = _bench_offset_variant(K, W, torch)
     if rank == 0 and world == 1 and not args.skip_cpu:
         result["cpu_baseline"] = _cpu_baseline()
     return result

@@ -145,6 +145,32 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
                            float* cache_norms, int64_t s_max, const int32_t* slot, tq_stream stream);
 
 /*
+ * The offset + half-precision-scale variant ("TurboQuant efficient
+ * inference", section "1. The quantizer": remove a small per-vector offset,
+ * rotate, round each coordinate to a level, keep one scale alongside; codes
+ * packed two per byte at 4 bits, scales in half precision). Per vector:
+ * offset mu16 = fp16(mean(x)) (the mean accumulated in f32), y = x - mu16,
+ * scale n16 = fp16(||y||); the codes are those of tq_encode applied to y
+ * with n16 in place of the norm (decided exactly, as tq_encode's).
+ *   packed  device, [n, tq_packed_bytes] uint8 out (same layout as tq_encode).
+ *   side    device, [n] uint32 out: fp16 bits of mu16 | fp16 bits of n16 << 16.
+ * A constant vector gets scale 0 and decodes to itself; a vector with
+ * ||x - mean|| above the fp16 range gets an infinite scale and an
+ * unspecified decode. Asynchronous on `stream`.
+ */
+tq_status tq_encode_os(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, uint32_t* side,
+                       tq_stream stream);
+
+/*
+ * Decode of the offset variant: x_hat = mu16 + (n16 / head_dim) D H_pm c[idx]
+ * (H_pm the +-1 Walsh-Hadamard matrix), computed in f32 (a product and a sum
+ * of the offset, each rounded once) and rounded to fp16.
+ *   packed, side as written by tq_encode_os; x_f16 device [n, head_dim] out.
+ */
+tq_status tq_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x_f16,
+                       tq_stream stream);
+
+/*
  * Encode-on-write into a paged cache ("aither-kvcache", section "Custom
  * inference loop": encode where the K/V of new tokens are written; the
  * slot-mapping form of serving engines): token t of x is encoded and written

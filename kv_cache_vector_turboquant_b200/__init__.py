@@ -39,6 +39,8 @@ from ._binding import (  # noqa: F401
     tq_device_error,
     tq_encode,
     tq_encode_append,
+    tq_encode_os,
+    tq_decode_os,
     tq_encode_slots,
     tq_get_tables,
     tq_status_string,
@@ -99,6 +101,28 @@ class TurboQuant:
         _require(d == self.head_dim, "last dim must be head_dim")
         s_max = cache_packed.shape[1]
         tq_encode_append(self.ctx, x, n_seq, h, cache_packed, cache_norms, s_max, slot, stream)
+
+    def encode_os(self, x, stream=None):
+        """Offset + fp16-scale variant: x [..., d] fp16 -> (packed [..., P]
+        uint8, side [...] int32 = fp16 offset | fp16 scale << 16)."""
+        import torch
+
+        _require(x.shape[-1] == self.head_dim, "last dim must be head_dim")
+        lead = x.shape[:-1]
+        n = x.numel() // self.head_dim
+        packed = torch.empty(*lead, self.packed_bytes, dtype=torch.uint8, device=x.device)
+        side = torch.empty(lead, dtype=torch.int32, device=x.device)
+        tq_encode_os(self.ctx, x, n, packed, side, stream)
+        return packed, side
+
+    def decode_os(self, packed, side, stream=None):
+        import torch
+
+        lead = packed.shape[:-1]
+        n = packed.numel() // self.packed_bytes
+        out = torch.empty(*lead, self.head_dim, dtype=torch.float16, device=packed.device)
+        tq_decode_os(self.ctx, packed, side, n, out, stream)
+        return out
 
     def encode_slots(self, x, cache_packed, cache_norms, slot_mapping, stream=None):
         """Encode-on-write: x [n_tok, h, d] into slot slot_mapping[t] of a pool

@@ -36,6 +36,8 @@ _PROTOS = {
     "tq_decode": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_append": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_slots": (_c_int, [_vp, _vp, _c_i64, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
+    "tq_encode_os": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
+    "tq_decode_os": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_attend_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64]),
     "tq_attend_decode": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64,
                                   _vp, _vp, _vp, _c_size, _vp]),
@@ -167,6 +169,14 @@ def tq_encode_append(ctx: Ctx, x, n_seq: int, h: int, cache_packed, cache_norms,
                      stream=None) -> None:
     _check(_lib.tq_encode_append(ctx.handle, _ptr(x), int(n_seq), int(h), _ptr(cache_packed), _ptr(cache_norms),
                                  int(s_max), _ptr(slot), _stream(stream)), "tq_encode_append")
+
+
+def tq_encode_os(ctx: Ctx, x, n: int, packed, side, stream=None) -> None:
+    _check(_lib.tq_encode_os(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(side), _stream(stream)), "tq_encode_os")
+
+
+def tq_decode_os(ctx: Ctx, packed, side, n: int, x, stream=None) -> None:
+    _check(_lib.tq_decode_os(ctx.handle, _ptr(packed), _ptr(side), int(n), _ptr(x), _stream(stream)), "tq_decode_os")
 
 
 def tq_encode_slots(ctx: Ctx, x, n_tok: int, h: int, cache_packed, cache_norms, num_slots: int, slot_mapping,

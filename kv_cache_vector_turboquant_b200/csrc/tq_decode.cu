@@ -92,7 +92,7 @@ TQ_DEV f2 lds_f2(uint32_t addr) {
   return r;
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool OS>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     decode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ DecArgs a) {
   using Cfg = DecCfg<D, BITS>;
@@ -249,7 +249,16 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
       }
     }
 
-    // ---- scale by N/d, round to fp16, apply the signs, stage the tile
+    // ---- scale by N/d, round to fp16, apply the signs, stage the tile. The
+    // offset variant's side word is fp16 offset | fp16 scale << 16: it
+    // scales by scale/d, flips signs in f32 and adds the offset before the
+    // rounding.
+    float mu = 0.f;
+    if constexpr (OS) {
+      const uint32_t sw32 = __float_as_uint(nrm);
+      mu = __half2float(__ushort_as_half((unsigned short)(sw32 & 0xffffu)));
+      nrm = __half2float(__ushort_as_half((unsigned short)(sw32 >> 16)));
+    }
     const float sc = nrm * (1.0f / (float)D);
     const f2 sc2 = make_float2(sc, sc);
     // the previous tile's bulk store must have finished reading the buffer
@@ -258,6 +267,30 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
 #pragma unroll
     for (int c = 0; c < C / 8; ++c) {
       uint32_t h[4];
+      if constexpr (OS) {
+        const f2 mu2 = make_float2(mu, mu);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i0 = 2 * (4 * c + q);  // coordinate within this lane's part
+          uint32_t m0, m1;
+          if constexpr (LPV == 1) {
+            m0 = T.sign_f32[i0], m1 = T.sign_f32[i0 + 1];
+          } else if constexpr (LPV == 2) {
+            m0 = T.sign_f32[i0], m1 = T.sign_f32[i0 + 1];
+            if (part) m0 ^= T.sign_f32_dx[i0], m1 ^= T.sign_f32_dx[i0 + 1];
+          } else {
+            const uint32_t mh = reinterpret_cast<const uint32_t*>(my_masks)[4 * c + q];
+            m0 = (mh << 16) & 0x80000000u, m1 = mh & 0x80000000u;
+          }
+          f2 y = mul2(v[4 * c + q], sc2);
+          y = make_float2(__uint_as_float(__float_as_uint(y.x) ^ m0), __uint_as_float(__float_as_uint(y.y) ^ m1));
+          y = add2(y, mu2);
+          const __half2 hv = __floats2half2_rn(y.x, y.y);
+          h[q] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(orow + 16 * (c ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
+        continue;
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const f2 y = mul2(v[4 * c + q], sc2);
@@ -289,7 +322,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   if (lane == 0) bulk_wait_all<0>();
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool OS>
 static cudaError_t launch_decode_t(const tq_codec_tables& T, DecArgs a, cudaStream_t st) {
   using Cfg = DecCfg<D, BITS>;
   constexpr size_t smem = DecSmem<D, BITS>::BYTES;
@@ -299,7 +332,7 @@ static cudaError_t launch_decode_t(const tq_codec_tables& T, DecArgs a, cudaStre
   static std::atomic<uint64_t> configured{0};
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(decode_kernel<D, BITS, OS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -329,7 +362,7 @@ static cudaError_t launch_decode_t(const tq_codec_tables& T, DecArgs a, cudaStre
     const int64_t tiles = (n + Cfg::VPW - 1) / Cfg::VPW;
     const int64_t ctas = (tiles + DEC_WARPS - 1) / DEC_WARPS;
     const int grid = (int)std::min<int64_t>(ctas, (int64_t)tq_sm_count(dev));
-    decode_kernel<D, BITS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
+    decode_kernel<D, BITS, OS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -355,10 +388,33 @@ tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* n
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorInvalidValue;
 #define TQ_DEC_CASE(D_, B_) \
-  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_t<D_, B_>(ctx->t, a, st);
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_t<D_, B_, false>(ctx->t, a, st);
   TQ_DEC_CASE(64, 2) TQ_DEC_CASE(64, 3) TQ_DEC_CASE(64, 4)
   TQ_DEC_CASE(128, 2) TQ_DEC_CASE(128, 3) TQ_DEC_CASE(128, 4)
   TQ_DEC_CASE(256, 2) TQ_DEC_CASE(256, 3) TQ_DEC_CASE(256, 4)
 #undef TQ_DEC_CASE
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_launch_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,
+                              void* stream) {
+  if (n == 0) return TQ_OK;
+  DecArgs a;
+  memset(&a, 0, sizeof(a));
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.norms = reinterpret_cast<const float*>(side);  // side words travel in the norms slot, bit for bit
+  a.n = n;
+  a.x = static_cast<__half*>(x);
+  a.err = tq_error_word();
+  if (!a.err) return TQ_ERR_CUDA;
+  a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+#define TQ_DECOS_CASE(D_, B_) \
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_t<D_, B_, true>(ctx->t, a, st);
+  TQ_DECOS_CASE(64, 2) TQ_DECOS_CASE(64, 3) TQ_DECOS_CASE(64, 4)
+  TQ_DECOS_CASE(128, 2) TQ_DECOS_CASE(128, 3) TQ_DECOS_CASE(128, 4)
+  TQ_DECOS_CASE(256, 2) TQ_DECOS_CASE(256, 3) TQ_DECOS_CASE(256, 4)
+#undef TQ_DECOS_CASE
   return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

@@ -73,6 +73,7 @@ struct EncArgs {
   int64_t s_max;        // cache positions per sequence (append mode) or slots of the pool (slot_abs)
   int slot_abs;         // 1: row slot[token] of a pool of s_max rows; a negative slot is skipped silently
   uint32_t* err;
+  uint32_t* side;        // offset variant: per vector fp16 offset | fp16 scale << 16 (instead of norms)
   int fault_inject;      // test hook: 1 = never issue the tile copies
   long long wait_limit;  // bound on each mbarrier wait, SM cycles
 };
@@ -131,6 +132,23 @@ TQ_DEV f2 first_butterfly(uint32_t h2) {
   return make_float2(s, d);
 }
 
+// acc + x0 + x1 for the fp16 pair in h2 (two mixed-precision adds).
+TQ_DEV float add_f16_pair(uint32_t h2, float acc) {
+  const uint16_t x0 = (uint16_t)(h2 & 0xffffu), x1 = (uint16_t)(h2 >> 16);
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(acc) : "h"(x0), "f"(acc));
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(acc) : "h"(x1), "f"(acc));
+  return acc;
+}
+
+// (x0 - mu, x1 - mu) in f32 for the fp16 pair in h2, each rounded once.
+TQ_DEV f2 sub_offset_pair(uint32_t h2, float mu) {
+  const uint16_t x0 = (uint16_t)(h2 & 0xffffu), x1 = (uint16_t)(h2 >> 16);
+  float y0, y1;
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(y0) : "h"(x0), "f"(mu));
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(y1) : "h"(x1), "f"(mu));
+  return make_float2(y0, y1);
+}
+
 // Pack code m (< 2^BITS) of coordinate i into the lane's word array.
 template <int BITS, int WL>
 TQ_DEV void put_code(uint32_t (&words)[WL], int i, uint32_t m) {
@@ -165,10 +183,10 @@ TQ_DEV uint32_t swz_addr(uint32_t stage_addr, int r, int k) {
 // rotated f32 values (published by the source lane); on return scratch[j]
 // holds, as a uint32, the exact code of coordinate j for every bit j of the
 // returned mask. Called by the whole warp; rare, so kept out of line.
-template <int D, int BITS>
+template <int D, int BITS, bool OS>
 __device__ __noinline__ uint32_t recheck_group(float* scratch, float srcR, float qoff, float gq, uint32_t lut_lane,
                                                uint32_t st_addr, int row0, int gi0, const uint32_t* smask,
-                                               const float* sbound) {
+                                               const float* sbound, float mu, float nq) {
   constexpr int C = EncCfg<D, BITS>::C;
   constexpr uint32_t FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
@@ -179,27 +197,33 @@ __device__ __noinline__ uint32_t recheck_group(float* scratch, float srcR, float
   const uint2 ent = lds_u2(qb * 128u + lut_lane);
   const float dlj = __uint_as_float(ent.x) - q;
   const uint32_t cm = __ballot_sync(FULL, fabsf(dlj) < gq);
-  // N in fp64 from the fp16 inputs still in the stage
-  double sq = 0.0;
-#pragma unroll
-  for (int t = 0; t < D / 32; ++t) {
-    const int k = lane + 32 * t;
-    const double xk = (double)__half2float(__ushort_as_half(lds_u16(swz_addr(st_addr, row0 + k / C, k % C))));
-    sq = fma(xk, xk, sq);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(FULL, sq, o);
-  const double n64 = sqrt(sq);
-  uint32_t code = 0;
-  for (uint32_t c2 = cm; c2; c2 &= c2 - 1) {
-    const int j = __ffs(c2) - 1;
-    const int gi = gi0 + j;  // coordinate index in the vector
-    // w_gi = sum_k s_k (-1)^popcount(gi & k) x_k: exact in fp64 for fp16 x
-    double ps = 0.0;
+  // N in fp64 from the fp16 inputs still in the stage (the offset variant
+  // compares against its stored fp16 scale instead)
+  double n64 = (double)nq;
+  if constexpr (!OS) {
+    double sq = 0.0;
 #pragma unroll
     for (int t = 0; t < D / 32; ++t) {
       const int k = lane + 32 * t;
       const double xk = (double)__half2float(__ushort_as_half(lds_u16(swz_addr(st_addr, row0 + k / C, k % C))));
+      sq = fma(xk, xk, sq);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(FULL, sq, o);
+    n64 = sqrt(sq);
+  }
+  uint32_t code = 0;
+  for (uint32_t c2 = cm; c2; c2 &= c2 - 1) {
+    const int j = __ffs(c2) - 1;
+    const int gi = gi0 + j;  // coordinate index in the vector
+    // w_gi = sum_k s_k (-1)^popcount(gi & k) y_k with y = x (or x - offset):
+    // exact in fp64 for fp16 x and offset
+    double ps = 0.0;
+#pragma unroll
+    for (int t = 0; t < D / 32; ++t) {
+      const int k = lane + 32 * t;
+      double xk = (double)__half2float(__ushort_as_half(lds_u16(swz_addr(st_addr, row0 + k / C, k % C))));
+      if constexpr (OS) xk -= (double)mu;
       const uint32_t sbit = (smask[k >> 1] >> (15 + 16 * (k & 1))) & 1u;
       const uint32_t neg = sbit ^ (uint32_t)(__popc(gi & k) & 1);
       ps += neg ? -xk : xk;
@@ -218,7 +242,7 @@ __device__ __noinline__ uint32_t recheck_group(float* scratch, float srcR, float
   return cm;
 }
 
-template <int D, int BITS, int W>
+template <int D, int BITS, int W, bool OS>
 __global__ void __launch_bounds__(W * 32, 1)
     encode_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ EncArgs a) {
   using Cfg = EncCfg<D, BITS>;
@@ -314,6 +338,26 @@ __global__ void __launch_bounds__(W * 32, 1)
     const uint32_t st_addr = stage0 + (uint32_t)(stage * Cfg::STAGE);
     const uint32_t my_row = st_addr + row_off;
 
+    // ---- offset variant: the vector's mean, rounded to fp16, is subtracted first
+    float mu = 0.f;
+    if constexpr (OS) {
+      float sx[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int b = 0; b < Cfg::BOXES; ++b) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 r = lds_u4(my_row + (uint32_t)(b * ENC_BOX_BYTES) + ((c ^ sw) << 4));
+          const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) sx[q] = add_f16_pair(w4[q], sx[q]);
+        }
+      }
+      float sum = (sx[0] + sx[1]) + (sx[2] + sx[3]);
+#pragma unroll
+      for (int m = 1; m < LPV; m <<= 1) sum += __shfl_xor_sync(FULL, sum, m);
+      mu = __half2float(__float2half_rn(sum * (1.0f / (float)D)));
+    }
+
     // ---- load, sign flip (XOR of fp16 sign bits), first butterfly stage
     f2 v[NP];
     f2 acc[4];
@@ -324,6 +368,28 @@ __global__ void __launch_bounds__(W * 32, 1)
         const uint4 r = lds_u4(my_row + (uint32_t)(b * ENC_BOX_BYTES) + ((c ^ sw) << 4));
         const int k0 = b * 32 + c * 4;  // first pair of the chunk
         uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+        if constexpr (OS) {
+          // y = x - offset in f32, then the sign flip on the f32 values
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i0 = 2 * (k0 + q);  // coordinate within this lane's part
+            uint32_t m0, m1;
+            if constexpr (LPV == 1) {
+              m0 = T.sign_f32[i0], m1 = T.sign_f32[i0 + 1];
+            } else if constexpr (LPV == 2) {
+              m0 = T.sign_f32[i0], m1 = T.sign_f32[i0 + 1];
+              if (part) m0 ^= T.sign_f32_dx[i0], m1 ^= T.sign_f32_dx[i0 + 1];
+            } else {
+              const uint32_t mh = smask[part * NP + k0 + q];
+              m0 = (mh << 16) & 0x80000000u, m1 = mh & 0x80000000u;
+            }
+            const f2 y = sub_offset_pair(w4[q], mu);
+            const float y0 = __uint_as_float(__float_as_uint(y.x) ^ m0), y1 = __uint_as_float(__float_as_uint(y.y) ^ m1);
+            v[k0 + q] = make_float2(y0 + y1, y0 - y1);
+            acc[q] = (k0 == 0) ? mul2(v[q], v[q]) : fma2(v[k0 + q], v[k0 + q], acc[q]);
+          }
+          continue;
+        }
         if constexpr (LPV <= 2) {  // masks from the constant bank
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -347,7 +413,13 @@ __global__ void __launch_bounds__(W * 32, 1)
     float sum2 = s4.x + s4.y;
 #pragma unroll
     for (int m = 1; m < LPV; m <<= 1) sum2 += __shfl_xor_sync(FULL, sum2, m);
-    const float nrm = sqrtf(0.5f * sum2);
+    float nrm = sqrtf(0.5f * sum2);
+    uint32_t side_word = 0;
+    if constexpr (OS) {  // the scale is stored in fp16 and the codes are taken relative to it
+      const __half n16 = __float2half_rn(nrm);
+      nrm = __half2float(n16);
+      side_word = (uint32_t)__half_as_ushort(__float2half_rn(mu)) | ((uint32_t)__half_as_ushort(n16) << 16);
+    }
 
     // ---- remaining Walsh-Hadamard stages: in registers, then across the lanes of the vector
     wht_pairs<NP>(v);
@@ -366,7 +438,7 @@ __global__ void __launch_bounds__(W * 32, 1)
     // ---- quantize + pack, 32 coordinates (one guard group) at a time; a
     // group with a coordinate inside the guard band is redone at once, while
     // its rotated values are still in registers
-    const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite vector
+    const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite vector (or fp16 scale)
     const float R = special ? 0.f : __fdiv_rn(Rscale, nrm);
     uint32_t words[WL];
 #pragma unroll
@@ -412,8 +484,9 @@ __global__ void __launch_bounds__(W * 32, 1)
           }
         }
         __syncwarp();
-        const uint32_t cm = recheck_group<D, BITS>(scratch, srcR, qoff, gq, lut_lane, st_addr, row0,
-                                                   src_part * C + g * 32, smask, sbound);
+        const float src_mu = __shfl_sync(FULL, mu, src), src_nq = __shfl_sync(FULL, nrm, src);
+        const uint32_t cm = recheck_group<D, BITS, OS>(scratch, srcR, qoff, gq, lut_lane, st_addr, row0,
+                                                       src_part * C + g * 32, smask, sbound, src_mu, src_nq);
         if (lane == src) {
           for (uint32_t c2 = cm; c2; c2 &= c2 - 1) {
             const int j = __ffs(c2) - 1;
@@ -436,7 +509,12 @@ __global__ void __launch_bounds__(W * 32, 1)
 #pragma unroll
           for (int w = 0; w < WL; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
         }
-        if (part == 0) a.norms[(r0 + lane) / LPV] = nrm;
+        if (part == 0) {
+          if constexpr (OS)
+            a.side[(r0 + lane) / LPV] = side_word;
+          else
+            a.norms[(r0 + lane) / LPV] = nrm;
+        }
       }
     } else if (active) {
       const int64_t r = a.vec_base + (r0 + lane) / LPV;
@@ -468,18 +546,19 @@ __global__ void __launch_bounds__(W * 32, 1)
 constexpr int ENC_WARPS_BULK = 16;
 constexpr int ENC_WARPS_SMALL = 2;
 
-template <int D, int BITS, int W>
+template <int D, int BITS, int W, bool OS>
 static cudaError_t configure_encode(size_t smem, int dev) {
   static std::atomic<uint64_t> configured{0};  // one bit per device
   const uint64_t bit = 1ull << (dev & 63);
   if (configured.load() & bit) return cudaSuccess;
   const cudaError_t e =
-      cudaFuncSetAttribute(encode_kernel<D, BITS, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(encode_kernel<D, BITS, W, OS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) configured.fetch_or(bit);
   return e;
 }
 
-template <int D, int BITS>
+// OS: the offset + fp16-scale variant (bulk launches only, 16 warps).
+template <int D, int BITS, bool OS>
 static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const void* x, cudaStream_t st) {
   using Cfg = EncCfg<D, BITS>;
   int dev = 0;
@@ -487,8 +566,8 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
   if (e != cudaSuccess) return e;
   const size_t smem_bulk = EncSmem<D, BITS, ENC_WARPS_BULK>::bytes(T.lut_cells);
   const size_t smem_small = EncSmem<D, BITS, ENC_WARPS_SMALL>::bytes(T.lut_cells);
-  if ((e = configure_encode<D, BITS, ENC_WARPS_BULK>(smem_bulk, dev)) != cudaSuccess) return e;
-  if ((e = configure_encode<D, BITS, ENC_WARPS_SMALL>(smem_small, dev)) != cudaSuccess) return e;
+  if ((e = configure_encode<D, BITS, ENC_WARPS_BULK, OS>(smem_bulk, dev)) != cudaSuccess) return e;
+  if (!OS && (e = configure_encode<D, BITS, ENC_WARPS_SMALL, false>(smem_small, dev)) != cudaSuccess) return e;
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
   if (!enc) return cudaErrorNotSupported;
   const int sms = tq_sm_count(dev);
@@ -497,13 +576,17 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
   const int64_t n_total = a.n;
   uint8_t* packed0 = a.packed;
   float* norms0 = a.norms;
+  uint32_t* side0 = a.side;
   for (int64_t off = 0; off < n_total; off += max_vec) {
     const int64_t n = std::min(max_vec, n_total - off);
     a.n = n;
     a.vec_base = off;
     if (a.slot == nullptr) {
       a.packed = packed0 + off * Cfg::P;
-      a.norms = norms0 + off;
+      if (OS)
+        a.side = side0 + off;
+      else
+        a.norms = norms0 + off;
     }
     const cuuint64_t dims[2] = {(cuuint64_t)Cfg::C, (cuuint64_t)(n * Cfg::LPV)};
     const cuuint64_t strides[1] = {(cuuint64_t)Cfg::C * 2};
@@ -515,13 +598,13 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
     const int64_t tiles = (n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
-    if (tiles <= (int64_t)ENC_WARPS_SMALL * sms) {
+    if (!OS && tiles <= (int64_t)ENC_WARPS_SMALL * sms) {
       const int grid = (int)((tiles + ENC_WARPS_SMALL - 1) / ENC_WARPS_SMALL);
-      encode_kernel<D, BITS, ENC_WARPS_SMALL><<<grid, ENC_WARPS_SMALL * 32, smem_small, st>>>(T, a);
+      encode_kernel<D, BITS, ENC_WARPS_SMALL, false><<<grid, ENC_WARPS_SMALL * 32, smem_small, st>>>(T, a);
     } else {
       const int64_t ctas_needed = (tiles + ENC_WARPS_BULK - 1) / ENC_WARPS_BULK;
       const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)sms);
-      encode_kernel<D, BITS, ENC_WARPS_BULK><<<grid, ENC_WARPS_BULK * 32, smem_bulk, st>>>(T, a);
+      encode_kernel<D, BITS, ENC_WARPS_BULK, OS><<<grid, ENC_WARPS_BULK * 32, smem_bulk, st>>>(T, a);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -554,10 +637,35 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
   cudaError_t e = cudaErrorInvalidValue;
   const tq_codec_tables& T = ctx->t;
 #define TQ_ENC_CASE(D_, B_) \
-  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_>(T, a, x, st);
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_, false>(T, a, x, st);
   TQ_ENC_CASE(64, 2) TQ_ENC_CASE(64, 3) TQ_ENC_CASE(64, 4)
   TQ_ENC_CASE(128, 2) TQ_ENC_CASE(128, 3) TQ_ENC_CASE(128, 4)
   TQ_ENC_CASE(256, 2) TQ_ENC_CASE(256, 3) TQ_ENC_CASE(256, 4)
 #undef TQ_ENC_CASE
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_launch_encode_os(const tq_ctx* ctx, const void* x, int64_t n, void* packed, uint32_t* side,
+                              void* stream) {
+  if (n == 0) return TQ_OK;
+  EncArgs a;
+  memset(&a, 0, sizeof(a));
+  a.n = n;
+  a.packed = static_cast<uint8_t*>(packed);
+  a.side = side;
+  a.h = 1;
+  a.s_max = 1;
+  a.err = tq_error_word();
+  if (!a.err) return TQ_ERR_CUDA;
+  a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  const tq_codec_tables& T = ctx->t;
+#define TQ_ENCOS_CASE(D_, B_) \
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_, true>(T, a, x, st);
+  TQ_ENCOS_CASE(64, 2) TQ_ENCOS_CASE(64, 3) TQ_ENCOS_CASE(64, 4)
+  TQ_ENCOS_CASE(128, 2) TQ_ENCOS_CASE(128, 3) TQ_ENCOS_CASE(128, 4)
+  TQ_ENCOS_CASE(256, 2) TQ_ENCOS_CASE(256, 3) TQ_ENCOS_CASE(256, 4)
+#undef TQ_ENCOS_CASE
   return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

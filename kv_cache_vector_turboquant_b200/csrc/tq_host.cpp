@@ -139,6 +139,8 @@ tq_status tq_create(int head_dim, int bits, uint64_t seed, tq_ctx** out) {
     t.sign_h2[i / 2] = ((a >> 63) ? 0x8000u : 0u) | ((b >> 63) ? 0x80000000u : 0u);
   }
   for (int k = 0; k < 32 && k + 32 < head_dim / 2; ++k) t.sign_h2_dx[k] = t.sign_h2[k] ^ t.sign_h2[k + 32];
+  for (int i = 0; i < head_dim; ++i) t.sign_f32[i] = ((t.sign_h2[i / 2] >> (15 + 16 * (i & 1))) & 1u) << 31;
+  for (int i = 0; i < 64 && i + 64 < head_dim; ++i) t.sign_f32_dx[i] = t.sign_f32[i] ^ t.sign_f32[i + 64];
 
   double delta = 0.0, frac = 0.0;
   if (!choose_grid(t.bounds, L - 1, &delta, &frac)) {
@@ -224,6 +226,24 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
   if (!aligned(x_f16, 16) || !aligned(cache_packed, 16) || !aligned(cache_norms, 4) || !aligned(slot, 4))
     return TQ_ERR_ALIGNMENT;
   return tq_launch_encode(ctx, x_f16, (int64_t)n_seq * h, cache_packed, cache_norms, slot, h, s_max, stream, 0);
+}
+
+tq_status tq_encode_os(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, uint32_t* side,
+                       tq_stream stream) {
+  if (!ctx || n < 0) return TQ_ERR_INVALID_ARG;
+  if (n == 0) return TQ_OK;
+  if (!x_f16 || !packed || !side) return TQ_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(side, 4)) return TQ_ERR_ALIGNMENT;
+  return tq_launch_encode_os(ctx, x_f16, n, packed, side, stream);
+}
+
+tq_status tq_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x_f16,
+                       tq_stream stream) {
+  if (!ctx || n < 0) return TQ_ERR_INVALID_ARG;
+  if (n == 0) return TQ_OK;
+  if (!x_f16 || !packed || !side) return TQ_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(side, 4)) return TQ_ERR_ALIGNMENT;
+  return tq_launch_decode_os(ctx, packed, side, n, x_f16, stream);
 }
 
 tq_status tq_encode_slots(const tq_ctx* ctx, const void* x_f16, int64_t n_tok, int h, void* cache_packed,

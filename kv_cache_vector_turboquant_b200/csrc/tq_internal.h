@@ -21,6 +21,12 @@ struct tq_codec_tables {
   // 64-coordinate halves of a head_dim-128 vector (a lane holding the upper
   // half applies it on top of the lower half's mask).
   uint32_t sign_h2_dx[32];
+  // float32 sign masks per coordinate (bit 31 set <=> negated), and the
+  // change between the two 64-coordinate halves of a head_dim-128 vector
+  // (used by the offset + fp16-scale variant, which flips signs after
+  // subtracting the offset in f32)
+  uint32_t sign_f32[TQ_MAX_D];
+  uint32_t sign_f32_dx[64];
   float levels[TQ_MAX_L];      // format levels c_k (2^-14 grid), ascending
   float bounds[TQ_MAX_L - 1];  // decision boundaries t_j in z units (2^-15 grid)
   // Encode quantizer lookup table, in "q units" q = z * inv_delta + q_offset:
@@ -59,6 +65,10 @@ inline double tq_guard_z(int head_dim) { return head_dim <= 128 ? 1.0e-5 : 2.0e-
 tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
                            const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject,
                            int slot_abs = 0);
+tq_status tq_launch_encode_os(const tq_ctx* ctx, const void* x, int64_t n, void* packed, uint32_t* side,
+                              void* stream);
+tq_status tq_launch_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,
+                              void* stream);
 tq_status tq_launch_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n,
                            void* x, void* stream);
 tq_status tq_launch_attend(const tq_ctx* k, const tq_ctx* v, const void* q, int B, int hq, int hkv,

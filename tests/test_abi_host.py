@@ -205,3 +205,20 @@ def test_encode_slots_validation(K):
     assert _raw(K, fn, h, A + 8, 4, 8, A, A, 64, A, None) == K.TQ_ERR_ALIGNMENT
     assert _raw(K, fn, h, A, 4, 8, A, A + 2, 64, A, None) == K.TQ_ERR_ALIGNMENT
     assert _raw(K, fn, h, A, 0, 8, A, A, 64, A, None) == K.TQ_OK
+
+
+def test_offset_variant_validation(K):
+    ctx = K.tq_create(128, 4)
+    h = ctx.handle
+    A = 0x100000
+    # tq_encode_os(ctx, x, n, packed, side, stream); tq_decode_os(ctx, packed, side, n, x, stream)
+    assert _raw(K, "tq_encode_os", None, A, 4, A, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_os", h, A, -1, A, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_os", h, A, 0, A, A, None) == K.TQ_OK
+    assert _raw(K, "tq_decode_os", None, A, A, 4, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_decode_os", h, A, A, -1, A, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_decode_os", h, A, A, 0, A, None) == K.TQ_OK
+    assert _raw(K, "tq_encode_os", h, A, 4, A, None, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_encode_os", h, A + 2, 4, A, A, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_encode_os", h, A, 4, A, A + 2, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_decode_os", h, A, A + 1, 4, A, None) == K.TQ_ERR_ALIGNMENT

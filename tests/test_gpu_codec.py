@@ -274,6 +274,55 @@ def test_encode_slots_out_of_range_is_flagged(K, W):
     assert st == K.TQ_ERR_DEVICE and bits == K.TQ_DEVERR_SLOT_RANGE
 
 
+def _os_decode_ok(gpu16, exact, mu16):
+    """fp16 decode of the offset variant against the fp64 value of the same
+    bytes: within half an fp16 ulp of the exact value plus the two f32
+    roundings (product, sum with the offset)."""
+    g = np.asarray(gpu16, dtype=np.float64)
+    a = np.abs(exact)
+    ulp = np.where(a >= 2.0 ** -14, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10), 2.0 ** -24)
+    mu = np.abs(mu16.astype(np.float64))[:, None]
+    tol = 0.5 * ulp + 2.0 ** -22 * (mu + np.abs(exact - mu16.astype(np.float64)[:, None])) + 1e-30
+    return np.abs(g - exact) <= tol
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_offset_variant_matches_oracle(K, W, d, bits):
+    """Offset + fp16-scale variant on rows with random offsets and outliers
+    (ragged n): side data within one fp16 ulp of the oracle's (the GPU
+    accumulates the mean in f32), codes bit-exact given the GPU's side data,
+    decode of the same bytes within the fp16 rounding."""
+    n = 3001
+    g = torch.Generator().manual_seed(d * 7 + bits)
+    x = torch.randn(n, d, generator=g) * torch.exp(torch.randn(n, 1, generator=g))
+    x += torch.randn(n, 1, generator=g) * 3
+    hit = torch.rand(n, d, generator=g) < 0.005
+    x = torch.where(hit, x * 20, x).to(torch.float16)
+    x[0] = 0.0
+    x[1] = 2.5
+    tq = K.TurboQuant(d, bits)
+    packed, side = tq.encode_os(x.cuda())
+    dec = tq.decode_os(packed, side)
+    torch.cuda.synchronize()
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    xs = x.numpy()
+    side_u = side.cpu().numpy().view(np.uint32)
+    own = O.encode_os_detail(xs, bits, 42)
+    gmu = (side_u & 0xFFFF).astype(np.uint16).view(np.float16)
+    gn = (side_u >> 16).astype(np.uint16).view(np.float16)
+    from parity import fp16_ulp_distance
+    assert fp16_ulp_distance(gmu, own["mu16"]).max() <= 1
+    assert fp16_ulp_distance(gn, own["n16"]).max() <= 1
+    det = O.encode_os_detail(xs, bits, 42, side=side_u)
+    gp = packed.cpu().numpy()
+    assert code_mismatches(gp, det, bits, d) == 0
+    exact = O.decode_os_f64(gp, side_u, bits, 42, d)
+    assert np.all(_os_decode_ok(dec.cpu().numpy(), exact, gmu))
+    # the zero row decodes to zeros and the constant row to itself
+    assert torch.all(dec[0] == 0) and torch.all(dec[1].cpu() == x[1])
+
+
 def test_append_out_of_range_slot_is_skipped_and_flagged(K, W):
     tq = K.TurboQuant(128, 4)
     n_seq, h, s_max = 4, 8, 8
