@@ -460,6 +460,9 @@ __global__ void __launch_bounds__(ATT_WARPS * 32, 2) attend_partial_kernel(const
 // o = D_V H_pm o~ / d, rounded to fp16. One CTA of d threads per row.
 template <int D>
 __global__ void __launch_bounds__(D) attend_combine_kernel(const __grid_constant__ AttnArgs a) {
+  // launched as a programmatic dependent of the partial kernel: wait until
+  // that grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float o[D];
   const int h = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
   const int64_t base = ((int64_t)b * a.hq + h) * a.n_split;
@@ -513,11 +516,23 @@ using namespace tq;
 
 cudaError_t tq_launch_attend_combine(const AttnArgs& a, int d, cudaStream_t st) {
   const dim3 grid(a.hq, a.B);
-  if (d == 64) attend_combine_kernel<64><<<grid, 64, 0, st>>>(a);
-  else if (d == 128) attend_combine_kernel<128><<<grid, 128, 0, st>>>(a);
-  else if (d == 256) attend_combine_kernel<256><<<grid, 256, 0, st>>>(a);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  // programmatic dependent launch: the merge grid is set up while the
+  // partial kernel runs and starts as its CTAs retire (it waits for the
+  // partial grid's completion before reading the workspace)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(d);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (d == 64) return cudaLaunchKernelEx(&cfg, attend_combine_kernel<64>, a);
+  if (d == 128) return cudaLaunchKernelEx(&cfg, attend_combine_kernel<128>, a);
+  if (d == 256) return cudaLaunchKernelEx(&cfg, attend_combine_kernel<256>, a);
+  return cudaErrorInvalidValue;
 }
 
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max) {
