@@ -535,39 +535,56 @@ def run_ours(args, rank, world, local_rank):
 
 
 def _e2e(K, torch, S, steps, world, dist):
+    """End to end through the public API: every step copies each tensor's
+    fp16 rows from pinned host memory, encodes, copies codes and norms back,
+    copies them to the device again, decodes and copies the fp16 rows back,
+    at 2, 3 and 4 bits. K and V each run on their own stream with their own
+    device buffers, so one tensor's host-to-device copies overlap the other's
+    device-to-host copies and kernels."""
     n = S["n"]
     host_x = {t: S["xs"][t].cpu().pin_memory() for t in "KV"}
     host_p = {k: v.cpu().pin_memory() for k, v in S["packed"].items()}
     host_n = {k: v.cpu().pin_memory() for k, v in S["norms"].items()}
-    host_o = torch.empty(n, D, dtype=torch.float16).pin_memory()
-    dx = torch.empty(n, D, dtype=torch.float16, device="cuda")
-    dp = {b: torch.empty(n, S["codecs"][b].packed_bytes, dtype=torch.uint8, device="cuda") for b in BITS}
-    dn = torch.empty(n, dtype=torch.float32, device="cuda")
+    host_o = {t: torch.empty(n, D, dtype=torch.float16).pin_memory() for t in "KV"}
+    dx = {t: torch.empty(n, D, dtype=torch.float16, device="cuda") for t in "KV"}
+    dp = {(b, t): torch.empty(n, S["codecs"][b].packed_bytes, dtype=torch.uint8, device="cuda")
+          for b in BITS for t in "KV"}
+    dn = {t: torch.empty(n, dtype=torch.float32, device="cuda") for t in "KV"}
+    streams = {t: torch.cuda.Stream() for t in "KV"}
     h2d = d2h = 0
 
     def step():
-        nonlocal h2d, d2h
-        for b in BITS:
-            c = S["codecs"][b].ctx
-            for t in "KV":  # encode: x host -> device, codes back to the host
-                dx.copy_(host_x[t], non_blocking=True)
-                K.tq_encode(c, dx, n, dp[b], dn)
-                host_p[b, t].copy_(dp[b], non_blocking=True)
-                host_n[b, t].copy_(dn, non_blocking=True)
-            for t in "KV":  # decode: codes host -> device, fp16 rows back to the host
-                dp[b].copy_(host_p[b, t], non_blocking=True)
-                dn.copy_(host_n[b, t], non_blocking=True)
-                K.tq_decode(c, dp[b], dn, n, dx)
-                host_o.copy_(dx, non_blocking=True)
+        for t in "KV":
+            with torch.cuda.stream(streams[t]):
+                for b in BITS:
+                    c = S["codecs"][b].ctx
+                    p = dp[b, t]
+                    dx[t].copy_(host_x[t], non_blocking=True)  # encode: rows in, codes and norms out
+                    K.tq_encode(c, dx[t], n, p, dn[t])
+                    host_p[b, t].copy_(p, non_blocking=True)
+                    host_n[b, t].copy_(dn[t], non_blocking=True)
+                    p.copy_(host_p[b, t], non_blocking=True)  # decode: codes and norms in, rows out
+                    dn[t].copy_(host_n[b, t], non_blocking=True)
+                    K.tq_decode(c, p, dn[t], n, dx[t])
+                    host_o[t].copy_(dx[t], non_blocking=True)
 
-    step()
+    def run(k):
+        ev0 = _ev(torch)
+        ev0.record()
+        for t in "KV":
+            streams[t].wait_event(ev0)
+        for _ in range(k):
+            step()
+        for t in "KV":
+            torch.cuda.current_stream().wait_stream(streams[t])
+
+    run(1)
     torch.cuda.synchronize()
     e0, e1 = _ev(torch), _ev(torch)
     if world > 1:
         dist.barrier()
     e0.record()
-    for _ in range(steps):
-        step()
+    run(steps)
     e1.record()
     torch.cuda.synchronize()
     ms = reduce_max_ms(e0.elapsed_time(e1), world, dist, "cuda")
@@ -578,8 +595,8 @@ def _e2e(K, torch, S, steps, world, dist):
     fp16eq = 12 * 2 * D * n
     return {"value": job_throughput(fp16eq, steps, world, ms), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "note": "tq_encode/tq_decode with inputs copied from pinned host memory and results copied back, "
-                    "one stream"}
+            "note": "tq_encode/tq_decode with inputs copied from pinned host memory and results copied back; "
+                    "K and V on two streams (copies in one direction overlap the other tensor's)"}
 
 
 def run_reference(args):
