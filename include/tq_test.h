@@ -22,6 +22,20 @@ extern "C" {
 tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms,
                                  tq_stream stream);
 
+/*
+ * tq_encode through a chosen kernel, whatever n is:
+ *   path 1  the CUDA-core kernel (tq_encode's choice below
+ *           128 x SM-count vectors),
+ *   path 2  the tensor-core kernel (tq_encode's choice from there on),
+ *   path 3  the tensor-core kernel with its row copies withheld, like
+ *           tq_test_encode_stalled: TQ_DEVERR_TIMEOUT after about 10 ms per
+ *           wait, nothing written.
+ * Same arguments, alignment rules and asynchrony as tq_encode; n must be > 0;
+ * any other path is TQ_ERR_INVALID_ARG.
+ */
+tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms, int path,
+                              tq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

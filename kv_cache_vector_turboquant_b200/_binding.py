@@ -47,6 +47,7 @@ _PROTOS = {
                                         _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
+    "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _f = getattr(_lib, _name)
@@ -227,3 +228,10 @@ def tq_device_error(stream=None) -> tuple[int, int]:
 def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> int:
     """Test hook: encode with the row copies withheld; returns the launch status."""
     return _lib.tq_test_encode_stalled(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), _stream(stream))
+
+
+def tq_test_encode_path(ctx: Ctx, x, n: int, packed, norms, path: int, stream=None) -> int:
+    """Test hook: encode through kernel `path` (1 CUDA cores, 2 tensor cores, 3 tensor
+    cores with the row copies withheld); returns the launch status."""
+    return _lib.tq_test_encode_path(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), int(path),
+                                    _stream(stream))

@@ -37,6 +37,10 @@ TQ_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
+TQ_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 TQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

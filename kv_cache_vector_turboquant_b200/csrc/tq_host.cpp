@@ -206,6 +206,7 @@ tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packe
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
+  if (n >= tq_encode_tc_min_rows()) return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 0);
 }
 
@@ -316,6 +317,19 @@ tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n
   if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 1);
+}
+
+// Test hook (declared in include/tq_test.h): tq_encode through a chosen kernel.
+tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms, int path,
+                              tq_stream stream) {
+  if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
+  switch (path) {
+    case 1: return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 0);
+    case 2: return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
+    case 3: return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 1);
+    default: return TQ_ERR_INVALID_ARG;
+  }
 }
 
 }  // extern "C"

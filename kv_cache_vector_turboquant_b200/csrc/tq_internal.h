@@ -65,6 +65,12 @@ inline double tq_guard_z(int head_dim) { return head_dim <= 128 ? 1.0e-5 : 2.0e-
 tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
                            const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject,
                            int slot_abs = 0);
+// Bulk encode on the tensor cores (tq_encode_tc.cu): the same outputs as
+// tq_launch_encode without append slots. tq_encode uses it from
+// tq_encode_tc_min_rows() vectors on (one 128-vector tile per SM).
+tq_status tq_launch_encode_tc(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms, void* stream,
+                              int fault_inject);
+int64_t tq_encode_tc_min_rows(void);
 tq_status tq_launch_encode_os(const tq_ctx* ctx, const void* x, int64_t n, void* packed, uint32_t* side,
                               void* stream);
 tq_status tq_launch_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,

@@ -3,7 +3,8 @@
 * codes: bit-exact, except coordinates whose oracle value z lies within 1e-5
   of a decision boundary; those mismatches are counted and must stay below
   1e-6 of all coordinates (``max_boundary_frac``);
-* norms: relative error <= 1e-6;
+* norms: relative error <= 1e-6 (CUDA-core encode kernel) or 2e-6 (tensor-core
+  kernel, whose norm comes from the 16-point block transforms; bound 1.8e-6);
 * decoded fp16: <= 1 fp16 ulp from the oracle's decode of the same bytes;
 * attention: per output row, max |o - o_ref| / max |o_ref| <= 2e-3.
 """
@@ -16,6 +17,7 @@ import oracle as O
 
 BOUNDARY_BAND = 1e-5
 NORM_RTOL = 1e-6
+NORM_RTOL_TC = 2e-6
 ATTN_RTOL = 2e-3
 
 
@@ -37,11 +39,11 @@ def code_mismatches(gpu_packed: np.ndarray, detail: dict, bits: int, d: int, max
     return n
 
 
-def assert_norms(gpu_norms: np.ndarray, detail: dict):
+def assert_norms(gpu_norms: np.ndarray, detail: dict, rtol: float = NORM_RTOL):
     g = np.asarray(gpu_norms, dtype=np.float64).reshape(-1)
     ref = detail["norm64"]
     err = np.abs(g - ref)
-    lim = NORM_RTOL * np.abs(ref)
+    lim = rtol * np.abs(ref)
     assert np.all(err <= lim), f"norm rel err {np.max(err / np.maximum(np.abs(ref), 1e-300)):.3g}"
 
 

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity import assert_decode_ulp, assert_norms, code_mismatches
+from parity import NORM_RTOL_TC, assert_decode_ulp, assert_norms, code_mismatches
 
 pytestmark = pytest.mark.gpu
 
@@ -125,7 +125,7 @@ def test_llama_layer_full_size_sampled(K, W, bits):
         gp = packed[rows.cuda()].cpu().numpy()
         gn = norms[rows.cuda()].cpu().numpy()
         assert code_mismatches(gp, det, bits, 128) == 0
-        assert_norms(gn, det)
+        assert_norms(gn, det, NORM_RTOL_TC)  # a bulk launch: the tensor-core kernel
         assert_decode_ulp(dec[rows.cuda()].cpu().numpy(), O.decode(gp, gn, bits, 42, 128))
         # whole-tensor property for the isotropic tensor (V: iid N(0,1), so the
         # unit direction is uniform on the sphere): the distortion equals the
@@ -159,7 +159,7 @@ def test_long_context_layer_sampled(K, W, layer):
         det = O.encode_detail(xs, 3, 42)
         gp, gn = packed[rows].cpu().numpy(), norms[rows].cpu().numpy()
         assert code_mismatches(gp, det, 3, 128) == 0
-        assert_norms(gn, det)
+        assert_norms(gn, det, NORM_RTOL_TC)  # a bulk launch: the tensor-core kernel
         assert_decode_ulp(dec[rows].cpu().numpy(), O.decode(gp, gn, 3, 42, 128))
         del packed, norms, dec
     assert K.tq_device_error()[0] == K.TQ_OK
