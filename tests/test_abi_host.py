@@ -125,6 +125,19 @@ def test_encode_decode_validation(K):
     assert _raw(K, "tq_decode", h, A, C, 4, B_ + 8, None) == K.TQ_ERR_ALIGNMENT
 
 
+def test_encode_path_hook_validation(K):
+    """The test hook that picks the encode kernel validates before launching."""
+    ctx = K.tq_create(128, 4)
+    h = ctx.handle
+    A, B_, C = 0x10000, 0x20000, 0x30000
+    for bad_path in (0, 4, -1):
+        assert _raw(K, "tq_test_encode_path", h, A, 4, B_, C, bad_path, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_encode_path", None, A, 4, B_, C, 2, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_encode_path", h, A, 0, B_, C, 2, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_encode_path", h, A + 8, 4, B_, C, 2, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_test_encode_path", h, A, 4, B_ + 4, C, 2, None) == K.TQ_ERR_ALIGNMENT
+
+
 def test_append_validation(K):
     ctx = K.tq_create(128, 3)
     h = ctx.handle
