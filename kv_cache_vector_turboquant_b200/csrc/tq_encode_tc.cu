@@ -26,9 +26,10 @@
 //  * three epilogue warpgroups (two at d = 256) take turns on the tiles, one
 //    vector per thread (TMEM lane = tile row): sum_{b,j} S^2 = 16 ||x||^2
 //    gives the norm; the remaining log2(d/16) butterfly stages run in
-//    registers with packed f32x2 on 2 positions j at a time; the quantiser,
-//    guard band and fp64 recheck are those of encode_kernel; each thread
-//    stores its packed row and norm.
+//    registers with packed f32x2 on 4 positions j at a time (2 at d = 256),
+//    two such chunks per loop iteration; the quantiser, guard band and fp64
+//    recheck are those of encode_kernel; each thread stores its packed row
+//    and norm.
 //
 // Exactness: the tensor core's arithmetic for kind::f16 with f32 accumulation
 // was measured on B200 (every product exact; each addend's magnitude cut to a
@@ -80,8 +81,7 @@ struct TcCfg {
   // JC codes 2^(BITS-1) (the code of a zero or non-finite vector), BITS apart
   static constexpr uint32_t HALF_FIELD = (uint32_t)(L / 2) * (JC == 4 ? (1u | 1u << BITS | 1u << 2 * BITS | 1u << 3 * BITS)
                                                                       : (1u | 1u << BITS));
-  // shared memory, from a 1024-aligned base
-  static constexpr int STAGE0 = 0;
+  // shared memory, from a 1024-aligned base: the stages first
   static constexpr int BREG = STAGES * TILE_BYTES;   // NB/4 regions of 16 rows x 128 B
   static constexpr int BAR = BREG + NB / 4 * 2048;   // full, empty, tfull, tempty, done
   static constexpr int NBARS = 2 * STAGES + 2 * NACC + 1;
