@@ -36,6 +36,21 @@ tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n
 tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms, int path,
                               tq_stream stream);
 
+/*
+ * One fifth-generation tensor-core MMA (tcgen05.mma kind::f16, M = 128,
+ * N = K = 16, f32 accumulator starting from zero), with the shared-memory
+ * layout and tensor-memory readback of the tensor-core encode kernel:
+ *   d[m][n] = sum_k a[m][k] * b[n][k]
+ *   a_f16  device, [128][16] fp16 (row-major), 2-byte aligned;
+ *   b_f16  device, [16][16] fp16 (row-major: b[n][k]), 2-byte aligned;
+ *   d      device, [128][16] float32 out, 4-byte aligned.
+ * Lets the tests check, on the GPU the library runs on, the rounding that the
+ * encode kernel's exactness argument assumes. One CTA, asynchronous on
+ * `stream`; TQ_ERR_INVALID_ARG for a null pointer, TQ_ERR_ALIGNMENT for a
+ * misaligned one; a wait that runs out is reported through tq_device_error.
+ */
+tq_status tq_test_umma_block(const void* a_f16, const void* b_f16, float* d, tq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,6 +48,7 @@ _PROTOS = {
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
+    "tq_test_umma_block": (_c_int, [_vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _f = getattr(_lib, _name)
@@ -228,6 +229,11 @@ def tq_device_error(stream=None) -> tuple[int, int]:
 def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> int:
     """Test hook: encode with the row copies withheld; returns the launch status."""
     return _lib.tq_test_encode_stalled(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), _stream(stream))
+
+
+def tq_test_umma_block(a, b, d, stream=None) -> int:
+    """Test hook: one tcgen05 MMA d[128,16] = a[128,16] @ b[16,16]^T (fp16 in, f32 out)."""
+    return _lib.tq_test_umma_block(_ptr(a), _ptr(b), _ptr(d), _stream(stream))
 
 
 def tq_test_encode_path(ctx: Ctx, x, n: int, packed, norms, path: int, stream=None) -> int:

@@ -138,6 +138,15 @@ def test_encode_path_hook_validation(K):
     assert _raw(K, "tq_test_encode_path", h, A, 4, B_ + 4, C, 2, None) == K.TQ_ERR_ALIGNMENT
 
 
+def test_umma_block_hook_validation(K):
+    A, B_, C = 0x10000, 0x20000, 0x30000
+    assert _raw(K, "tq_test_umma_block", None, B_, C, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_umma_block", A, None, C, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_umma_block", A, B_, None, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_umma_block", A + 1, B_, C, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_test_umma_block", A, B_, C + 2, None) == K.TQ_ERR_ALIGNMENT
+
+
 def test_append_validation(K):
     ctx = K.tq_create(128, 3)
     h = ctx.handle

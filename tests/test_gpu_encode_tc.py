@@ -167,3 +167,101 @@ def test_tc_bounded_wait_times_out_and_context_survives(K, W):
     assert K.tq_device_error() == (K.TQ_OK, 0)
     det = O.encode_detail(x.cpu().numpy(), 4, 42)
     assert code_mismatches(p2.cpu().numpy(), det, 4, 128) == 0
+
+
+# ---------------------------------------------------------------- the tensor core's arithmetic
+# The tensor-core encode kernel's exactness argument assumes, for one
+# kind::f16 MMA with f32 accumulation and K = 16: products exact, each
+# addend's magnitude cut to a multiple of 2^(E-25) (E the exponent of the
+# largest addend), the sum rounded toward zero to f32. These tests pin that on
+# the GPU the library runs on.
+
+
+def _umma(K, a, b):
+    at = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float16)).cuda()
+    bt = torch.from_numpy(np.ascontiguousarray(b, dtype=np.float16)).cuda()
+    d = torch.zeros(128, 16, dtype=torch.float32, device="cuda")
+    assert K._binding.tq_test_umma_block(at, bt, d) == K.TQ_OK
+    torch.cuda.synchronize()
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    return d.cpu().numpy().astype(np.float64)
+
+
+def _round_toward_zero_f32(x):
+    from fractions import Fraction
+
+    x = Fraction(x)
+    if x == 0:
+        return 0.0
+    s, m = (1, x) if x > 0 else (-1, -x)
+    e = m.numerator.bit_length() - m.denominator.bit_length()
+    if Fraction(2) ** e > m:
+        e -= 1
+    ulp = Fraction(2) ** (e - 23)
+    return s * float((m // ulp) * ulp)
+
+
+def test_tensor_core_cuts_addends_at_2_pow_minus_25_and_rounds_toward_zero(K):
+    """Rows 1 (or -1) plus fifteen terms +-2^-t, t = 0 ... 39: the small terms
+    count in full for t <= 25 and vanish beyond; the sum is rounded toward zero."""
+    from fractions import Fraction
+
+    a = np.zeros((128, 16))
+    b = np.zeros((16, 16))
+    for r in range(128):
+        e = r % 25
+        a[r, 0] = -1.0 if (r // 25) % 2 else 1.0
+        a[r, 1:] = (-1.0 if (r // 50) % 2 else 1.0) * 2.0 ** -e
+    for n in range(16):
+        b[n, 0] = 1.0
+        b[n, 1:] = 2.0 ** -n
+    got = _umma(K, a, b)
+    for r in range(128):
+        for n in range(16):
+            t = r % 25 + n
+            small = Fraction(a[r, 1]) * Fraction(b[n, 1])
+            kept = Fraction(a[r, 0]) + (15 * small if t <= 25 else 0)
+            assert got[r, n] == _round_toward_zero_f32(kept), (r, n, t, got[r, n])
+
+
+@pytest.mark.parametrize("cls", ["normal", "outliers", "log-uniform", "one-large", "cancelling"])
+def test_tensor_core_error_within_the_bound_the_encode_kernel_uses(K, cls):
+    """+-1-weighted 16-term sums (the 16-point Hadamard blocks) of five input
+    classes: |S' - S| <= 15 * 2^(E-25) + 2^-23 |S| for every output."""
+    import math
+
+    g = np.random.default_rng(sum(map(ord, cls)))
+    worst = 0.0
+    for rep in range(8):
+        if cls == "normal":
+            a = g.standard_normal((128, 16))
+        elif cls == "outliers":
+            a = g.standard_normal((128, 16)) * np.where(g.random((128, 16)) < 0.06, 20.0, 1.0)
+        elif cls == "log-uniform":
+            a = np.where(g.random((128, 16)) < 0.5, -1.0, 1.0) * 2.0 ** (-24 + 39 * g.random((128, 16)))
+        elif cls == "one-large":
+            a = g.standard_normal((128, 16)) * 2.0 ** -8
+            a[np.arange(128), g.integers(0, 16, 128)] = 1024.0 * (1 + g.random(128))
+        else:
+            x = (g.standard_normal((128, 8)) * 100).astype(np.float16).astype(np.float64)
+            a = np.empty((128, 16))
+            a[:, 0::2] = x
+            a[:, 1::2] = -x + g.standard_normal((128, 8)) * 0.01
+        a = a.astype(np.float16).astype(np.float64)
+        b = np.where(g.random((16, 16)) < 0.5, -1.0, 1.0)
+        got = _umma(K, a, b)
+        for r in range(128):
+            for n in range(16):
+                p = a[r] * b[n]  # exact products
+                s = math.fsum(p)
+                mx = np.max(np.abs(p))
+                if mx == 0:
+                    assert got[r, n] == 0.0
+                    continue
+                e = math.floor(math.log2(mx))
+                # fifteen cut addends, then rounding toward zero of the cut sum
+                bound = 15 * 2.0 ** (e - 25) * (1 + 2.0 ** -23) + 2.0 ** -23 * abs(s)
+                err = abs(got[r, n] - s)
+                assert err <= bound, (cls, r, n, err, bound)
+                worst = max(worst, err / bound)
+    assert worst <= 1.0
