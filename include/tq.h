@@ -112,6 +112,12 @@ tq_status tq_get_tables(const tq_ctx* ctx, float* levels, float* boundaries, uin
  *           code i of a row occupies stream bits [i*bits, i*bits+bits),
  *           stream bit k = bit (k mod 8) of byte k/8.
  *   norms   device, [n] float32 out: the L2 norm of each input row.
+ * Codes are those of exact arithmetic (coordinates within a proven f32 error
+ * band of a decision boundary are redone in fp64); norms are within 2e-6 of
+ * the exact norm (relative). Launches of at least 128 x SM-count vectors run
+ * on the tensor cores (the 16-point Hadamard blocks as tcgen05 MMAs), smaller
+ * ones on the CUDA cores; both give the same codes, norms may differ in the
+ * last bits.
  * n == 0 is a no-op (pointers may then be NULL). Inputs and outputs must not
  * overlap. The call is asynchronous on `stream`.
  */
