@@ -130,6 +130,11 @@ tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packe
  *   packed  device, [n, tq_packed_bytes] uint8, 16-byte aligned.
  *   norms   device, [n] float32.
  *   x_f16   device, [n, head_dim] fp16 out, 16-byte aligned.
+ * H c is summed exactly; the only roundings are the product by
+ * norm / head_dim and the fp16 conversion. Launches of at least
+ * 128 x SM-count vectors at head_dim 64 and 128 run on the tensor cores (the
+ * 16-point Hadamard blocks as tcgen05 MMAs with A in tensor memory), other
+ * launches on the CUDA cores; the outputs are bit-identical.
  * n == 0 is a no-op. Asynchronous on `stream`.
  */
 tq_status tq_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,

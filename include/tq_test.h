@@ -37,6 +37,16 @@ tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, v
                               tq_stream stream);
 
 /*
+ * tq_decode through a chosen kernel, whatever n is: path 1 the CUDA-core
+ * kernel (tq_decode's choice below 128 x SM-count vectors, and at
+ * head_dim 256), path 2 the tensor-core kernel (head_dim 64 and 128 only:
+ * TQ_ERR_UNSUPPORTED at 256). Same arguments, alignment rules and asynchrony
+ * as tq_decode; n must be > 0; any other path is TQ_ERR_INVALID_ARG.
+ */
+tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
+                              int path, tq_stream stream);
+
+/*
  * One fifth-generation tensor-core MMA (tcgen05.mma kind::f16, M = 128,
  * N = K = 16, f32 accumulator starting from zero), with the shared-memory
  * layout and tensor-memory readback of the tensor-core encode kernel:

@@ -49,6 +49,7 @@ _PROTOS = {
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
     "tq_test_umma_block": (_c_int, [_vp, _vp, _vp, _vp]),
+    "tq_test_decode_path": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _c_int, _vp]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _f = getattr(_lib, _name)
@@ -229,6 +230,11 @@ def tq_device_error(stream=None) -> tuple[int, int]:
 def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> int:
     """Test hook: encode with the row copies withheld; returns the launch status."""
     return _lib.tq_test_encode_stalled(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), _stream(stream))
+
+
+def tq_test_decode_path(ctx: Ctx, packed, norms, n: int, x, path: int, stream=None) -> int:
+    """Test hook: decode through kernel `path` (1 CUDA cores, 2 tensor cores); returns the launch status."""
+    return _lib.tq_test_decode_path(ctx.handle, _ptr(packed), _ptr(norms), int(n), _ptr(x), int(path), _stream(stream))
 
 
 def tq_test_umma_block(a, b, d, stream=None) -> int:

@@ -1,0 +1,511 @@
+// Decode on the fifth-generation tensor cores: (packed codes, f32 norms) ->
+// fp16 vectors, the same outputs as decode_kernel, for bulk launches at
+// head_dim 64 and 128.
+//
+// Method ("aither-kvcache" PyPI page, section "Algorithm": decoding reverses
+// steps 4-1): x_hat = D (H_pm c[idx]) * (N / d), H_pm the +-1 natural-order
+// Walsh-Hadamard matrix, D the seeded sign flip, c the codebook levels.
+//
+// Factorisation used: H_pm = H_{d/16} (x) H_16 (Sylvester's construction):
+// coordinate 16 b' + j of H_pm c is sum_b (-1)^popc(b' & b) S[b][j] with
+// S[b] = H_16 c_b. The tensor cores compute every S[b] of a 128-vector tile.
+// The levels lie on the 2^-14 grid (16 significant bits), so each level is
+// split into an fp16 value and an fp16 remainder (both exact); two MMAs per
+// block accumulate H_16 (value) + H_16 (remainder). Every addend is a
+// multiple of 2^-14 below 2^6 and the tensor core cuts addends only below
+// 2^(E-25) with E <= 6, so the block sums are exact; the f32 butterflies
+// across blocks are exact too (multiples of 2^-14 below 2^10), and the only
+// roundings are the product by N / d and the fp16 conversion, as in
+// decode_kernel.
+//
+// B200 mapping (one persistent CTA of 18 warps per SM, warp-specialised):
+//  * warp 0: 1-D bulk copies of each full tile's packed rows into a ring of
+//    shared-memory stages (a partial last tile is read with plain loads);
+//  * warps 2-9 (two builder warpgroups taking alternate tiles, one row per
+//    thread): each pair of codes indexes a
+//    lane-replicated table of {value pair, remainder pair} as packed fp16,
+//    which go straight into tensor memory with tcgen05.st (A operand: row m
+//    in lane m, two fp16 per 32-bit column, 8 columns per 16-element block);
+//  * warp 1: per tile 2 d/16 MMAs with A from tensor memory ([a-tmem] form)
+//    and B = H_16 (fp16 +-1, shared memory), f32 accumulators in tensor
+//    memory: two A operands (the builders refill one as soon as the MMAs
+//    that read it commit) and one accumulator per epilogue warpgroup;
+//  * warps 10-17 (two epilogue warpgroups, one row per thread): the
+//    log2(d/16) cross-block butterflies in f32x2, the scale N / d, the
+//    fp16 conversion and the sign flip on fp16 pairs, staged in the group's
+//    128-byte-swizzled tile and written by 2-D tensor stores (which clip a
+//    partial last tile).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+
+#include "tq_common.cuh"
+#include "tq_umma.cuh"
+
+namespace tq {
+
+constexpr int DT_ROWS = 128;
+constexpr int DT_WARPS = 18;  // copies, MMAs, 2 builder and 2 epilogue warpgroups
+constexpr int DT_TMEM_COLS = 512;
+constexpr size_t DT_SMEM_MAX = 232448;
+
+template <int D, int BITS>
+struct DtCfg {
+  static constexpr int NB = D / 16;                 // 16-point blocks per vector
+  static constexpr int BOXES = D / 64;              // 64-column store boxes per tile
+  static constexpr int P = D * BITS / 8;            // packed bytes per vector
+  static constexpr int WORDS = P / 4;
+  static constexpr int TILE_P = DT_ROWS * P;        // packed bytes of a full tile
+  static constexpr int E = 1 << (2 * BITS);         // pair-table entries
+  // tensor memory: NA A operands (values d/2 + remainders d/2 columns each),
+  // then one accumulator (d columns) per epilogue warpgroup
+  static constexpr int NA = 2;
+  static constexpr int ACC0 = NA * D;
+  static constexpr int STAGES = 8;
+  static constexpr int JC = 4;                      // positions j per epilogue chunk
+  static constexpr int CHUNKS = 16 / JC;
+  // shared memory, from a 1024-aligned base
+  static constexpr int OUT = 0;                     // 2 groups x BOXES x [128 rows x 128 B]
+  static constexpr int OUT_BYTES = BOXES * DT_ROWS * 128;
+  static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_16, 16 rows x 128 B
+  static constexpr int IN = BREG + 2048;            // STAGES x TILE_P
+  static constexpr int LUT = IN + STAGES * TILE_P;  // E x 32 lane copies x 8 B
+  static constexpr int BAR = LUT + E * 32 * 8;
+  // full[S], empty[S], aready[NA][2], aempty[NA][2], tfull[2], tempty[2], done
+  static constexpr int NBARS = 2 * STAGES + 4 * NA + 4 + 1;
+  static constexpr int SLOT = BAR + NBARS * 8;
+  static constexpr size_t BYTES = 1024 + (size_t)SLOT + 16;
+};
+
+struct DtArgs {
+  CUtensorMap tm_out;  // output as [n rows, d cols] fp16, box 64 x 128, 128-byte swizzle
+  const uint8_t* packed;
+  const float* norms;
+  int64_t n;
+  uint32_t* err;
+  long long wait_limit;
+};
+
+TQ_DEV uint2 dt_lds_u2(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+TQ_DEV void dt_tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+
+TQ_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+TQ_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[bdesc]^T (A in tensor memory), one thread.
+TQ_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(DT_WARPS * 32, 1)
+    decode_tc_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ DtArgs a) {
+  using Cfg = DtCfg<D, BITS>;
+  constexpr int NB = Cfg::NB, S = Cfg::STAGES, NA = Cfg::NA, WORDS = Cfg::WORDS, JC = Cfg::JC;
+  constexpr uint32_t FULL = 0xffffffffu;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sm = smem_raw + (base - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int64_t n_tiles = (a.n + DT_ROWS - 1) / DT_ROWS;
+  const int cnt = (int64_t)blockIdx.x < n_tiles ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  auto tile_of = [&](int i) { return (int64_t)blockIdx.x + (int64_t)i * gridDim.x; };
+  auto full_tile = [&](int i) { return (tile_of(i) + 1) * DT_ROWS <= a.n; };
+
+  const uint32_t bar0 = base + Cfg::BAR;
+  // full[s]: stage s holds tile i's rows; empty[s]: the builders read it;
+  // aready[a][h] / aempty[a][h]: half h (blocks h d/32 ...) of A operand a
+  // written / read by its MMAs;
+  // tfull[g] / tempty[g]: accumulator g written / read by epilogue group g;
+  // done: every MMA is done
+  const uint32_t full0 = bar0, empty0 = bar0 + 8u * S, aready0 = bar0 + 16u * S, aempty0 = aready0 + 16u * NA,
+                 tfull0 = aempty0 + 16u * NA, tempty0 = tfull0 + 16u, done_b = tempty0 + 16u;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 4);
+    }
+    for (int q = 0; q < 2 * NA; ++q) {
+      mbar_init(aready0 + 8u * q, 4);
+      mbar_init(aempty0 + 8u * q, 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(tfull0 + 8u * g, 1);
+      mbar_init(tempty0 + 8u * g, 4);
+    }
+    mbar_init(done_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + Cfg::SLOT, DT_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Cfg::SLOT);
+  // A operand k: values at columns k d + [0, d/2), remainders at + [d/2, d);
+  // accumulator of epilogue group g at columns NA d + g d + [0, d).
+  // The tables are filled after this point, so the first copies are in
+  // flight meanwhile.
+
+  // ---- pair table, built by warps 2-17 (the epilogue warps have nothing to
+  // do before the first accumulator): entry (f, lane), f = code_a | code_b <<
+  // BITS, holds the A-operand columns {value_a | value_b << 16, remainder_a |
+  // remainder_b << 16} (fp16; value + remainder = level exactly: a
+  // 2^-14-grid level below 4 has at most 16 significant bits, its fp16
+  // remainder is a multiple of 2^-14 below 2^-9). Each thread computes one
+  // entry and writes its copies for 32 / (512 / E) lanes, two lanes per
+  // 16-byte store, the stores rotated so a warp's stores spread over banks.
+  if (warp >= 2) {
+    constexpr int E = Cfg::E, PER = 512 / E, LANES = 32 / PER;
+    static_assert(E <= 512 && 512 % E == 0 && PER * LANES == 32, "one thread per entry and lane group");
+    const int t = tid - 64, f = t / PER, part = t % PER;
+    const float ca = T.levels[f & ((1 << BITS) - 1)], cb = T.levels[f >> BITS];
+    const __half va = __float2half_rn(ca), vb = __float2half_rn(cb);
+    const __half ra = __float2half_rn(ca - __half2float(va)), rb = __float2half_rn(cb - __half2float(vb));
+    const uint32_t ev = (uint32_t)__half_as_ushort(va) | ((uint32_t)__half_as_ushort(vb) << 16);
+    const uint32_t er = (uint32_t)__half_as_ushort(ra) | ((uint32_t)__half_as_ushort(rb) << 16);
+    uint8_t* row = sm + Cfg::LUT + f * 256 + part * LANES * 8;
+    if constexpr (LANES == 1) {
+      *reinterpret_cast<uint2*>(row) = make_uint2(ev, er);
+    } else {
+#pragma unroll
+      for (int j = 0; j < LANES / 2; ++j) {
+        const int jj = (j + t) % (LANES / 2);
+        *reinterpret_cast<uint4*>(row + jj * 16) = make_uint4(ev, er, ev, er);
+      }
+    }
+    asm volatile("bar.sync 3, 512;" ::: "memory");  // the table is complete
+  }
+
+  if (warp == 0) {
+    // ---- producer: full tiles by one bulk copy each; the partial last tile
+    // only completes the stage's phase (the builders load it themselves)
+    if (lane == 0) {
+      for (int i = 0; i < cnt; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait_bounded(empty0 + 8u * s, ((i / S) - 1) & 1, a.wait_limit)) {
+          record_error(a.err, TQ_DEVERR_TIMEOUT);
+          break;
+        }
+        if (full_tile(i)) {
+          mbar_arrive_expect_tx(full0 + 8u * s, Cfg::TILE_P);
+          bulk_g2s(base + Cfg::IN + s * Cfg::TILE_P, a.packed + tile_of(i) * Cfg::TILE_P, Cfg::TILE_P, full0 + 8u * s);
+        } else {
+          mbar_arrive(full0 + 8u * s);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer: per block, S = A_value H_16^T + A_remainder H_16^T
+    // ---- B = H_16 (the signs are applied to the fp16 output), K-major swizzled
+    for (int e = lane; e < 256; e += 32) {
+      const int j = e >> 4, k = e & 15;
+      const uint32_t off = Cfg::BREG + j * 128 + ((((k * 2) >> 4) ^ (j & 7)) << 4) + ((k * 2) & 15);
+      *reinterpret_cast<uint16_t*>(sm + off) = (__popc(j & k) & 1) ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
+    }
+    fence_proxy_async_smem();  // B is read by the tensor cores
+    __syncwarp();
+    if (lane == 0) {
+      constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, 16);
+      const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG);
+      bool ok = true;
+      for (int i = 0; i < cnt && ok; ++i) {
+        const int k = i % NA, g = i & 1;
+        const uint32_t ab = tmem + (uint32_t)(k * D), db = tmem + (uint32_t)(Cfg::ACC0 + g * D);
+        // each half of the A operand is multiplied as soon as it is written
+        // and handed back as soon as its MMAs complete
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait_bounded(aready0 + 8u * (2 * k + h), (i / NA) & 1, a.wait_limit) ||
+              (h == 0 && i >= 2 && !mbar_wait_bounded(tempty0 + 8u * g, ((i >> 1) - 1) & 1, a.wait_limit))) {
+            record_error(a.err, TQ_DEVERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int b = h * NB / 2; b < (h + 1) * NB / 2; ++b) {
+            umma_f16_ts(db + (uint32_t)(16 * b), ab + (uint32_t)(8 * b), bdesc, IDESC, false);
+            umma_f16_ts(db + (uint32_t)(16 * b), ab + (uint32_t)(D / 2 + 8 * b), bdesc, IDESC, true);
+          }
+          umma_commit(aempty0 + 8u * (2 * k + h));  // this half may be rewritten
+        }
+        if (ok) umma_commit(tfull0 + 8u * g);  // the accumulator may be read
+      }
+      umma_commit(done_b);
+      if (!mbar_wait_bounded(done_b, 0, a.wait_limit)) record_error(a.err, TQ_DEVERR_TIMEOUT);
+    }
+  } else if (warp < 10) {
+    // ---- builder warpgroup bg (warps 2 + 4 bg ... 5 + 4 bg): tiles bg, bg + 2,
+    // ... into A operand bg; one row per thread (tensor-memory lane = tile row)
+    const int bg = (warp - 2) >> 2, quarter = warp & 3, r = 32 * quarter + lane;
+    const uint32_t lanebase = (uint32_t)(32 * quarter) << 16;
+    const uint32_t lut_lane = base + Cfg::LUT + (uint32_t)lane * 8u;
+    bool alive = true;
+    for (int i = bg; i < cnt && alive; i += 2) {
+      const int s = i % S, k = i % NA;
+      if (!__all_sync(FULL, mbar_wait_bounded(full0 + 8u * s, (i / S) & 1, a.wait_limit))) {
+        if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+        break;
+      }
+      const int64_t row = tile_of(i) * DT_ROWS + r;
+      uint32_t words[WORDS];
+      if (full_tile(i)) {
+        const uint8_t* src = sm + Cfg::IN + s * Cfg::TILE_P + r * Cfg::P;
+        if constexpr (Cfg::P % 16 == 0) {
+#pragma unroll
+          for (int w = 0; w < WORDS; w += 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + 4 * w);
+            words[w] = v.x, words[w + 1] = v.y, words[w + 2] = v.z, words[w + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int w = 0; w < WORDS; w += 2) {
+            const uint2 v = *reinterpret_cast<const uint2*>(src + 4 * w);
+            words[w] = v.x, words[w + 1] = v.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < WORDS; ++w) words[w] = 0u;
+        if (row < a.n) {
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(a.packed + row * Cfg::P);
+#pragma unroll
+          for (int w = 0; w < WORDS; ++w) words[w] = __ldg(src + w);
+        }
+      }
+      const uint32_t sb = tmem + lanebase + (uint32_t)(k * D);
+      // A column p = pair of coordinates (2p, 2p + 1), 16 columns per store;
+      // half h = value (and remainder) columns [h d/4, (h + 1) d/4)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (i >= NA &&
+            !__all_sync(FULL, mbar_wait_bounded(aempty0 + 8u * (2 * k + h), ((i / NA) - 1) & 1, a.wait_limit))) {
+          if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = h * D / 4; c0 < (h + 1) * D / 4; c0 += 16) {
+          uint32_t vv[16], rr[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            constexpr int FB = 2 * BITS;
+            const int off = (c0 + t) * FB;
+            uint32_t f = words[off >> 5] >> (off & 31);
+            if ((off & 31) + FB > 32) f |= words[(off >> 5) + 1] << (32 - (off & 31));
+            f &= (uint32_t)(Cfg::E - 1);
+            const uint2 ent = dt_lds_u2(f * 256u + lut_lane);
+            vv[t] = ent.x;
+            rr[t] = ent.y;
+          }
+          tmem_st16(sb + (uint32_t)c0, vv);
+          tmem_st16(sb + (uint32_t)(D / 2 + c0), rr);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(aready0 + 8u * (2 * k + h));
+      }
+      // The stage is handed back only once every word read from it has been
+      // consumed by a tensor-memory store that has completed: a release right
+      // after the loads let the next tile's copy land before loads that the
+      // compiler had scheduled later (seen at 4 bits, d = 128).
+      if (alive && lane == 0) mbar_arrive(empty0 + 8u * s);
+    }
+  } else {
+    // ---- epilogue warpgroup g (warps 10 + 4g ... 13 + 4g): tiles g, g + 2, ...
+    const int g = (warp - 10) >> 2, quarter = warp & 3, r = 32 * quarter + lane;
+    const bool leader = warp == 10 + 4 * g && lane == 0;
+    const uint32_t lanebase = (uint32_t)(32 * quarter) << 16;
+    const uint32_t stage_out = base + Cfg::OUT + (uint32_t)(g * Cfg::OUT_BYTES);
+    uint8_t* out_sm = sm + Cfg::OUT + g * Cfg::OUT_BYTES;
+    bool stored_once = false;
+    // norms are loaded one tile ahead, so their latency is off the chain
+    auto load_norm = [&](int i) {
+      const int64_t row = tile_of(i) * DT_ROWS + r;
+      return (i < cnt && row < a.n) ? __ldg(a.norms + row) : 0.f;
+    };
+    float nrm_next = load_norm(g);
+    for (int i = g; i < cnt; i += 2) {
+      const float nrm = nrm_next;
+      nrm_next = load_norm(i + 2);
+      const bool ok = mbar_wait_bounded(tfull0 + 8u * g, (i >> 1) & 1, a.wait_limit);
+      if (!__all_sync(FULL, ok)) {
+        if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int64_t tile = tile_of(i);
+      const float sc = nrm * (1.0f / (float)D);
+      const f2 sc2 = make_float2(sc, sc);
+      // the group's staging tile must have been read by its previous store
+      if (leader && stored_once) bulk_wait_read<0>();
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
+      const uint32_t tl = tmem + lanebase + (uint32_t)(Cfg::ACC0 + g * D);
+#pragma unroll
+      for (int c = 0; c < Cfg::CHUNKS; ++c) {
+        const int j0 = c * JC;
+        uint32_t rv[NB][JC];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) tmem_ld4(tl + (uint32_t)(16 * b + j0), rv[b]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int b = 0; b < NB; ++b) tmem_regs_after_wait(rv[b]);
+        if (c == Cfg::CHUNKS - 1) {  // every load of the accumulator is done: free the slot
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8u * g);
+        }
+        f2 v[JC / 2][NB];
+#pragma unroll
+        for (int h = 0; h < JC / 2; ++h) {
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+            v[h][b] = make_float2(__uint_as_float(rv[b][2 * h]), __uint_as_float(rv[b][2 * h + 1]));
+          wht_pairs<NB>(v[h]);
+        }
+#pragma unroll
+        for (int bp = 0; bp < NB; ++bp) {
+          uint32_t hw[JC / 2];
+#pragma unroll
+          for (int h = 0; h < JC / 2; ++h) {
+            const int k = 16 * bp + j0 + 2 * h;  // first coordinate of the pair
+            const f2 y = mul2(v[h][bp], sc2);
+            const __half2 hv = __floats2half2_rn(y.x, y.y);
+            hw[h] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[k >> 1];
+          }
+          // coordinates 16 b' + j0 ... + 3: 8 bytes of the swizzled staging row
+          const int k0 = 16 * bp + j0, box = k0 >> 6, col = k0 & 63;
+          const uint32_t off = (uint32_t)(box * DT_ROWS * 128 + r * 128) +
+                               ((uint32_t)(((col >> 3) ^ (r & 7))) << 4) + (uint32_t)((col & 7) * 2);
+          *reinterpret_cast<uint2*>(out_sm + off) = make_uint2(hw[0], hw[1]);
+        }
+      }
+      fence_proxy_async_smem();
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
+      if (leader) {
+        // rows past the end of a partial tile are clipped by the tensor store
+#pragma unroll
+        for (int bx = 0; bx < Cfg::BOXES; ++bx)
+          dt_tma_store_2d(&a.tm_out, 64 * bx, (int)(tile * DT_ROWS), stage_out + (uint32_t)(bx * DT_ROWS * 128));
+        bulk_commit();
+        stored_once = true;
+      }
+    }
+    if (leader) bulk_wait_all<0>();
+  }
+  // ---- teardown: every role is done (or gave up); free the tensor memory
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, DT_TMEM_COLS);
+  }
+}
+
+template <int D, int BITS>
+static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* x, cudaStream_t st) {
+  using Cfg = DtCfg<D, BITS>;
+  static_assert(Cfg::BYTES <= DT_SMEM_MAX, "shared memory of the tensor-core decode");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> configured{0};  // one bit per device
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(decode_tc_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
+  if (!enc) return cudaErrorNotSupported;
+  const int sms = tq_sm_count(dev);
+  // launches of at most 2^30 rows keep the store coordinates in int32
+  const int64_t max_rows = (int64_t)1 << 30;
+  const int64_t n_total = a.n;
+  const uint8_t* packed0 = a.packed;
+  const float* norms0 = a.norms;
+  for (int64_t off = 0; off < n_total; off += max_rows) {
+    const int64_t n = std::min(max_rows, n_total - off);
+    a.n = n;
+    a.packed = packed0 + off * Cfg::P;
+    a.norms = norms0 + off;
+    __half* xo = static_cast<__half*>(x) + off * D;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)n};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)DT_ROWS};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&a.tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<void*>(xo), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+    const int64_t tiles = (n + DT_ROWS - 1) / DT_ROWS;
+    const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms);
+    decode_tc_kernel<D, BITS><<<grid, DT_WARPS * 32, Cfg::BYTES, st>>>(T, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
+                              void* stream) {
+  if (n == 0) return TQ_OK;
+  if (ctx->d > 128) return TQ_ERR_UNSUPPORTED;  // one tile would fill tensor memory
+  DtArgs a;
+  memset(&a, 0, sizeof(a));
+  a.n = n;
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.norms = norms;
+  a.err = tq_error_word();
+  if (!a.err) return TQ_ERR_CUDA;
+  a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  const tq_codec_tables& T = ctx->t;
+#define TQ_DECTC_CASE(D_, B_) \
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_tc_t<D_, B_>(T, a, x, st);
+  TQ_DECTC_CASE(64, 2) TQ_DECTC_CASE(64, 3) TQ_DECTC_CASE(64, 4)
+  TQ_DECTC_CASE(128, 2) TQ_DECTC_CASE(128, 3) TQ_DECTC_CASE(128, 4)
+#undef TQ_DECTC_CASE
+  if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}

@@ -216,6 +216,11 @@ tq_status tq_decode(const tq_ctx* ctx, const void* packed, const float* norms, i
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
+  if (n >= tq_encode_tc_min_rows()) {
+    // the tensor-core kernel at head_dim <= 128
+    const tq_status st = tq_launch_decode_tc(ctx, packed, norms, n, x_f16, stream);
+    if (st != TQ_ERR_UNSUPPORTED) return st;
+  }
   return tq_launch_decode(ctx, packed, norms, n, x_f16, stream);
 }
 
@@ -317,6 +322,18 @@ tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n
   if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 1);
+}
+
+// Test hook (declared in include/tq_test.h): tq_decode through a chosen kernel.
+tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
+                              int path, tq_stream stream) {
+  if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
+  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
+  switch (path) {
+    case 1: return tq_launch_decode(ctx, packed, norms, n, x_f16, stream);
+    case 2: return tq_launch_decode_tc(ctx, packed, norms, n, x_f16, stream);
+    default: return TQ_ERR_INVALID_ARG;
+  }
 }
 
 // Test hook (declared in include/tq_test.h): tq_encode through a chosen kernel.

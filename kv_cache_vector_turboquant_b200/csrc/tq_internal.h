@@ -71,6 +71,11 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
 tq_status tq_launch_encode_tc(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms, void* stream,
                               int fault_inject);
 int64_t tq_encode_tc_min_rows(void);
+// Bulk decode on the tensor cores (tq_decode_tc.cu), head_dim <= 128: the same
+// outputs as tq_launch_decode. TQ_ERR_UNSUPPORTED otherwise (then the CUDA-core
+// kernel is used). tq_decode uses it from tq_encode_tc_min_rows() vectors on.
+tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
+                              void* stream);
 tq_status tq_launch_encode_os(const tq_ctx* ctx, const void* x, int64_t n, void* packed, uint32_t* side,
                               void* stream);
 tq_status tq_launch_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,

@@ -138,6 +138,18 @@ def test_encode_path_hook_validation(K):
     assert _raw(K, "tq_test_encode_path", h, A, 4, B_ + 4, C, 2, None) == K.TQ_ERR_ALIGNMENT
 
 
+def test_decode_path_hook_validation(K):
+    ctx = K.tq_create(128, 4)
+    h = ctx.handle
+    A, B_, C = 0x10000, 0x20000, 0x30000
+    for bad_path in (0, 3, -1):
+        assert _raw(K, "tq_test_decode_path", h, A, C, 4, B_, bad_path, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_decode_path", None, A, C, 4, B_, 2, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_decode_path", h, A, C, 0, B_, 2, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, "tq_test_decode_path", h, A + 8, C, 4, B_, 2, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, "tq_test_decode_path", h, A, C + 2, 4, B_, 2, None) == K.TQ_ERR_ALIGNMENT
+
+
 def test_umma_block_hook_validation(K):
     A, B_, C = 0x10000, 0x20000, 0x30000
     assert _raw(K, "tq_test_umma_block", None, B_, C, None) == K.TQ_ERR_INVALID_ARG

@@ -1,0 +1,97 @@
+"""The tensor-core decode kernel (needs a B200).
+
+tq_decode runs it for head_dim 64 and 128 from 128 x SM-count vectors on; the
+test hook tq_test_decode_path runs it (path 2) or the CUDA-core kernel
+(path 1) at any size. Both compute H_pm c exactly and round only the product
+by N / d and the fp16 conversion, so their outputs are bit-identical; the
+oracle bounds both to 1 fp16 ulp.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity import assert_decode_ulp
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K(cuda_device):
+    import kv_cache_vector_turboquant_b200 as K
+
+    return K
+
+
+@pytest.fixture(scope="module")
+def W():
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    return W
+
+
+def _dec_path(K, tq, packed, norms, path):
+    n = norms.numel()
+    x = torch.full((n, tq.head_dim), 7.0, dtype=torch.float16, device="cuda")
+    assert K._binding.tq_test_decode_path(tq.ctx, packed, norms, n, x, path) == K.TQ_OK
+    torch.cuda.synchronize()
+    return x
+
+
+def _random_codes(tq, n, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    packed = torch.randint(0, 256, (n, tq.packed_bytes), generator=g, device="cuda", dtype=torch.int32).to(torch.uint8)
+    norms = torch.rand(n, generator=g, device="cuda") * 30.0
+    if n > 3:
+        norms[0] = 0.0
+        norms[1] = 1.0e-30
+        norms[2] = 6.0e4
+    return packed, norms
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("n", [1, 127, 128, 129, 4103])
+def test_tc_decode_ragged_sizes(K, d, bits, n):
+    """Random bytes and norms (zero, tiny and large among them): partial
+    tiles (read with plain loads, stores clipped), one tile, 33 tiles."""
+    tq = K.TurboQuant(d, bits, seed=5 + bits)
+    packed, norms = _random_codes(tq, n, 100 * d + 10 * bits + n)
+    x2 = _dec_path(K, tq, packed, norms, 2)
+    x1 = _dec_path(K, tq, packed, norms, 1)
+    assert torch.equal(x1, x2)
+    ref = O.decode(packed.cpu().numpy(), norms.cpu().numpy(), bits, 5 + bits, d)
+    assert_decode_ulp(x2.cpu().numpy(), ref)
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+@pytest.mark.parametrize("d,per_cta", [(64, 13), (128, 9)])
+def test_tc_decode_many_tiles_per_cta(K, W, d, per_cta):
+    """Every CTA cycles its stage ring, both tensor-memory slots and both
+    epilogue warpgroups several times; the layer's own codes."""
+    n = 148 * 128 * per_cta + 77
+    x = W.single_tensor(n=n, d=d, seed=77 + d, outlier_frac=0.02).cuda()
+    for bits in (2, 3, 4):
+        tq = K.TurboQuant(d, bits)
+        packed, norms = tq.encode(x)
+        x2 = _dec_path(K, tq, packed, norms, 2)
+        x1 = _dec_path(K, tq, packed, norms, 1)
+        assert torch.equal(x1, x2), bits
+        rows = torch.randperm(n, generator=torch.Generator().manual_seed(bits))[:2048].sort().values.cuda()
+        ref = O.decode(packed[rows].cpu().numpy(), norms[rows].cpu().numpy(), bits, 42, d)
+        assert_decode_ulp(x2[rows].cpu().numpy(), ref)
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+def test_tc_decode_bulk_call_uses_it_and_head_dim_256_does_not(K, W):
+    n = 148 * 128 * 2 + 3
+    tq = K.TurboQuant(128, 4)
+    packed, norms = _random_codes(tq, n, 11)
+    xb = tq.decode(packed, norms)
+    torch.cuda.synchronize()
+    assert torch.equal(xb, _dec_path(K, tq, packed, norms, 2))
+    t256 = K.TurboQuant(256, 4)
+    p256, n256 = _random_codes(t256, 300, 12)
+    x = torch.empty(300, 256, dtype=torch.float16, device="cuda")
+    assert K._binding.tq_test_decode_path(t256.ctx, p256, n256, 300, x, 2) == K.TQ_ERR_UNSUPPORTED
