@@ -494,7 +494,7 @@ def run_ours(args, rank, world, local_rank):
         v["share"] = v["share"] / tot
     dom_name = max(kernels, key=lambda n: kernels[n]["share"])
     dom = kernels[dom_name]
-    src = "tq_encode_tc.cu" if dom_name.startswith("encode") else "tq_decode.cu"
+    src = "tq_encode_tc.cu" if dom_name.startswith("encode") else "tq_decode_tc.cu"
     traffic = _profile_traffic(src, f"{dom_name.split('_')[0]}_llama_layer_{dom_name.split('_')[1]}.txt")
     roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom["GBps"], "peak": peak, "unit": "GB/s",
             "frac": dom["frac"], "traffic": traffic, "peak_kind": f"{peak_kind} copy (MEASURED_PEAKS.json hbm_gbs)",
