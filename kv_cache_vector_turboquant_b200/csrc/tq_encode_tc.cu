@@ -203,36 +203,6 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
   const int64_t n_tiles = (a.n + TC_ROWS - 1) / TC_ROWS;
   const int cnt = (int64_t)blockIdx.x < n_tiles ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
 
-  // ---- B operands: block b holds H_16[j][k] * s_{16 b + k} as fp16 +-1 in
-  // the K-major 128-byte-swizzled layout, four blocks side by side in one
-  // 16-row region (block b: region b / 4, bytes 32 (b % 4) ... + 31 of row j)
-  for (int e = tid; e < NB * 256; e += blockDim.x) {
-    const int b = e >> 8, j = (e >> 4) & 15, k = e & 15, i = 16 * b + k;
-    const uint32_t neg = ((T.sign_h2[i >> 1] >> (15 + 16 * (i & 1))) & 1u) ^ (uint32_t)(__popc(j & k) & 1);
-    const int kb = 32 * (b & 3) + 2 * k;  // byte of the element within the row
-    const uint32_t off = Cfg::BREG + (b >> 2) * 2048 + j * 128 + (((kb >> 4) ^ (j & 7)) << 4) + (kb & 15);
-    *reinterpret_cast<uint16_t*>(sm + off) = neg ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
-  }
-  uint32_t* sgn = reinterpret_cast<uint32_t*>(sm + Cfg::SIGN);
-  if (tid < D / 32) {
-    uint32_t w = 0;
-    for (int l = 0; l < 32; ++l) {
-      const int i = 32 * tid + l;
-      w |= ((T.sign_h2[i >> 1] >> (15 + 16 * (i & 1))) & 1u) << l;
-    }
-    sgn[tid] = w;
-  }
-  float* sbound = reinterpret_cast<float*>(sm + Cfg::BND);
-  if (tid < L - 1) sbound[tid] = T.bounds[tid];
-  {
-    // cell table: entry (cell, copy) = {boundary bits, count below}
-    uint2* lut = reinterpret_cast<uint2*>(sm + Cfg::LUT);
-    const int entries = T.lut_cells * TC_LUT_COPIES;
-    for (int e = tid; e < entries; e += blockDim.x) {
-      const int cell = e / TC_LUT_COPIES;
-      lut[e] = make_uint2(T.cell[cell][0], T.cell[cell][1]);
-    }
-  }
   const uint32_t bar0 = base + Cfg::BAR;
   const uint32_t done_bar = bar0 + 8u * (2 * S + 2 * NACC);
   if (tid == 0) {
@@ -247,7 +217,6 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
     mbar_init(done_bar, 1);
     fence_mbar_init();
   }
-  fence_proxy_async_smem();  // the B operands are read by the tensor cores
   if (warp == 1) {
     tmem_alloc(base + Cfg::SLOT, TC_TMEM_COLS);
     tmem_relinquish();
@@ -256,6 +225,41 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + Cfg::SLOT);
+  uint32_t* sgn = reinterpret_cast<uint32_t*>(sm + Cfg::SIGN);
+  float* sbound = reinterpret_cast<float*>(sm + Cfg::BND);
+
+  // ---- tables, built by warps 1 ... while warp 0 already streams the first
+  // tiles in:
+  //  * B operands: block b holds H_16[j][k] * s_{16 b + k} as fp16 +-1 in the
+  //    K-major 128-byte-swizzled layout, four blocks side by side in one
+  //    16-row region (block b: region b / 4, bytes 32 (b % 4) ... + 31 of row j);
+  //  * the D sign bits (word t, bit l: coordinate 32 t + l), one ballot each;
+  //  * the boundaries in z units (fp64 recheck);
+  //  * the cell table: entry (cell, copy) = {boundary bits, count below}.
+  if (warp >= 1) {
+    const int t = tid - 32, nt = (int)blockDim.x - 32;
+    for (int e = t; e < NB * 256; e += nt) {
+      const int b = e >> 8, j = (e >> 4) & 15, k = e & 15, i = 16 * b + k;
+      const uint32_t neg = ((T.sign_h2[i >> 1] >> (15 + 16 * (i & 1))) & 1u) ^ (uint32_t)(__popc(j & k) & 1);
+      const int kb = 32 * (b & 3) + 2 * k;  // byte of the element within the row
+      const uint32_t off = Cfg::BREG + (b >> 2) * 2048 + j * 128 + (((kb >> 4) ^ (j & 7)) << 4) + (kb & 15);
+      *reinterpret_cast<uint16_t*>(sm + off) = neg ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
+    }
+    fence_proxy_async_smem();  // the B operands are read by the tensor cores
+    for (int w = warp - 1; w < D / 32; w += Cfg::WARPS - 1) {
+      const int i = 32 * w + lane;
+      const uint32_t word = __ballot_sync(FULL, (T.sign_h2[i >> 1] >> (15 + 16 * (i & 1))) & 1u);
+      if (lane == 0) sgn[w] = word;
+    }
+    if (t < L - 1) sbound[t] = T.bounds[t];
+    uint2* lut = reinterpret_cast<uint2*>(sm + Cfg::LUT);
+    const int entries = T.lut_cells * TC_LUT_COPIES;
+    for (int e = t; e < entries; e += nt) {
+      const int cell = e / TC_LUT_COPIES;
+      lut[e] = make_uint2(T.cell[cell][0], T.cell[cell][1]);
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");  // the tables are complete
+  }
 
   if (warp == 0) {
     // ---- producer: tile i of this CTA into stage i % S as soon as the MMAs
