@@ -136,6 +136,19 @@ def _ev(torch):
     return torch.cuda.Event(enable_timing=True)
 
 
+def _bracketed_ms(torch, call, steps):
+    """Mean ms per call over `steps` back-to-back calls between two events
+    (no event between the calls, which would serialise them)."""
+    t0, t1 = _ev(torch), _ev(torch)
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(steps):
+        call()
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
 def reduce_max_ms(ms: float, world: int, dist=None, device=None) -> float:
     """Max over ranks of a per-rank time (the slowest rank sets the job time)."""
     if world <= 1:
@@ -200,8 +213,8 @@ def _bench_attention(K, W, torch, steps, warmup):
         call()
         e1.record()
     torch.cuda.synchronize()
-    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    t = statistics.mean(ms) / 1e3
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]  # per step, with events around each
+    t = _bracketed_ms(torch, call, steps) / 1e3    # back-to-back steps
     pk, pv = a["d"] * a["kb"] // 8, a["d"] * a["vb"] // 8
     alg = a["B"] * a["S"] * a["Hkv"] * (pk + pv + 8) + 2 * 2 * a["B"] * a["Hq"] * a["d"]
     peak, kind = _peaks()
@@ -251,7 +264,7 @@ def _bench_attention_paged(K, torch, a, q, kc, vc, kp, kn, vp, vn, pos, steps, w
         call()
         e1.record()
     torch.cuda.synchronize()
-    t = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs) / 1e3
+    t = _bracketed_ms(torch, call, steps) / 1e3
     peak, kind = _peaks()
     st = K.tq_device_error()
     del kpool, knpool, vpool, vnpool
@@ -470,15 +483,23 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         t0.record()
         for s in range(args.steps):
-            step(evs[s])
+            step()
         t1.record()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    ms = reduce_max_ms(t0.elapsed_time(t1), world, dist, "cuda")
+        ms = reduce_max_ms(t0.elapsed_time(t1), world, dist, "cuda")
+        # per-launch durations from a second loop of the same `steps` steps with
+        # an event pair around every launch: events between launches serialise
+        # them (about 2.7 us per launch measured), so the headline loop above
+        # has only its two bracketing events
+        torch.cuda.synchronize()
+        for s in range(args.steps):
+            step(evs[s])
+        torch.cuda.synchronize()
     ms_step = ms / args.steps
 
-    # per-kernel averages inside the timed region
+    # per-kernel averages (second loop)
     per = {}
     for s in range(args.steps):
         for i, L in enumerate(launches):
@@ -521,6 +542,8 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "clocks": clk.summary(),
         "gpu_launches": len(launches) * args.steps,
+        "kernel_timing": "per-launch CUDA events in a second loop of the same steps right after the timed one "
+                         "(events between launches add ~2.7 us each, so the timed loop has none)",
         "device_error_after_warmup": list(err),
     }
     # end to end through the public API with pinned host buffers
