@@ -104,6 +104,13 @@ struct TcArgs {
   long long wait_limit;  // bound on each mbarrier wait, SM cycles
 };
 
+// 32-byte store (sm_100): one instruction writes 8 words of a thread's row
+TQ_DEV void tc_stg_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 TQ_DEV uint2 tc_lds_u2(uint32_t addr) {
   uint2 r;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
@@ -490,13 +497,26 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
       // ---- this thread's packed row and norm
       if (active) {
         uint8_t* dst = a.packed + row * Cfg::P;
-        if constexpr (Cfg::P % 16 == 0) {
+        // rows of a multiple of 32 bytes from a 32-byte aligned base: 32-byte
+        // stores (a warp's store then touches half as many cache lines)
+        bool stored = false;
+        if constexpr (Cfg::P % 32 == 0) {
+          if ((reinterpret_cast<uintptr_t>(a.packed) & 31u) == 0) {
 #pragma unroll
-          for (int w = 0; w < WORDS; w += 4)
-            *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
-        } else {
+            for (int w = 0; w < WORDS; w += 8) tc_stg_v8(dst + 4 * w, words + w);
+            stored = true;
+          }
+        }
+        if (!stored) {
+          if constexpr (Cfg::P % 16 == 0) {
 #pragma unroll
-          for (int w = 0; w < WORDS; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
+            for (int w = 0; w < WORDS; w += 4)
+              *reinterpret_cast<uint4*>(dst + 4 * w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+          } else {
+#pragma unroll
+            for (int w = 0; w < WORDS; w += 2)
+              *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
+          }
         }
         a.norms[row] = nrm;
       }

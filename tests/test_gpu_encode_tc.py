@@ -136,6 +136,28 @@ def test_tc_block_spikes_with_fine_residue(K, d):
         _parity(K, x16, d, bits, max_boundary_frac=None)
 
 
+@pytest.mark.parametrize("d,bits", [(64, 4), (128, 2), (128, 3), (128, 4), (256, 4)])
+def test_tc_output_rows_at_16_but_not_32_byte_alignment(K, W, d, bits):
+    """Rows whose size is a multiple of 32 bytes are written with 32-byte
+    stores only from a 32-byte aligned base; a base that is 16-byte aligned
+    (all the API asks) but not 32 takes the 16-byte stores, same bytes."""
+    n = 148 * 128 + 9
+    x = W.single_tensor(n=n, d=d, seed=31 + d + bits).cuda()
+    tq = K.TurboQuant(d, bits)
+    ref, ref_n = _enc_path(K, tq, x, 2)
+    P = tq.packed_bytes
+    buf = torch.zeros(n * P + 64, dtype=torch.uint8, device="cuda")
+    off = 16 if buf.data_ptr() % 32 == 0 else 0
+    assert (buf.data_ptr() + off) % 32 == 16
+    packed = buf[off:off + n * P].view(n, P)
+    norms = torch.zeros(n, dtype=torch.float32, device="cuda")
+    assert K._binding.tq_test_encode_path(tq.ctx, x, n, packed, norms, 2) == K.TQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(packed, ref) and torch.equal(norms, ref_n)
+    assert int(buf[:off].sum()) == 0 and int(buf[off + n * P:].sum()) == 0  # nothing outside the rows
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
 def test_tc_bulk_encode_uses_the_tensor_core_kernel(K, W):
     """tq_encode of a bulk launch gives exactly the tensor-core kernel's
     output (codes and norms), and the CUDA-core kernel's codes."""
