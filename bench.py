@@ -42,6 +42,10 @@ APPEND = dict(n_seq=256, H=8, d=128, bits=4, s_max=1024)
 L2_BYTES = 126 * 1024 * 1024
 
 
+HBM_NOMINAL_GBS = 8000.0  # B200 nominal HBM3e bandwidth, printed beside the measured copy peak
+FP32_LANES_PER_SM = 128   # FP32 FMA lanes per SM (4 sub-partitions x 32)
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -189,7 +193,7 @@ def _codec_step_setup(K, W, torch, rank):
     return dict(n=n, xs=xs, codecs=codecs, packed=packed, norms=norms, out=out, launches=launches)
 
 
-def _bench_attention(K, W, torch, steps, warmup):
+def _bench_attention(K, W, torch, steps, warmup, sm_mhz=1965.0):
     a = ATTN
     q, k, v = W.decode_step(a["B"], a["Hq"], a["Hkv"], a["S"], a["d"])
     kc, vc = K.TurboQuant(a["d"], a["kb"]), K.TurboQuant(a["d"], a["vb"])
@@ -219,6 +223,9 @@ def _bench_attention(K, W, torch, steps, warmup):
     alg = a["B"] * a["S"] * a["Hkv"] * (pk + pv + 8) + 2 * 2 * a["B"] * a["Hq"] * a["d"]
     peak, kind = _peaks()
     ach = alg / t / 1e9
+    g = a["Hq"] // a["Hkv"]
+    flops = 4 * g * a["d"] * a["B"] * a["S"] * a["Hkv"]
+    fp32_peak = torch.cuda.get_device_properties(0).multi_processor_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6
     st = K.tq_device_error()
     paged = _bench_attention_paged(K, torch, a, q, kc, vc, kp, kn, vp, vn, pos, steps, warmup, alg)
     return {"workload": "decode_step: q [16,32,128] fp16, K 4-bit / V 2-bit packed caches [16,32768,8,*]",
@@ -226,8 +233,14 @@ def _bench_attention(K, W, torch, steps, warmup):
             "cache_positions_heads_per_s": a["B"] * a["S"] * a["Hkv"] / t,
             "launches_per_step": 2,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                         "frac_of_nominal": ach / HBM_NOMINAL_GBS,
                          "traffic": _profile_traffic("tq_attend_fast.cu", "attend_fast_decode_step.txt"),
                          "peak_kind": kind, "algorithmic_bytes": alg},
+            # 2 g d multiply-adds per (position, kv head), g = Hq / Hkv: on the
+            # FP32 pipes (SMs x 128 lanes x 2 flop per cycle) this step could
+            # not beat `fp32_bound_us`; the kernel runs both contractions on
+            # the tensor cores instead
+            "flops": flops, "fp32_bound_us": flops / fp32_peak * 1e6, "fp32_peak_tflops": fp32_peak / 1e12,
             "device_error": list(st), "paged": paged}
 
 
@@ -508,8 +521,11 @@ def run_ours(args, rank, world, local_rank):
     kernels = {}
     for (kind, b), vals in per.items():
         avg = statistics.mean(v[0] for v in vals) / 1e3
-        kernels[f"{kind}_b{b}"] = {"us": avg * 1e6, "GBps": vals[0][1] / avg / 1e9,
-                                   "frac": vals[0][1] / avg / 1e9 / peak, "share": sum(v[0] for v in vals)}
+        kernels[f"{kind}_b{b}"] = {"us": avg * 1e6, "us_median": statistics.median(v[0] for v in vals) * 1e3,
+                                   "us_best": min(v[0] for v in vals) * 1e3, "GBps": vals[0][1] / avg / 1e9,
+                                   "frac": vals[0][1] / avg / 1e9 / peak,
+                                   "frac_of_nominal": vals[0][1] / avg / 1e9 / HBM_NOMINAL_GBS,
+                                   "share": sum(v[0] for v in vals)}
     tot = sum(v["share"] for v in kernels.values())
     for v in kernels.values():
         v["share"] = v["share"] / tot
@@ -532,6 +548,7 @@ def run_ours(args, rank, world, local_rank):
             "frac": alg_dom / dom_s / 1e9 / peak, "traffic": traffic,
             "peak_kind": f"{peak_kind} copy (MEASURED_PEAKS.json hbm_gbs)",
             "algorithmic_bytes_per_launch": alg_dom, "launch_us": dom_s * 1e6,
+            "frac_of_nominal": alg_dom / dom_s / 1e9 / HBM_NOMINAL_GBS, "nominal_gbs": HBM_NOMINAL_GBS,
             "launch_us_with_events": dom["us"],
             "timing": "the kernel's K and V launches of the step back to back between two CUDA events"}
 
@@ -563,7 +580,8 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with pinned host buffers
     result["e2e"] = _e2e(K, torch, S, max(2, min(args.steps, 3)), world, dist)
     if not args.skip_extras:
-        result["attn"] = _bench_attention(K, W, torch, max(args.steps, 5), max(args.warmup, 3))
+        result["attn"] = _bench_attention(K, W, torch, max(args.steps, 5), max(args.warmup, 3),
+                                          float(result["clocks"].get("sm_mhz") or 1965.0))
         result["append"] = _bench_append(K, W, torch)
         result["long_context"] = _bench_long_context(K, W, torch)
         result["offset_variant"] = _bench_offset_variant(K, W, torch)
