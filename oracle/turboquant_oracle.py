@@ -23,7 +23,7 @@ Sources (page title, then section):
   fused decode path": rotating only the query and folding the rotation onto the
   output equals the straightforward computation up to rounding.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * rotation = random +-1 sign flip D, then the orthonormal Walsh-Hadamard matrix
   H in natural (Sylvester) order, H[i, j] = (-1)^popcount(i & j) / sqrt(d);
