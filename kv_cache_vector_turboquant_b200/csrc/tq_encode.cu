@@ -158,15 +158,21 @@ TQ_DEV void put_code(uint32_t (&words)[WL], int i, uint32_t m) {
   if ((off & 31) + BITS > 32) words[(off >> 5) + 1] += m >> (32 - (off & 31));
 }
 
-// Replace code i (runtime index) by m in the lane's word array.
+// Replace code i (runtime index) by m in the lane's word array. Every word
+// goes through the same masked update, so the array is never indexed at run
+// time (which would move it to local memory).
 template <int BITS, int WL>
 TQ_DEV void set_code(uint32_t (&words)[WL], int i, uint32_t m) {
   const int off = i * BITS, w0 = off >> 5, sh = off & 31;
   const uint32_t msk = (1u << BITS) - 1u;
+  const bool straddles = sh + BITS > 32;
+  const uint32_t lo_mask = msk << sh, lo_val = m << sh;
+  const uint32_t hi_mask = straddles ? msk >> (32 - sh) : 0u, hi_val = straddles ? m >> (32 - sh) : 0u;
 #pragma unroll
   for (int w = 0; w < WL; ++w) {
-    if (w == w0) words[w] = (words[w] & ~(msk << sh)) | (m << sh);
-    if (w == w0 + 1 && sh + BITS > 32) words[w] = (words[w] & ~(msk >> (32 - sh))) | (m >> (32 - sh));
+    const uint32_t mk = (w == w0 ? lo_mask : 0u) | (w == w0 + 1 ? hi_mask : 0u);
+    const uint32_t v = (w == w0 ? lo_val : 0u) | (w == w0 + 1 ? hi_val : 0u);
+    words[w] = (words[w] & ~mk) | v;
   }
 }
 

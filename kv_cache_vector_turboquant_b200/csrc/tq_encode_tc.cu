@@ -446,9 +446,12 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
                 const int e = __ffs(cc) - 1;
                 const uint32_t sh = (uint32_t)(BITS * (u * JC + e % JC)),
                                m = reinterpret_cast<const uint32_t*>(scratch)[e];
+                const int eb = e / JC;
 #pragma unroll
-                for (int bp = 0; bp < NB; ++bp)
-                  if (bp == e / JC) fld[bp] = (fld[bp] & ~(((1u << BITS) - 1u) << sh)) | (m << sh);
+                for (int bp = 0; bp < NB; ++bp) {
+                  const uint32_t mk = bp == eb ? ((1u << BITS) - 1u) << sh : 0u;
+                  fld[bp] = (fld[bp] & ~mk) | ((m << sh) & mk);
+                }
               }
             }
             __syncwarp();
