@@ -3,6 +3,10 @@
 // error word. Hand-written PTX, no library kernels.
 #pragma once
 
+#include <cuda_runtime.h>
+
+#include <utility>
+
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -55,6 +59,18 @@ TQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for phase `parity` of the barrier to complete, for at most `limit`
 // SM clock cycles. Returns false if the bound ran out.
+// Programmatic dependent launch (sm_90 and later). A kernel launched with
+// programmatic stream serialisation (tq_launch_pdl) may start while the
+// previous kernel of the stream is still finishing: grid_dep_wait() blocks the
+// calling thread until that kernel has completed and its memory operations
+// are visible, so every thread that touches global memory calls it first;
+// grid_dep_launch() lets the next such kernel start once every CTA of this
+// grid has issued it or exited. Kernels that use them are launched with at
+// most one CTA per SM (one wave), so a dependent CTA waiting for this grid
+// never holds an SM this grid still needs.
+TQ_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+TQ_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 TQ_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -136,6 +152,23 @@ TQ_DEV uint32_t lane_id() {
   uint32_t l;
   asm("mov.u32 %0, %%laneid;" : "=r"(l));
   return l;
+}
+
+// Launch with programmatic stream serialisation (see grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t tq_launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace tq

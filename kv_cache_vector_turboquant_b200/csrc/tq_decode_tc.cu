@@ -135,6 +135,9 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sm = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the next kernel of the stream may start its own set-up as this grid's
+  // CTAs exit (it waits for this grid before touching global memory)
+  if (tid == 0) grid_dep_launch();
 
   const int64_t n_tiles = (a.n + DT_ROWS - 1) / DT_ROWS;
   const int cnt = (int64_t)blockIdx.x < n_tiles ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
@@ -212,6 +215,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     // ---- producer: full tiles by one bulk copy each; the partial last tile
     // only completes the stage's phase (the builders load it themselves)
     if (lane == 0) {
+      grid_dep_wait();  // the previous kernel of the stream may still write the codes
       for (int i = 0; i < cnt; ++i) {
         const int s = i % S;
         if (i >= S && !mbar_wait_bounded(empty0 + 8u * s, ((i / S) - 1) & 1, a.wait_limit)) {
@@ -237,6 +241,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     fence_proxy_async_smem();  // B is read by the tensor cores
     __syncwarp();
     if (lane == 0) {
+      grid_dep_wait();  // (its only global access is the error word)
       constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, 16);
       const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG);
       bool ok = true;
@@ -272,6 +277,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     const int bg = (warp - 2) >> 2, quarter = warp & 3, r = 32 * quarter + lane;
     const uint32_t lanebase = (uint32_t)(32 * quarter) << 16;
     const uint32_t lut_lane = base + Cfg::LUT + (uint32_t)lane * 8u;
+    grid_dep_wait();  // a partial tile's rows are read from global memory
     bool alive = true;
     for (int i = bg; i < cnt && alive; i += 2) {
       const int s = i % S, k = i % NA;
@@ -358,6 +364,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       const int64_t row = tile_of(i) * DT_ROWS + r;
       return (i < cnt && row < a.n) ? __ldg(a.norms + row) : 0.f;
     };
+    grid_dep_wait();  // before the first norm load and the first store
     float nrm_next = load_norm(g);
     for (int i = g; i < cnt; i += 2) {
       const float nrm = nrm_next;
@@ -475,8 +482,7 @@ static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* 
       return cudaErrorNotSupported;
     const int64_t tiles = (n + DT_ROWS - 1) / DT_ROWS;
     const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms);
-    decode_tc_kernel<D, BITS><<<grid, DT_WARPS * 32, Cfg::BYTES, st>>>(T, a);
-    e = cudaGetLastError();
+    e = tq_launch_pdl(decode_tc_kernel<D, BITS>, dim3(grid), dim3(DT_WARPS * 32), Cfg::BYTES, st, T, a);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -206,6 +206,9 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sm = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the next kernel of the stream may start its own set-up as this grid's
+  // CTAs exit (it waits for this grid before touching global memory)
+  if (tid == 0) grid_dep_launch();
 
   const int64_t n_tiles = (a.n + TC_ROWS - 1) / TC_ROWS;
   const int cnt = (int64_t)blockIdx.x < n_tiles ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
@@ -272,6 +275,7 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
     // ---- producer: tile i of this CTA into stage i % S as soon as the MMAs
     // of tile i - S have released it
     if (lane == 0 && !a.fault_inject) {
+      grid_dep_wait();  // the previous kernel of the stream may still write x
       for (int i = 0; i < cnt; ++i) {
         const int s = i % S;
         if (i >= S && !mbar_wait_bounded(bar0 + 8u * (S + s), ((i / S) - 1) & 1, a.wait_limit)) {
@@ -288,6 +292,7 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
   } else if (warp == 1) {
     // ---- MMA issuer: S[b] = A_b * B_b^T for the d/16 blocks of tile i
     if (lane == 0) {
+      grid_dep_wait();  // (its only global access is the error word)
       constexpr uint32_t IDESC = umma_idesc_f16(TC_ROWS, 16);
       for (int i = 0; i < cnt; ++i) {
         const int s = i % S, q = i % NACC;
@@ -320,6 +325,7 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
     const uint32_t lut_lane = base + Cfg::LUT + (uint32_t)(lane & (TC_LUT_COPIES - 1)) * 8u - 0x80000000u;
     const float Rscale = T.inv_delta, qoff = T.q_offset, gq = T.guard_q;
     const f2 Q2 = make_float2(qoff, qoff), M2 = make_float2(TC_MAGIC_2P23, TC_MAGIC_2P23);
+    grid_dep_wait();  // before the first store and the first recheck load
     for (int i = g; i < cnt; i += Cfg::GROUPS) {
       const int q = i % NACC;
       // warp-uniform decision: the tensor-memory loads below are warp-collective
@@ -575,8 +581,7 @@ static cudaError_t launch_encode_tc_t(const tq_codec_tables& T, TcArgs a, const 
       return cudaErrorNotSupported;
     const int64_t tiles = (n + TC_ROWS - 1) / TC_ROWS;
     const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms);
-    encode_tc_kernel<D, BITS><<<grid, Cfg::WARPS * 32, smem, st>>>(T, a);
-    e = cudaGetLastError();
+    e = tq_launch_pdl(encode_tc_kernel<D, BITS>, dim3(grid), dim3(Cfg::WARPS * 32), smem, st, T, a);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
