@@ -367,3 +367,36 @@ def test_bounded_wait_times_out_and_context_survives(K, W):
     assert K.tq_device_error() == (K.TQ_OK, 0)
     det = O.encode_detail(x.cpu().numpy(), 4, 42)
     assert code_mismatches(p2.cpu().numpy(), det, 4, 128) == 0
+
+
+@pytest.mark.parametrize("d,bits", [(64, 3), (128, 2), (128, 4)])
+def test_back_to_back_bulk_launches_see_each_others_outputs(K, W, d, bits):
+    """The bulk kernels start while the previous kernel of the stream is
+    finishing (programmatic dependent launch) and wait for it before
+    touching global memory. A chain in which every launch consumes the
+    previous one's output, issued with no synchronisation, gives the same
+    bytes as the chain synchronised after every call."""
+    n = 148 * 128 * 3 + 41
+    x = W.single_tensor(n=n, d=d, seed=300 + d + bits).cuda()
+    tq = K.TurboQuant(d, bits)
+
+    def chain(sync):
+        p1, n1 = tq.encode(x)
+        if sync:
+            torch.cuda.synchronize()
+        y1 = tq.decode(p1, n1)  # reads the encode's codes and norms
+        if sync:
+            torch.cuda.synchronize()
+        p2, n2 = tq.encode(y1)  # reads the decode's rows
+        if sync:
+            torch.cuda.synchronize()
+        y2 = tq.decode(p2, n2)
+        torch.cuda.synchronize()
+        return p1, n1, y1, p2, n2, y2
+
+    ref = chain(True)
+    for _ in range(3):
+        got = chain(False)
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+    assert K.tq_device_error() == (K.TQ_OK, 0)
