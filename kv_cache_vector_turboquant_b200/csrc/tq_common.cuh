@@ -65,9 +65,10 @@ TQ_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // calling thread until that kernel has completed and its memory operations
 // are visible, so every thread that touches global memory calls it first;
 // grid_dep_launch() lets the next such kernel start once every CTA of this
-// grid has issued it or exited. Kernels that use them are launched with at
-// most one CTA per SM (one wave), so a dependent CTA waiting for this grid
-// never holds an SM this grid still needs.
+// grid has issued it or exited. A CTA that has not started has issued
+// nothing, so dependents are scheduled only when every CTA of this grid is
+// running or done: a dependent CTA waiting for this grid never holds an SM
+// that one of its CTAs still needs, whatever the grid size.
 TQ_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 TQ_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

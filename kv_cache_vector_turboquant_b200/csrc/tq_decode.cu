@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // programmatic dependent launch: the next kernel may set up as CTAs exit
+  if (threadIdx.x == 0) grid_dep_launch();
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t out_addr = (smem_base + Sm::OUT + 1023u) & ~1023u;
   const uint32_t lut_addr = out_addr + Sm::OUT_BYTES;
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
     __syncwarp();
   };
 
+  grid_dep_wait();  // the previous kernel of the stream may still write the codes
 #pragma unroll
   for (int s = 0; s < DEC_STAGES; ++s) {
     const int64_t t = gw + s * n_warps;
@@ -362,8 +365,7 @@ static cudaError_t launch_decode_t(const tq_codec_tables& T, DecArgs a, cudaStre
     const int64_t tiles = (n + Cfg::VPW - 1) / Cfg::VPW;
     const int64_t ctas = (tiles + DEC_WARPS - 1) / DEC_WARPS;
     const int grid = (int)std::min<int64_t>(ctas, (int64_t)tq_sm_count(dev));
-    decode_kernel<D, BITS, OS><<<grid, DEC_WARPS * 32, smem, st>>>(T, a);
-    e = cudaGetLastError();
+    e = tq_launch_pdl(decode_kernel<D, BITS, OS>, dim3(grid), dim3(DEC_WARPS * 32), smem, st, T, a);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -260,6 +260,8 @@ __global__ void __launch_bounds__(W * 32, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // programmatic dependent launch: the next kernel may set up as CTAs exit
+  if (threadIdx.x == 0) grid_dep_launch();
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t in_addr = (smem_base + Sm::HEADER + 1023u) & ~1023u;  // stages: 1024-byte aligned
   const uint32_t lut_addr = in_addr + Sm::IN_BYTES;
@@ -315,6 +317,7 @@ __global__ void __launch_bounds__(W * 32, 1)
     __syncwarp();
   };
 
+  grid_dep_wait();  // the previous kernel of the stream may still write the inputs
 #pragma unroll
   for (int s = 0; s < ENC_STAGES; ++s) {
     const int t = gw + s * n_warps;
@@ -606,13 +609,14 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
     const int64_t tiles = (n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
     if (!OS && tiles <= (int64_t)ENC_WARPS_SMALL * sms) {
       const int grid = (int)((tiles + ENC_WARPS_SMALL - 1) / ENC_WARPS_SMALL);
-      encode_kernel<D, BITS, ENC_WARPS_SMALL, false><<<grid, ENC_WARPS_SMALL * 32, smem_small, st>>>(T, a);
+      e = tq_launch_pdl(encode_kernel<D, BITS, ENC_WARPS_SMALL, false>, dim3(grid), dim3(ENC_WARPS_SMALL * 32),
+                        smem_small, st, T, a);
     } else {
       const int64_t ctas_needed = (tiles + ENC_WARPS_BULK - 1) / ENC_WARPS_BULK;
       const int grid = (int)std::min<int64_t>(ctas_needed, (int64_t)sms);
-      encode_kernel<D, BITS, ENC_WARPS_BULK, OS><<<grid, ENC_WARPS_BULK * 32, smem_bulk, st>>>(T, a);
+      e = tq_launch_pdl(encode_kernel<D, BITS, ENC_WARPS_BULK, OS>, dim3(grid), dim3(ENC_WARPS_BULK * 32), smem_bulk,
+                        st, T, a);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
