@@ -22,7 +22,11 @@
  *  - Execution: device work is enqueued asynchronously on `stream` (a
  *    cudaStream_t; NULL = the legacy default stream) of the current device.
  *    Argument validation happens on the host before anything is enqueued; on
- *    any error nothing is enqueued.
+ *    any error nothing is enqueued. The encode and decode kernels are
+ *    launched with programmatic stream serialisation: a kernel may start its
+ *    set-up (shared and tensor memory only) while the previous kernel of the
+ *    stream is finishing, and touches global memory only after that kernel
+ *    has completed, so stream order holds for every buffer.
  *  - Layout: fp16 data is IEEE binary16 stored as uint16; every tensor is
  *    dense row-major; leading dimensions are flattened, so any [..., d] tensor
  *    is `n` rows.
