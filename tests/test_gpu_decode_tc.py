@@ -95,3 +95,22 @@ def test_tc_decode_bulk_call_uses_it_and_head_dim_256_does_not(K, W):
     p256, n256 = _random_codes(t256, 300, 12)
     x = torch.empty(300, 256, dtype=torch.float16, device="cuda")
     assert K._binding.tq_test_decode_path(t256.ctx, p256, n256, 300, x, 2) == K.TQ_ERR_UNSUPPORTED
+
+
+def test_tc_decode_matches_cuda_core_kernel_on_random_sizes(K, W):
+    """30 seeded random (d, bits, n, seed), n up to 300k (uneven tile counts
+    per CTA, every ragged tail), the layer's own codes: the two decode
+    kernels give identical fp16 rows."""
+    g = np.random.default_rng(2027)
+    for t in range(30):
+        d = int(g.choice([64, 128]))
+        bits = int(g.integers(2, 5))
+        n = int(g.integers(1, 300_000))
+        x = W.single_tensor(n=n, d=d, seed=500 + t, outlier_frac=0.02).cuda()
+        tq = K.TurboQuant(d, bits, seed=int(g.integers(0, 2**31)))
+        packed, norms = tq.encode(x)
+        x2 = _dec_path(K, tq, packed, norms, 2)
+        x1 = _dec_path(K, tq, packed, norms, 1)
+        assert torch.equal(x1, x2), (d, bits, n)
+        del x, packed, norms, x1, x2
+    assert K.tq_device_error() == (K.TQ_OK, 0)
