@@ -426,36 +426,57 @@ def _bench_long_context(K, W, torch, reps=2):
     return out
 
 
-def _cpu_baseline(seconds_target=12.0):
-    """The fp64 oracle, as it stands, on a bounded sample of the same workload:
-    encode + decode of sampled K rows of the layer at 4 bits."""
-    import numpy as np
-    import torch
+LLAMA_WORKLOAD = ("llama_layer: K and V fp16 [8,8192,8,128] (K with 4 x10 channels per head), "
+                  "encode+decode at bits 2,3,4")
 
-    import oracle as O
-    from kv_cache_vector_turboquant_b200 import workloads as W
 
+def _oracle_cores() -> int:
     try:
         from threadpoolctl import threadpool_info
 
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count() or 1
-    k, _ = W.llama_layer(device="cpu")
-    flat = k.reshape(-1, D)
-    rows = torch.randperm(flat.shape[0], generator=torch.Generator().manual_seed(0))
-    done, t_total, chunk = 0, 0.0, 16384
-    while t_total < seconds_target and done + chunk <= flat.shape[0]:
-        xs = flat[rows[done:done + chunk]].numpy()
+        return os.cpu_count() or 1
+
+
+def _oracle_sample(rows: int, seed: int):
+    """`rows` random rows of each of the layer's K and V tensors (same rows)."""
+    import torch
+
+    from kv_cache_vector_turboquant_b200 import workloads as W
+
+    k, v = W.llama_layer(device="cpu")
+    fk, fv = k.reshape(-1, D), v.reshape(-1, D)
+    idx = torch.randperm(fk.shape[0], generator=torch.Generator().manual_seed(seed))[:rows]
+    return fk[idx].numpy(), fv[idx].numpy()
+
+
+def _oracle_step(xk, xv) -> int:
+    """One pass of the benchmarked step on a sample: encode and decode of the
+    K and V rows at 2, 3 and 4 bits. Returns its fp16-equivalent bytes."""
+    import oracle as O
+
+    for bits in BITS:
+        for xs in (xk, xv):
+            p, nrm = O.encode(xs, bits, 42)
+            O.decode(p, nrm, bits, 42, D)
+    return len(BITS) * 2 * 2 * (2 * D) * (len(xk))
+
+
+def _cpu_baseline(seconds_target=12.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the same
+    workload: the benchmarked step (K and V, encode + decode at 2, 3 and 4
+    bits) on chunks of randomly sampled rows until about `seconds_target`."""
+    chunk, t_total, done, nbytes = 2048, 0.0, 0, 0
+    xk, xv = _oracle_sample(128 * chunk, 0)
+    while t_total < seconds_target and done + chunk <= len(xk):
         t0 = time.perf_counter()
-        p, nrm = O.encode(xs, 4, 42)
-        O.decode(p, nrm, 4, 42, D)
+        nbytes += _oracle_step(xk[done:done + chunk], xv[done:done + chunk])
         t_total += time.perf_counter() - t0
         done += chunk
-    fp16eq = 2 * (2 * D) * done  # encode + decode of `done` vectors
-    return {"value": fp16eq / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done} random rows of the layer's K tensor, encode+decode at 4 bits, fp64 numpy "
-                      f"({t_total:.1f} s)"}
+    return {"value": nbytes / t_total / 1e9, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{done} random rows of each of the layer's K and V tensors, encode+decode at 2, 3 and 4 "
+                      f"bits, fp64 numpy ({t_total:.1f} s)"}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -565,8 +586,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "llama_layer: K and V fp16 [8,8192,8,128] (K with 4 x10 channels per head), "
-                               "encode+decode at bits 2,3,4", "head_dim": D, "vectors_per_tensor": S["n"],
+        "config": {"workload": LLAMA_WORKLOAD, "head_dim": D, "vectors_per_tensor": S["n"],
                    "l2": "inputs larger than L2 (128 MiB per tensor; no launch re-reads what the previous wrote)",
                    "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
         "roofline": roof,
@@ -656,35 +676,31 @@ def _e2e(K, torch, S, steps, world, dist):
 
 
 def run_reference(args):
-    """The fp64 oracle on the host cores, as it stands, on a bounded sample."""
-    base = _cpu_baseline(seconds_target=max(2.0, 20.0 / max(1, args.steps + args.warmup)))
-    # each step: encode + decode of a fixed 16384-row sample at 4 bits
-    import numpy as np
-    import torch
-
-    import oracle as O
-    from kv_cache_vector_turboquant_b200 import workloads as W
-
-    k, _ = W.llama_layer(device="cpu")
-    xs = k.reshape(-1, D)[torch.randperm(k.numel() // D, generator=torch.Generator().manual_seed(1))[:16384]].numpy()
+    """The fp64 oracle on the host cores, as it stands: each step is the
+    benchmarked step (K and V, encode + decode at 2, 3 and 4 bits) on a fixed
+    sample of rows, sized so the whole run ends within a few minutes."""
+    rows = 2048
+    xk, xv = _oracle_sample(rows, 1)
     for _ in range(args.warmup):
-        O.decode(*O.encode(xs, 4, 42), 4, 42, D)
+        _oracle_step(xk, xv)
     t0 = time.perf_counter()
+    nbytes = 0
     for _ in range(args.steps):
-        O.decode(*O.encode(xs, 4, 42), 4, 42, D)
+        nbytes += _oracle_step(xk, xv)
     dt = time.perf_counter() - t0
-    val = 2 * 2 * D * len(xs) * args.steps / dt / 1e9
-    base["value"] = val
-    base["sample"] = f"16384 random rows of the layer's K tensor per step, encode+decode at 4 bits, fp64 numpy"
+    val = nbytes / dt / 1e9
+    sample = (f"{rows} random rows of each of the layer's K and V tensors per step, encode+decode at 2, 3 and 4 "
+              f"bits, fp64 numpy")
     return {"impl": "reference", "metric": "encode/decode GB/s (fp16-equivalent) & % of HBM roofline; "
                                            "fused attn tokens/s",
             "value": val, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama_layer: K fp16 [8,8192,8,128], 16384 sampled rows per step, "
-                                   "encode+decode at 4 bits"},
-            "cpu_baseline": base, "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0,
-                                          "d2h_bytes_per_step": 0}}
+            "config": {"workload": LLAMA_WORKLOAD, "head_dim": D, "vectors_per_tensor": 8 * 8192 * 8,
+                       "sample": sample},
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 PROFILE_CASES = ["encode_b2", "encode_b3", "encode_b4", "decode_b2", "decode_b3", "decode_b4", "attn"]
