@@ -30,6 +30,9 @@ Readings taken where the pages are silent:
   z = sqrt(d) * H D u.
 * sign i is -1 iff bit 63 of the i-th splitmix64 output (seeded with ``seed``)
   is set (splitmix64: S. Vigna, public-domain reference generator).
+  ``splitmix64`` and ``sign_vector`` are pinned to Vigna's published outputs,
+  but the pages neither name their own generator nor print any sign or
+  packed byte, so agreement with the pages' sign table is parity unpinned.
 * the format codebook is the fp64 Lloyd-Max codebook for N(0, 1) snapped to the
   2^-14 grid; decision boundaries are the midpoints of the snapped levels;
   index = number of boundaries t with z >= t (ties go to the upper level).
