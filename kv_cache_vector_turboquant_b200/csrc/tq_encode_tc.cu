@@ -17,27 +17,33 @@
 //  * one thread of warp 0 streams 128-vector tiles into a ring of
 //    shared-memory stages (5 at d = 128) with 2-D tensor copies (64-column
 //    boxes, 128-byte swizzle, no multicast), refilling a stage as soon as its
-//    MMAs are done;
+//    MMAs are done and the norm warps have read it;
 //  * one thread of warp 1 issues per tile d/16 tcgen05 MMAs of M = 128
 //    vectors by N = K = 16 (A: the tile's columns of block b; B: H_16 with
 //    block b's signs folded in, fp16 +-1, built in shared memory once). The
 //    f32 results live in tensor memory: d columns per tile, 512/d tiles in
 //    flight;
+//  * two norm warps read each tile's fp16 rows from its shared-memory stage
+//    (before the stage is refilled) and sum x^2 on the CUDA cores, one
+//    mixed-precision FMA (fp16 inputs, f32 accumulator) per element in 8
+//    or 16 chains; the square root goes to the epilogue through a small
+//    per-accumulator buffer in shared memory;
 //  * three epilogue warpgroups (two at d = 256) take turns on the tiles, one
-//    vector per thread (TMEM lane = tile row): sum_{b,j} S^2 = 16 ||x||^2
-//    gives the norm; the remaining log2(d/16) butterfly stages run in
-//    registers with packed f32x2 on 4 positions j at a time (2 at d = 256),
-//    two such chunks per loop iteration; the quantiser, guard band and fp64
-//    recheck are those of encode_kernel; each thread stores its packed row
-//    and norm.
+//    vector per thread (TMEM lane = tile row): the remaining log2(d/16)
+//    butterfly stages run in registers with packed f32x2 on 4 positions j at
+//    a time (2 at d = 256), two such chunks per loop iteration; the
+//    quantiser, guard band and fp64 recheck are those of encode_kernel; each
+//    thread stores its packed row and norm.
 //
 // Exactness: the tensor core's arithmetic for kind::f16 with f32 accumulation
 // was measured on B200 (every product exact; each addend's magnitude cut to a
 // multiple of 2^(E-25), E the largest addend exponent; the sum rounded toward
 // zero). For one 16-term block that bounds the error of S[b][j] by
-// 7.5 u max_k |x_k| + 2 u |S[b][j]| (u = 2^-24); with the f32 stages, the norm
-// from S and the scaling, the error of q stays below the guard band of
-// encode_kernel (9.3e-6 at d = 128 against 1e-5; 1.3e-5 at d = 256 against
+// 7.5 u max_k |x_k| + 2 u |S[b][j]| (u = 2^-24); with the f32 stages, the
+// norm (at most 9.5 u relative at d <= 128, 10 u at 256: squares of fp16
+// values are exact in f32, chains of at most 16 terms and a tree of at most
+// 4 levels) and the scaling, the error of q stays below the guard band of
+// encode_kernel (7.4e-6 at d = 128 against 1e-5; 1.1e-5 at d = 256 against
 // 2e-5), so unflagged decisions are the exact ones and flagged coordinates
 // are recomputed in fp64 from the fp16 inputs.
 #include <cuda.h>
@@ -71,7 +77,10 @@ struct TcCfg {
   // waiting for use k of an accumulator's barrier always finds use k - 1
   // complete (a parity wait cannot tell use k from use k - 2)
   static constexpr int GROUPS = NACC < TC_GROUPS ? NACC : TC_GROUPS;
-  static constexpr int WARPS = 2 + 4 * GROUPS;       // warp 0: copies, warp 1: MMAs
+  static constexpr int NW0 = 2 + 4 * GROUPS;         // first of the two norm warps
+  static constexpr int WARPS = NW0 + 2;              // warp 0: copies, warp 1: MMAs
+  // f32 chains of the sum of squares (at most 16 terms each)
+  static constexpr int NCH = D == 256 ? 16 : 8;
   static constexpr int JC = D == 256 ? 2 : 4;        // positions j per epilogue chunk
   static constexpr int CHUNKS = 16 / JC;
   static constexpr int NV = NB * JC;                 // values per chunk (16 or 32)
@@ -83,9 +92,10 @@ struct TcCfg {
                                                                       : (1u | 1u << BITS));
   // shared memory, from a 1024-aligned base: the stages first
   static constexpr int BREG = STAGES * TILE_BYTES;   // NB/4 regions of 16 rows x 128 B
-  static constexpr int BAR = BREG + NB / 4 * 2048;   // full, empty, tfull, tempty, done
-  static constexpr int NBARS = 2 * STAGES + 2 * NACC + 1;
-  static constexpr int SLOT = BAR + NBARS * 8;       // TMEM base address
+  static constexpr int BAR = BREG + NB / 4 * 2048;   // full, empty, tfull, tempty, nfull, done
+  static constexpr int NBARS = 2 * STAGES + 3 * NACC + 1;
+  static constexpr int NRM = BAR + NBARS * 8;        // per accumulator: the tile's 128 norms
+  static constexpr int SLOT = NRM + NACC * TC_ROWS * 4;  // TMEM base address
   static constexpr int SIGN = SLOT + 16;             // D sign bits (bit l of word t: coordinate 32 t + l)
   static constexpr int BND = SIGN + 32;              // the 2^BITS - 1 boundaries, z units
   static constexpr int SCR = (BND + 64 + 127) & ~127;  // per epilogue warp: 32 words
@@ -115,6 +125,47 @@ TQ_DEV uint2 tc_lds_u2(uint32_t addr) {
   uint2 r;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
   return r;
+}
+
+TQ_DEV uint4 tc_lds_u4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
+}
+
+// a0 += lo(w)^2, a1 += hi(w)^2 for the fp16 pair w: mixed-precision FMAs of
+// sm_100 (fp16 operands, f32 addend and result). The square of an fp16 value
+// is exact in f32, so each step rounds once.
+TQ_DEV void tc_sq_acc2(float& a0, float& a1, uint32_t w) {
+  asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "fma.rn.f32.f16 %0, lo, lo, %0;\n\tfma.rn.f32.f16 %1, hi, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w));
+}
+
+// sqrt(sum x^2) of row r of a tile staged in shared memory at `st` (boxes of
+// 64 columns, 128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)), in
+// NCH f32 chains of at most 16 terms and a tree
+template <int D, int NCH>
+TQ_DEV float tc_row_norm(uint32_t st, int r) {
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  float ch[NCH];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) ch[c] = 0.f;
+#pragma unroll
+  for (int c = 0; c < CPR; ++c) {
+    const uint4 v = tc_lds_u4(st + (c >> 3) * (TC_ROWS * 128) + r * 128 + ((((c & 7) ^ (r & 7))) << 4));
+    float* cc = ch + ((c >> 3) & (NCH / 8 - 1)) * 8;
+    tc_sq_acc2(cc[0], cc[1], v.x);
+    tc_sq_acc2(cc[2], cc[3], v.y);
+    tc_sq_acc2(cc[4], cc[5], v.z);
+    tc_sq_acc2(cc[6], cc[7], v.w);
+  }
+#pragma unroll
+  for (int w = NCH / 2; w > 0; w >>= 1)
+#pragma unroll
+    for (int c = 0; c < w; ++c) ch[c] += ch[c + w];
+  return sqrtf(ch[0]);
 }
 
 TQ_DEV void tc_tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -214,15 +265,16 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
   const int cnt = (int64_t)blockIdx.x < n_tiles ? (int)((n_tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
 
   const uint32_t bar0 = base + Cfg::BAR;
-  const uint32_t done_bar = bar0 + 8u * (2 * S + 2 * NACC);
+  const uint32_t done_bar = bar0 + 8u * (2 * S + 3 * NACC);
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar0 + 8u * s, 1);        // full: tile landed
-      mbar_init(bar0 + 8u * (S + s), 1);  // empty: its MMAs done
+      mbar_init(bar0 + 8u * s, 1);             // full: tile landed
+      mbar_init(bar0 + 8u * (S + s), 1 + 64);  // empty: its MMAs done, its rows read by the norm warps
     }
     for (int q = 0; q < NACC; ++q) {
-      mbar_init(bar0 + 8u * (2 * S + q), 1);         // tfull: accumulator written
-      mbar_init(bar0 + 8u * (2 * S + NACC + q), 4);  // tempty: its 4 warps read it
+      mbar_init(bar0 + 8u * (2 * S + q), 1);             // tfull: accumulator written
+      mbar_init(bar0 + 8u * (2 * S + NACC + q), 4);      // tempty: its 4 warps read it (and its norms)
+      mbar_init(bar0 + 8u * (2 * S + 2 * NACC + q), 64);  // nfull: the tile's norms written
     }
     mbar_init(done_bar, 1);
     fence_mbar_init();
@@ -273,7 +325,7 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
 
   if (warp == 0) {
     // ---- producer: tile i of this CTA into stage i % S as soon as the MMAs
-    // of tile i - S have released it
+    // and the norm warps of tile i - S have released it
     if (lane == 0 && !a.fault_inject) {
       grid_dep_wait();  // the previous kernel of the stream may still write x
       for (int i = 0; i < cnt; ++i) {
@@ -326,10 +378,12 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
     const float Rscale = T.inv_delta, qoff = T.q_offset, gq = T.guard_q;
     const f2 Q2 = make_float2(qoff, qoff), M2 = make_float2(TC_MAGIC_2P23, TC_MAGIC_2P23);
     grid_dep_wait();  // before the first store and the first recheck load
+    const float* nbuf = reinterpret_cast<const float*>(sm + Cfg::NRM);
     for (int i = g; i < cnt; i += Cfg::GROUPS) {
       const int q = i % NACC;
       // warp-uniform decision: the tensor-memory loads below are warp-collective
-      const bool ok = mbar_wait_bounded(bar0 + 8u * (2 * S + q), (i / NACC) & 1, a.wait_limit);
+      const bool ok = mbar_wait_bounded(bar0 + 8u * (2 * S + q), (i / NACC) & 1, a.wait_limit) &&
+                      mbar_wait_bounded(bar0 + 8u * (2 * S + 2 * NACC + q), (i / NACC) & 1, a.wait_limit);
       if (!__all_sync(FULL, ok)) {
         if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
         break;
@@ -340,28 +394,8 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
       const bool active = row < a.n;
       const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(q * D);
 
-      // ---- norm: sum over b, j of S^2 = 16 ||x||^2, in 8 f32 chains
-      f2 acc[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(tl + c, r0);
-        tmem_ld16(tl + c + 16, r1);
-        tmem_wait_ld();
-        tmem_regs_after_wait(r0);
-        tmem_regs_after_wait(r1);
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const f2 v0 = make_float2(__uint_as_float(r0[2 * p]), __uint_as_float(r0[2 * p + 1]));
-          const f2 v1 = make_float2(__uint_as_float(r1[2 * p]), __uint_as_float(r1[2 * p + 1]));
-          acc[p & 3] = fma2(v0, v0, acc[p & 3]);
-          acc[p & 3] = fma2(v1, v1, acc[p & 3]);
-        }
-      }
-      const f2 s4 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-      const float nrm = sqrtf((s4.x + s4.y) * 0.0625f);
+      // ---- norm of this thread's vector, from the norm warps
+      const float nrm = nbuf[q * TC_ROWS + 32 * quarter + lane];
       const bool special = !(nrm > 0.f) || !(nrm <= 3.0e38f);  // zero or non-finite vector
       const float R = special ? 0.f : __fdiv_rn(Rscale, nrm);
       const f2 R2 = make_float2(R, R);
@@ -529,6 +563,32 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
         }
         a.norms[row] = nrm;
       }
+    }
+  } else if (warp >= Cfg::NW0) {
+    // ---- norm warps: rows 64 k + lane and 64 k + 32 + lane of every tile,
+    // read from the tile's stage as soon as it lands; N = sqrt(sum x^2) in
+    // NCH f32 chains (at most 16 terms each, then a tree), written to the
+    // accumulator's norm buffer once the epilogue has taken the previous
+    // tile's norms from it
+    const int k = warp - Cfg::NW0;
+    float* nbuf = reinterpret_cast<float*>(sm + Cfg::NRM);
+    for (int i = 0; i < cnt; ++i) {
+      const int s = i % S, q = i % NACC;
+      bool ok = mbar_wait_bounded(bar0 + 8u * s, (i / S) & 1, a.wait_limit);
+      if (ok && i >= NACC) ok = mbar_wait_bounded(bar0 + 8u * (2 * S + NACC + q), ((i / NACC) - 1) & 1, a.wait_limit);
+      if (!__all_sync(FULL, ok)) {
+        if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
+        break;
+      }
+      const uint32_t st = base + s * Cfg::TILE_BYTES;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int r = 64 * k + 32 * rr + lane;
+        nbuf[q * TC_ROWS + r] = tc_row_norm<D, Cfg::NCH>(st, r);
+      }
+      // every thread arrives: its reads of the stage are done and its norms written
+      mbar_arrive(bar0 + 8u * (S + s));
+      mbar_arrive(bar0 + 8u * (2 * S + 2 * NACC + q));
     }
   }
   // ---- teardown: every role is done (or gave up); free the tensor memory
