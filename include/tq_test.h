@@ -61,6 +61,15 @@ tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float
  */
 tq_status tq_test_umma_block(const void* a_f16, const void* b_f16, float* d, tq_stream stream);
 
+/*
+ * Forget the current device's result of the tensor-core check
+ * (tq_tensor_core_check), so that the next bulk tq_encode / tq_decode or
+ * tq_tensor_core_check runs it again. With force_fail != 0 that next check
+ * reports a mismatch whatever the MMA returned, so a test can see bulk
+ * launches fall back to the CUDA-core kernels. Host only.
+ */
+tq_status tq_test_reset_tensor_core_check(int force_fail);
+
 #ifdef __cplusplus
 }
 #endif

@@ -44,6 +44,7 @@ from ._binding import (  # noqa: F401
     tq_encode_slots,
     tq_get_tables,
     tq_status_string,
+    tq_tensor_core_check,
 )
 
 

@@ -46,6 +46,8 @@ _PROTOS = {
     "tq_attend_decode_paged": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64, _vp,
                                         _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "tq_tensor_core_check": (_c_int, [ctypes.POINTER(_c_int)]),
+    "tq_test_reset_tensor_core_check": (_c_int, [_c_int]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
     "tq_test_umma_block": (_c_int, [_vp, _vp, _vp, _vp]),
@@ -225,6 +227,20 @@ def tq_device_error(stream=None) -> tuple[int, int]:
     bits = ctypes.c_uint32(0)
     st = _lib.tq_device_error(_stream(stream), ctypes.byref(bits))
     return st, bits.value
+
+
+def tq_tensor_core_check() -> bool:
+    """Run (once per device) the check of the tensor-core rounding that the
+    bulk encode and decode kernels rely on; True if it passed."""
+    passed = _c_int(0)
+    _check(_lib.tq_tensor_core_check(ctypes.byref(passed)), "tq_tensor_core_check")
+    return bool(passed.value)
+
+
+def tq_test_reset_tensor_core_check(force_fail: bool = False) -> int:
+    """Test hook: forget the current device's check result (force the next
+    check to report a mismatch if `force_fail`); returns the status."""
+    return _lib.tq_test_reset_tensor_core_check(int(bool(force_fail)))
 
 
 def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> int:

@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtq.so")
 
-SOURCES = ["tq_host.cpp", "tq_device.cu", "tq_encode.cu", "tq_encode_tc.cu", "tq_decode.cu", "tq_decode_tc.cu", "tq_attend.cu", "tq_attend_fast.cu", "tq_attend_static.cu", "tq_test_umma.cu"]
+SOURCES = ["tq_host.cpp", "tq_device.cu", "tq_encode.cu", "tq_encode_tc.cu", "tq_decode.cu", "tq_decode_tc.cu", "tq_attend.cu", "tq_attend_fast.cu", "tq_attend_static.cu", "tq_mma_check.cu", "tq_test_umma.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]
 

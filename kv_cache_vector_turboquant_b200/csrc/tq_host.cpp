@@ -206,7 +206,8 @@ tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packe
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  if (n >= tq_encode_tc_min_rows()) return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
+  if (n >= tq_encode_tc_min_rows() && tq_tensor_cores_usable(stream))
+    return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 0);
 }
 
@@ -216,7 +217,7 @@ tq_status tq_decode(const tq_ctx* ctx, const void* packed, const float* norms, i
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  if (n >= tq_encode_tc_min_rows()) {
+  if (n >= tq_encode_tc_min_rows() && tq_tensor_cores_usable(stream)) {
     // the tensor-core kernel at head_dim <= 128
     const tq_status st = tq_launch_decode_tc(ctx, packed, norms, n, x_f16, stream);
     if (st != TQ_ERR_UNSUPPORTED) return st;

@@ -93,6 +93,13 @@ tq_status tq_launch_attend_paged(const tq_ctx* k, const tq_ctx* v, const void* q
                                  size_t ws_bytes, void* stream);
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max);
 
+// 1 if the tensor-core encode and decode kernels may run on the current
+// device: the run-time check of the tensor core's rounding (tq_mma_check.cu)
+// has passed there, running it first if it has not run yet (unless `stream`
+// is being captured: then 0 without running it, so the call takes the
+// CUDA-core kernel).
+int tq_tensor_cores_usable(void* stream);
+
 // cuTensorMapEncodeTiled from the driver (cached; null if unavailable).
 void* tq_tensor_map_encode_fn(void);
 
