@@ -439,11 +439,26 @@ def _oracle_cores() -> int:
         return os.cpu_count() or 1
 
 
+def _loaded_native_libs() -> list:
+    """Shared libraries of this repository mapped into this process."""
+    out = set()
+    try:
+        with open("/proc/self/maps") as f:
+            for ln in f:
+                path = ln.split()[-1] if ln.strip() else ""
+                if path.startswith(ROOT) and ".so" in os.path.basename(path):
+                    out.add(os.path.relpath(path, ROOT))
+    except OSError:
+        pass
+    return sorted(out)
+
+
 def _oracle_sample(rows: int, seed: int):
-    """`rows` random rows of each of the layer's K and V tensors (same rows)."""
+    """`rows` random rows of each of the layer's K and V tensors (same rows),
+    generated on the host (the oracle arm touches no GPU)."""
     import torch
 
-    from kv_cache_vector_turboquant_b200 import workloads as W
+    import tq_workloads as W
 
     k, v = W.llama_layer(device="cpu")
     fk, fv = k.reshape(-1, D), v.reshape(-1, D)
@@ -463,20 +478,125 @@ def _oracle_step(xk, xv) -> int:
     return len(BITS) * 2 * 2 * (2 * D) * (len(xk))
 
 
-def _cpu_baseline(seconds_target=12.0):
+def _ordered_f16(h):
+    """fp16 bit patterns -> integers ordered like the values (+0 == -0)."""
+    import numpy as np
+
+    u = np.asarray(h, dtype=np.float16).view(np.uint16).astype(np.int32)
+    return np.where(u & 0x8000, -(u & 0x7FFF), u)
+
+
+class _ParityTally:
+    """The GPU's outputs for sampled rows of the benchmarked tensors against
+    the oracle's: code mismatches (and how many of them lie outside the 1e-5
+    boundary band), the largest relative norm error and the largest fp16 ulp
+    distance between the GPU decode of the GPU's bytes and the oracle decode
+    of the same bytes, per width and tensor."""
+
+    def __init__(self):
+        self.t = {}
+
+    def add(self, bits, name, det, gp, gn, gx):
+        import numpy as np
+
+        import oracle as O
+
+        r = self.t.setdefault(f"{name}_b{bits}", {"coords_checked": 0, "boundary_mismatches": 0,
+                                                  "mismatches_outside_band": 0, "max_norm_rel_err": 0.0,
+                                                  "max_decode_ulp": 0})
+        gi = O.unpack_codes(gp, bits, D)
+        mism = gi != det["idx"]
+        r["coords_checked"] += int(gi.size)
+        r["boundary_mismatches"] += int(mism.sum())
+        if mism.any():
+            t = O.format_boundaries(O.format_levels(bits))
+            dist = np.min(np.abs(det["z"][mism][:, None] - t[None, :]), axis=1)
+            r["mismatches_outside_band"] += int((dist >= 1e-5).sum())
+        ref = det["norm64"]
+        ok = ref > 0
+        rel = np.abs(gn.astype(np.float64)[ok] - ref[ok]) / ref[ok]
+        r["max_norm_rel_err"] = max(r["max_norm_rel_err"], float(rel.max()) if rel.size else 0.0)
+        ulp = np.abs(_ordered_f16(gx) - _ordered_f16(O.decode(gp, gn, bits, 42, D)))
+        r["max_decode_ulp"] = max(r["max_decode_ulp"], int(ulp.max()))
+
+    def summary(self):
+        tot = sum(v["coords_checked"] for v in self.t.values())
+        mis = sum(v["boundary_mismatches"] for v in self.t.values())
+        return {"coords_checked": tot, "boundary_mismatches": mis,
+                "boundary_mismatch_frac": mis / tot if tot else None,
+                "mismatches_outside_band": sum(v["mismatches_outside_band"] for v in self.t.values()),
+                "max_norm_rel_err": max((v["max_norm_rel_err"] for v in self.t.values()), default=None),
+                "max_decode_ulp": max((v["max_decode_ulp"] for v in self.t.values()), default=None),
+                "per_tensor": self.t}
+
+
+def _gpu_sample(K, torch, S, rows, seed=0):
+    """`rows` random rows of the benchmarked K and V tensors and the GPU's
+    codes, norms and decoded rows for them at 2, 3 and 4 bits: the codes and
+    norms the timed step's encodes left in its buffers, the decode re-run
+    on them with the step's own launch (one bulk tq_decode per tensor)."""
+    n = S["n"]
+    idx = torch.randperm(n, generator=torch.Generator().manual_seed(seed))[:rows].sort().values.cuda()
+    xs = {t: S["xs"][t][idx].cpu().numpy() for t in "KV"}
+    gpu = {}
+    for b in BITS:
+        for t in "KV":
+            K.tq_decode(S["codecs"][b].ctx, S["packed"][b, t], S["norms"][b, t], n, S["out"])
+            gpu[b, t] = (S["packed"][b, t][idx].cpu().numpy(), S["norms"][b, t][idx].cpu().numpy(),
+                         S["out"][idx].cpu().numpy())
+    torch.cuda.synchronize()
+    return xs, gpu
+
+
+def _timed_oracle_chunks(xk, xv, seconds, start, chunk, tally=None, gpu=None):
+    """Oracle steps on consecutive chunks of the sample from row `start` until
+    about `seconds` of oracle time; returns (rows done, bytes, seconds). The
+    comparison with the GPU's outputs (when given) is not timed."""
+    import oracle as O
+
+    t_total, done, nbytes = 0.0, 0, 0
+    while t_total < seconds and start + done + chunk <= len(xk):
+        r0, r1 = start + done, start + done + chunk
+        for bits in BITS:
+            for name, xs in (("K", xk), ("V", xv)):
+                t0 = time.perf_counter()
+                det = O.encode_detail(xs[r0:r1], bits, 42)
+                O.decode(det["packed"], det["norms"], bits, 42, D)
+                t_total += time.perf_counter() - t0
+                nbytes += 2 * (2 * D) * chunk
+                if tally is not None:
+                    gp, gn, gx = gpu[bits, name]
+                    tally.add(bits, name, det, gp[r0:r1], gn[r0:r1], gx[r0:r1])
+        done += chunk
+    return done, nbytes, t_total
+
+
+def _cpu_baseline(xk, xv, gpu=None, seconds_target=9.0, single_thread_seconds=3.0, chunk=2048):
     """The fp64 oracle, as it stands, on a bounded sample of the same
     workload: the benchmarked step (K and V, encode + decode at 2, 3 and 4
-    bits) on chunks of randomly sampled rows until about `seconds_target`."""
-    chunk, t_total, done, nbytes = 2048, 0.0, 0, 0
-    xk, xv = _oracle_sample(128 * chunk, 0)
-    while t_total < seconds_target and done + chunk <= len(xk):
-        t0 = time.perf_counter()
-        nbytes += _oracle_step(xk[done:done + chunk], xv[done:done + chunk])
-        t_total += time.perf_counter() - t0
-        done += chunk
-    return {"value": nbytes / t_total / 1e9, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
-            "sample": f"{done} random rows of each of the layer's K and V tensors, encode+decode at 2, 3 and 4 "
-                      f"bits, fp64 numpy ({t_total:.1f} s)"}
+    bits) on chunks of the sampled rows, first with numpy's thread pool on
+    every core for about `seconds_target`, then on one thread for about
+    `single_thread_seconds`. With the GPU's outputs for the same rows, every
+    processed row is also compared with the oracle (untimed)."""
+    tally = _ParityTally() if gpu is not None else None
+    cores = _oracle_cores()
+    done, nbytes, t_all = _timed_oracle_chunks(xk, xv, seconds_target, 0, chunk, tally, gpu)
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            d1, b1, t1 = _timed_oracle_chunks(xk, xv, single_thread_seconds, done, chunk // 4)
+        if d1:
+            single = {"value": b1 / t1 / 1e9, "unit": "GB/s", "cores": 1,
+                      "sample": f"{d1} further rows of each tensor ({t1:.1f} s)"}
+    except ImportError:
+        pass
+    out = {"value": nbytes / t_all / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": f"{done} random rows of each of the layer's K and V tensors, encode+decode at 2, 3 and 4 "
+                     f"bits, fp64 numpy on {cores} threads ({t_all:.1f} s)",
+           "single_thread": single}
+    return out, (tally.summary() if tally is not None else None)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -484,7 +604,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import kv_cache_vector_turboquant_b200 as K
-    from kv_cache_vector_turboquant_b200 import workloads as W
+    import tq_workloads as W
 
     torch.cuda.set_device(local_rank)
     S = _codec_step_setup(K, W, torch, rank)
@@ -602,12 +722,33 @@ def run_ours(args, rank, world, local_rank):
     if not args.skip_extras:
         result["attn"] = _bench_attention(K, W, torch, max(args.steps, 5), max(args.warmup, 3),
                                           float(result["clocks"].get("sm_mhz") or 1965.0))
+        at = result["attn"]
+        result["attn_summary"] = {"tokens_per_s": at["tokens_per_s"], "us_per_step": at["ms_per_step"] * 1e3,
+                                  "GBps": at["roofline"]["achieved"], "frac": at["roofline"]["frac"],
+                                  "paged_us_per_step": at["paged"]["ms_per_step"] * 1e3,
+                                  "paged_frac": at["paged"]["frac"]}
         result["append"] = _bench_append(K, W, torch)
         result["long_context"] = _bench_long_context(K, W, torch)
         result["offset_variant"] = _bench_offset_variant(K, W, torch)
     if rank == 0 and world == 1 and not args.skip_cpu:
-        result["cpu_baseline"] = _cpu_baseline()
-    return result
+        xs, gpu = _gpu_sample(K, torch, S, 131072)
+        result["cpu_baseline"], result["parity"] = _cpu_baseline(xs["K"], xs["V"], gpu)
+    result["native_libs_loaded"] = _loaded_native_libs()
+    return _front(result)
+
+
+# keys printed first, so that a reader (or a tool that keeps only the head of
+# the line) sees the headline, the roofline, the parity tally and the
+# attention figures before the detail
+_FRONT = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+          "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "clocks", "gpu_launches", "parity",
+          "attn_summary", "cpu_baseline"]
+
+
+def _front(result: dict) -> dict:
+    out = {k: result[k] for k in _FRONT if k in result}
+    out.update({k: v for k, v in result.items() if k not in out})
+    return out
 
 
 def _e2e(K, torch, S, steps, world, dist, chunk_rows=65536, n_streams=4):
@@ -696,7 +837,7 @@ def run_reference(args):
     dt = time.perf_counter() - t0
     val = nbytes / dt / 1e9
     sample = (f"{rows} random rows of each of the layer's K and V tensors per step, encode+decode at 2, 3 and 4 "
-              f"bits, fp64 numpy")
+              f"bits, fp64 numpy on {_oracle_cores()} threads")
     return {"impl": "reference", "metric": "encode/decode GB/s (fp16-equivalent) & % of HBM roofline; "
                                            "fused attn tokens/s",
             "value": val, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -706,7 +847,8 @@ def run_reference(args):
                        "sample": sample},
             "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
                              "sample": sample},
-            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "native_libs_loaded": _loaded_native_libs()}
 
 
 PROFILE_CASES = ["encode_b2", "encode_b3", "encode_b4", "decode_b2", "decode_b3", "decode_b4", "attn"]
@@ -719,7 +861,7 @@ def run_profile_case(case: str, launches: int = 3):
     import torch
 
     import kv_cache_vector_turboquant_b200 as K
-    from kv_cache_vector_turboquant_b200 import workloads as W
+    import tq_workloads as W
 
     torch.cuda.set_device(0)
     if case == "attn":

@@ -90,6 +90,8 @@ def test_reference_arm_line_matches_the_gpu_arm_contract():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+    # the oracle arm maps none of the library's shared objects
+    assert line["native_libs_loaded"] == []
 
 
 def test_reference_arm_other_ranks_exit_quietly():

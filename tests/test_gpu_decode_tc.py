@@ -26,7 +26,7 @@ def K(cuda_device):
 
 @pytest.fixture(scope="module")
 def W():
-    from kv_cache_vector_turboquant_b200 import workloads as W
+    import tq_workloads as W
 
     return W
 
