@@ -664,9 +664,16 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
                   {(cuuint32_t)hw, 1, BP}))
     return cudaErrorNotSupported;
 
+  // the fast kernel's own split (one CTA per SM and kv-head group); the
+  // workspace was laid out for the generic kernel's a.n_split, so a larger
+  // split count would overrun it: leave such a launch to the generic kernel
+  int n_split = 0, chunk = 0;
+  attn_split_for(sm_count / hg, a.B, a.s_max, &n_split, &chunk);
+  if (n_split > a.n_split) return cudaErrorNotSupported;
   a.nt = nt;
   a.hw_max = hw;
-  attn_split_for(sm_count / hg, a.B, a.s_max, &a.n_split, &a.chunk);
+  a.n_split = n_split;
+  a.chunk = chunk;
   f.a = a;
   void (*kern)(FastArgs) = nullptr;
   if (d == 128) kern = hw == 4 ? attend_fast_kernel<128, 4> : hw == 8 ? attend_fast_kernel<128, 8> : attend_fast_kernel<128, 16>;
