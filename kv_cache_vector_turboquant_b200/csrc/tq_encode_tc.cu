@@ -29,7 +29,9 @@
 //    or 16 chains; the square root goes to the epilogue through a small
 //    per-accumulator buffer in shared memory;
 //  * three epilogue warpgroups (two at d = 256) take turns on the tiles, one
-//    vector per thread (TMEM lane = tile row): the remaining log2(d/16)
+//    vector per thread (TMEM lane = tile row); at d <= 128 setmaxnreg moves
+//    registers from warpgroup 0 (copies, MMAs, norms: 56 each) to them (152
+//    each), so more table lookups stay in flight: the remaining log2(d/16)
 //    butterfly stages run in registers with packed f32x2 on 4 positions j at
 //    a time (2 at d = 256), two such chunks per loop iteration; the
 //    quantiser, guard band and fp64 recheck are those of encode_kernel; each
@@ -77,8 +79,13 @@ struct TcCfg {
   // waiting for use k of an accumulator's barrier always finds use k - 1
   // complete (a parity wait cannot tell use k from use k - 2)
   static constexpr int GROUPS = NACC < TC_GROUPS ? NACC : TC_GROUPS;
-  static constexpr int NW0 = 2 + 4 * GROUPS;         // first of the two norm warps
-  static constexpr int WARPS = NW0 + 2;              // warp 0: copies, warp 1: MMAs
+  // warpgroup 0: copies, MMAs and the two norm warps; then the epilogue warpgroups
+  static constexpr int NW0 = 2;                      // first of the two norm warps
+  static constexpr int EPI0 = 4;                     // first epilogue warp
+  static constexpr int WARPS = EPI0 + 4 * GROUPS;
+  // registers per thread after the split (launch: 128 per thread at 16 warps)
+  static constexpr int REG_CTRL = 56, REG_EPI = 152;
+  static constexpr bool SPLIT = WARPS == 16;  // (d = 256 runs 12 warps at their launch registers)
   // f32 chains of the sum of squares (at most 16 terms each)
   static constexpr int NCH = D == 256 ? 16 : 8;
   static constexpr int JC = D == 256 ? 2 : 4;        // positions j per epilogue chunk
@@ -323,56 +330,89 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
     asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");  // the tables are complete
   }
 
-  if (warp == 0) {
-    // ---- producer: tile i of this CTA into stage i % S as soon as the MMAs
-    // and the norm warps of tile i - S have released it
-    if (lane == 0 && !a.fault_inject) {
-      grid_dep_wait();  // the previous kernel of the stream may still write x
-      for (int i = 0; i < cnt; ++i) {
-        const int s = i % S;
-        if (i >= S && !mbar_wait_bounded(bar0 + 8u * (S + s), ((i / S) - 1) & 1, a.wait_limit)) {
-          record_error(a.err, TQ_DEVERR_TIMEOUT);
-          break;
+  if (warp < Cfg::EPI0) {
+    // warpgroup 0: copies (warp 0), MMAs (warp 1), norms (warps 2, 3)
+    if constexpr (Cfg::SPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Cfg::REG_CTRL));
+    if (warp == 0) {
+      // ---- producer: tile i of this CTA into stage i % S as soon as the MMAs
+      // and the norm warps of tile i - S have released it
+      if (lane == 0 && !a.fault_inject) {
+        grid_dep_wait();  // the previous kernel of the stream may still write x
+        for (int i = 0; i < cnt; ++i) {
+          const int s = i % S;
+          if (i >= S && !mbar_wait_bounded(bar0 + 8u * (S + s), ((i / S) - 1) & 1, a.wait_limit)) {
+            record_error(a.err, TQ_DEVERR_TIMEOUT);
+            break;
+          }
+          const int y = (int)(((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * TC_ROWS);
+          mbar_arrive_expect_tx(bar0 + 8u * s, Cfg::TILE_BYTES);
+  #pragma unroll
+          for (int bx = 0; bx < Cfg::BOXES; ++bx)
+            tc_tma_load_2d(base + s * Cfg::TILE_BYTES + bx * Cfg::BOX_BYTES, &a.tm_x, 64 * bx, y, bar0 + 8u * s);
         }
-        const int y = (int)(((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * TC_ROWS);
-        mbar_arrive_expect_tx(bar0 + 8u * s, Cfg::TILE_BYTES);
-#pragma unroll
-        for (int bx = 0; bx < Cfg::BOXES; ++bx)
-          tc_tma_load_2d(base + s * Cfg::TILE_BYTES + bx * Cfg::BOX_BYTES, &a.tm_x, 64 * bx, y, bar0 + 8u * s);
       }
-    }
-  } else if (warp == 1) {
-    // ---- MMA issuer: S[b] = A_b * B_b^T for the d/16 blocks of tile i
-    if (lane == 0) {
-      grid_dep_wait();  // (its only global access is the error word)
-      constexpr uint32_t IDESC = umma_idesc_f16(TC_ROWS, 16);
+    } else if (warp == 1) {
+      // ---- MMA issuer: S[b] = A_b * B_b^T for the d/16 blocks of tile i
+      if (lane == 0) {
+        grid_dep_wait();  // (its only global access is the error word)
+        constexpr uint32_t IDESC = umma_idesc_f16(TC_ROWS, 16);
+        for (int i = 0; i < cnt; ++i) {
+          const int s = i % S, q = i % NACC;
+          if (!mbar_wait_bounded(bar0 + 8u * s, (i / S) & 1, a.wait_limit) ||
+              (i >= NACC && !mbar_wait_bounded(bar0 + 8u * (2 * S + NACC + q), ((i / NACC) - 1) & 1, a.wait_limit))) {
+            record_error(a.err, TQ_DEVERR_TIMEOUT);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = base + s * Cfg::TILE_BYTES;
+  #pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const uint64_t ad = umma_desc_sw128(st + (b >> 2) * Cfg::BOX_BYTES + (b & 3) * 32);
+            const uint64_t bd = umma_desc_sw128(base + Cfg::BREG + (b >> 2) * 2048 + (b & 3) * 32);
+            umma_f16(tmem + (uint32_t)(q * D + 16 * b), ad, bd, IDESC, false);
+          }
+          umma_commit(bar0 + 8u * (S + s));      // the stage may be refilled
+          umma_commit(bar0 + 8u * (2 * S + q));  // the accumulator may be read
+        }
+        // every MMA issued has completed before tensor memory is freed
+        umma_commit(done_bar);
+        if (!mbar_wait_bounded(done_bar, 0, a.wait_limit)) record_error(a.err, TQ_DEVERR_TIMEOUT);
+      }
+    } else {
+      // ---- norm warps: rows 64 k + lane and 64 k + 32 + lane of every tile,
+      // read from the tile's stage as soon as it lands; N = sqrt(sum x^2) in
+      // NCH f32 chains (at most 16 terms each, then a tree), written to the
+      // accumulator's norm buffer once the epilogue has taken the previous
+      // tile's norms from it
+      const int k = warp - Cfg::NW0;
+      float* nbuf = reinterpret_cast<float*>(sm + Cfg::NRM);
       for (int i = 0; i < cnt; ++i) {
         const int s = i % S, q = i % NACC;
-        if (!mbar_wait_bounded(bar0 + 8u * s, (i / S) & 1, a.wait_limit) ||
-            (i >= NACC && !mbar_wait_bounded(bar0 + 8u * (2 * S + NACC + q), ((i / NACC) - 1) & 1, a.wait_limit))) {
-          record_error(a.err, TQ_DEVERR_TIMEOUT);
+        bool ok = mbar_wait_bounded(bar0 + 8u * s, (i / S) & 1, a.wait_limit);
+        if (ok && i >= NACC) ok = mbar_wait_bounded(bar0 + 8u * (2 * S + NACC + q), ((i / NACC) - 1) & 1, a.wait_limit);
+        if (!__all_sync(FULL, ok)) {
+          if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
           break;
         }
-        tc_fence_after();
         const uint32_t st = base + s * Cfg::TILE_BYTES;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const uint64_t ad = umma_desc_sw128(st + (b >> 2) * Cfg::BOX_BYTES + (b & 3) * 32);
-          const uint64_t bd = umma_desc_sw128(base + Cfg::BREG + (b >> 2) * 2048 + (b & 3) * 32);
-          umma_f16(tmem + (uint32_t)(q * D + 16 * b), ad, bd, IDESC, false);
+  #pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int r = 64 * k + 32 * rr + lane;
+          nbuf[q * TC_ROWS + r] = tc_row_norm<D, Cfg::NCH>(st, r);
         }
-        umma_commit(bar0 + 8u * (S + s));      // the stage may be refilled
-        umma_commit(bar0 + 8u * (2 * S + q));  // the accumulator may be read
+        // every thread arrives: its reads of the stage are done and its norms written
+        mbar_arrive(bar0 + 8u * (S + s));
+        mbar_arrive(bar0 + 8u * (2 * S + 2 * NACC + q));
       }
-      // every MMA issued has completed before tensor memory is freed
-      umma_commit(done_bar);
-      if (!mbar_wait_bounded(done_bar, 0, a.wait_limit)) record_error(a.err, TQ_DEVERR_TIMEOUT);
     }
-  } else if (((warp - 2) >> 2) < Cfg::GROUPS) {
+  } else {
+    // the epilogue warpgroups; registers from warpgroup 0 move here:
+    // 3 x 128 x 152 + 128 x 56 = 512 x 128, the launch's total
+    if constexpr (Cfg::SPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Cfg::REG_EPI));
     // ---- epilogue warpgroup g (warps 4g + 2 ... 4g + 5, which cover the four
     // lane quarters of tensor memory): tiles g, g + GROUPS, ...; one vector per thread
-    const int g = (warp - 2) >> 2, quarter = warp & 3;
-    float* scratch = reinterpret_cast<float*>(sm + Cfg::SCR + (warp - 2) * 128);
+    const int g = (warp - Cfg::EPI0) >> 2, quarter = warp & 3;
+    float* scratch = reinterpret_cast<float*>(sm + Cfg::SCR + (warp - Cfg::EPI0) * 128);
     // (2^23 + cell) * 128 = 2^31 + cell * 128 (mod 2^32): the 2^31 is taken out here
     const uint32_t lut_lane = base + Cfg::LUT + (uint32_t)(lane & (TC_LUT_COPIES - 1)) * 8u - 0x80000000u;
     const float Rscale = T.inv_delta, qoff = T.q_offset, gq = T.guard_q;
@@ -564,32 +604,6 @@ __global__ void __launch_bounds__(TcCfg<D, BITS>::WARPS * 32, 1)
         a.norms[row] = nrm;
       }
     }
-  } else if (warp >= Cfg::NW0) {
-    // ---- norm warps: rows 64 k + lane and 64 k + 32 + lane of every tile,
-    // read from the tile's stage as soon as it lands; N = sqrt(sum x^2) in
-    // NCH f32 chains (at most 16 terms each, then a tree), written to the
-    // accumulator's norm buffer once the epilogue has taken the previous
-    // tile's norms from it
-    const int k = warp - Cfg::NW0;
-    float* nbuf = reinterpret_cast<float*>(sm + Cfg::NRM);
-    for (int i = 0; i < cnt; ++i) {
-      const int s = i % S, q = i % NACC;
-      bool ok = mbar_wait_bounded(bar0 + 8u * s, (i / S) & 1, a.wait_limit);
-      if (ok && i >= NACC) ok = mbar_wait_bounded(bar0 + 8u * (2 * S + NACC + q), ((i / NACC) - 1) & 1, a.wait_limit);
-      if (!__all_sync(FULL, ok)) {
-        if (lane == 0) record_error(a.err, TQ_DEVERR_TIMEOUT);
-        break;
-      }
-      const uint32_t st = base + s * Cfg::TILE_BYTES;
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = 64 * k + 32 * rr + lane;
-        nbuf[q * TC_ROWS + r] = tc_row_norm<D, Cfg::NCH>(st, r);
-      }
-      // every thread arrives: its reads of the stage are done and its norms written
-      mbar_arrive(bar0 + 8u * (S + s));
-      mbar_arrive(bar0 + 8u * (2 * S + 2 * NACC + q));
-    }
   }
   // ---- teardown: every role is done (or gave up); free the tensor memory
   tc_fence_before();
@@ -614,6 +628,17 @@ static cudaError_t launch_encode_tc_t(const tq_codec_tables& T, TcArgs a, const 
     e = cudaFuncSetAttribute(encode_tc_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Cfg::bytes(TQ_MAX_CELLS));
     if (e != cudaSuccess) return e;
+    if constexpr (Cfg::SPLIT) {
+      // the epilogue's setmaxnreg.inc waits until warpgroup 0 has released
+      // enough registers: it can only complete if the launch holds the whole
+      // split (3 x 128 x REG_EPI + 128 x REG_CTRL registers), so check the
+      // registers the kernel is launched with before the first launch
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, encode_tc_kernel<D, BITS>);
+      if (e != cudaSuccess) return e;
+      if ((int64_t)fa.numRegs * Cfg::WARPS * 32 < (int64_t)128 * (3 * Cfg::REG_EPI + Cfg::REG_CTRL))
+        return cudaErrorNotSupported;
+    }
     configured.fetch_or(bit);
   }
   auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tq_tensor_map_encode_fn());
@@ -678,5 +703,7 @@ tq_status tq_launch_encode_tc(const tq_ctx* ctx, const void* x, int64_t n, void*
   TQ_ENCTC_CASE(128, 2) TQ_ENCTC_CASE(128, 3) TQ_ENCTC_CASE(128, 4)
   TQ_ENCTC_CASE(256, 2) TQ_ENCTC_CASE(256, 3) TQ_ENCTC_CASE(256, 4)
 #undef TQ_ENCTC_CASE
-  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  // cudaErrorNotSupported: a launch this kernel cannot make (the caller
+  // takes the CUDA-core kernel)
+  return e == cudaSuccess ? TQ_OK : e == cudaErrorNotSupported ? TQ_ERR_UNSUPPORTED : TQ_ERR_CUDA;
 }

@@ -206,8 +206,10 @@ tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packe
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  if (n >= tq_encode_tc_min_rows() && tq_tensor_cores_usable(stream))
-    return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
+  if (n >= tq_encode_tc_min_rows() && tq_tensor_cores_usable(stream)) {
+    const tq_status st = tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
+    if (st != TQ_ERR_UNSUPPORTED) return st;
+  }
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 0);
 }
 

@@ -68,6 +68,8 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
 // Bulk encode on the tensor cores (tq_encode_tc.cu): the same outputs as
 // tq_launch_encode without append slots. tq_encode uses it from
 // tq_encode_tc_min_rows() vectors on (one 128-vector tile per SM).
+// TQ_ERR_UNSUPPORTED (nothing launched) when the kernel cannot be launched
+// as planned; the caller then takes the CUDA-core kernel.
 tq_status tq_launch_encode_tc(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms, void* stream,
                               int fault_inject);
 int64_t tq_encode_tc_min_rows(void);
