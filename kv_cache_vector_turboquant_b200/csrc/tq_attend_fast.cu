@@ -67,6 +67,12 @@ constexpr float FA_RESCALE_LOG2 = 8.f;  // raise the running max only past this 
 #define FA_V_LUT_GROUPS 3  // groups of value m-blocks (of 4) dequantised through the shared table
 #endif
 
+// Floats per staged norm row: the copy box is wider than the CTA's kv heads
+// (the excess is zero-filled), so the norms of the 8 positions a warp reads
+// at once fall in 8 different banks (a pitch of hw floats would put rows gq
+// and gq + 4 in one bank for hw = 8).
+__host__ __device__ constexpr int fa_norm_pitch(int hw) { return hw == 4 ? 12 : hw + 4; }
+
 struct FastArgs {
   CUtensorMap tm_k;   // K codes  box (D/2 bytes, 32 positions, hw heads) -> [head][position][D/2]
   CUtensorMap tm_v;   // V codes  box (hw * D/4 + 16 bytes, 1 group, 32 positions)
@@ -149,6 +155,7 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
   constexpr int VQW = D / 128;  // words of a V row per lane (an eighth)
   constexpr int VP = HW * PV + 16;  // shared pitch of a V position row
   constexpr int hw = HW;            // kv heads per CTA
+  constexpr int NPITCH = fa_norm_pitch(HW);  // floats per staged norm row
   const AttnArgs& a = f.a;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) != f.smem_base) {  // the table addressing needs the planned addresses
@@ -204,8 +211,8 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
         const int row = h ? rb : ra;
         tma_load_3d(smem_u32(smem + f.kbuf[s] + h * hw * ATT_BLOCK * PK), &f.tm_k, 0, row, hgrp * hw, bar);
         tma_load_3d(smem_u32(smem + f.vbuf[s] + h * ATT_BLOCK * VP), &f.tm_v, 0, hgrp, row, bar);
-        tma_load_3d(smem_u32(smem + f.knb[s] + h * ATT_BLOCK * hw * 4), &f.tm_kn, 0, hgrp, row, bar);
-        tma_load_3d(smem_u32(smem + f.vnb[s] + h * ATT_BLOCK * hw * 4), &f.tm_vn, 0, hgrp, row, bar);
+        tma_load_3d(smem_u32(smem + f.knb[s] + h * ATT_BLOCK * NPITCH * 4), &f.tm_kn, 0, hgrp, row, bar);
+        tma_load_3d(smem_u32(smem + f.vnb[s] + h * ATT_BLOCK * NPITCH * 4), &f.tm_vn, 0, hgrp, row, bar);
       }
       issued[s] += 1;
       return;
@@ -365,8 +372,8 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
         const uint32_t a3 = lds_tab32(__byte_perm(w1, LK, so));
         mma16816(c, a0, a1, a2, a3, bq[kb][0], bq[kb][1]);
       }
-      sc[mb16][0] = (c[0] + c[1]) * kns[r0 * hw];
-      sc[mb16][1] = (c[2] + c[3]) * kns[(r0 + 8) * hw];
+      sc[mb16][0] = (c[0] + c[1]) * kns[r0 * NPITCH];
+      sc[mb16][1] = (c[2] + c[3]) * kns[(r0 + 8) * NPITCH];
     }
     const bool ragged = nv < ATT_TILE;
     if (ragged) {
@@ -397,7 +404,7 @@ __global__ void __launch_bounds__(FA_WARPS * 32, 1) attend_fast_kernel(const __g
         const int row = mb16 * 16 + gq + 8 * r;
         const float p = fast_exp2(sc[mb16][r] - m_run);
         l_run += p;
-        float pv = p * vns[row * hw];
+        float pv = p * vns[row * NPITCH];
         if (ragged && row >= nv) pv = 0.f;
         bp[mb16][r] = transpose8x8(split_hi_lo(pv));
       }
@@ -627,7 +634,8 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   f.wpt = hw * nt;
   f.n_groups = FA_WARPS / f.wpt;
   f.vpitch = hw * pv + 16;
-  const int kbytes = ATT_TILE * hw * pk, vbytes = ATT_TILE * f.vpitch, nbytes = ATT_TILE * hw * 4;
+  const int np = fa_norm_pitch(hw);
+  const int kbytes = ATT_TILE * hw * pk, vbytes = ATT_TILE * f.vpitch, nbytes = ATT_TILE * np * 4;
   // paged: 2 KB after the 128-byte header hold the rows of the split's first
   // 512 blocks, so the issuing thread reads them from shared memory
   f.pg_off = 128;
@@ -659,9 +667,9 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
   if (!encode_map(&f.tm_v, U64, a.v_packed, {(cuuint64_t)hw * pv / 8, HG, R},
                   {(cuuint64_t)hw * pv, (cuuint64_t)a.hkv * pv}, {(cuuint32_t)f.vpitch / 8, 1, BP}) ||
       !encode_map(&f.tm_kn, F32, a.k_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
-                  {(cuuint32_t)hw, 1, BP}) ||
+                  {(cuuint32_t)np, 1, BP}) ||
       !encode_map(&f.tm_vn, F32, a.v_norms, {(cuuint64_t)hw, HG, R}, {(cuuint64_t)hw * 4, (cuuint64_t)a.hkv * 4},
-                  {(cuuint32_t)hw, 1, BP}))
+                  {(cuuint32_t)np, 1, BP}))
     return cudaErrorNotSupported;
 
   // the fast kernel's own split (one CTA per SM and kv-head group); the
