@@ -6,17 +6,17 @@
 // steps 4-1): x_hat = D (H_pm c[idx]) * (N / d), H_pm the +-1 natural-order
 // Walsh-Hadamard matrix, D the seeded sign flip, c the codebook levels.
 //
-// Factorisation used: H_pm = H_{d/16} (x) H_16 (Sylvester's construction):
-// coordinate 16 b' + j of H_pm c is sum_b (-1)^popc(b' & b) S[b][j] with
-// S[b] = H_16 c_b. The tensor cores compute every S[b] of a 128-vector tile.
-// The levels lie on the 2^-14 grid (16 significant bits), so each level is
-// split into an fp16 value and an fp16 remainder (both exact); two MMAs per
-// block accumulate H_16 (value) + H_16 (remainder). Every addend is a
-// multiple of 2^-14 below 2^6 and the tensor core cuts addends only below
-// 2^(E-25) with E <= 6, so the block sums are exact; the f32 butterflies
-// across blocks are exact too (multiples of 2^-14 below 2^10), and the only
-// roundings are the product by N / d and the fp16 conversion, as in
-// decode_kernel.
+// The whole transform runs on the tensor cores: per 128-vector tile,
+// Y = C H_pm^T with C the tile's levels (128 rows x d) and B = H_pm (d x d,
+// +-1), accumulated over the d/16 K-steps. The levels lie on the 2^-14 grid
+// (16 significant bits), so each level is split into an fp16 value and an
+// fp16 remainder (both exact) and both parts are multiplied (2 d/16 MMAs of
+// M = 128, N = d, K = 16 into one accumulator). Every product and every
+// partial sum is a multiple of 2^-14 below 2^9 (|H_pm c| <= d max|c| < 2^9),
+// so it is exact in f32, and the tensor core cuts addends only below
+// 2^(E-25) with E <= 9 and rounds an exact sum to itself: Y is exact. The
+// only roundings are the product by N / d and the fp16 conversion, as in
+// decode_kernel (outputs bit-identical).
 //
 // B200 mapping (one persistent CTA of 18 warps per SM, warp-specialised):
 //  * warp 0: 1-D bulk copies of each full tile's packed rows into a ring of
@@ -25,16 +25,16 @@
 //    thread): each pair of codes indexes a
 //    lane-replicated table of {value pair, remainder pair} as packed fp16,
 //    which go straight into tensor memory with tcgen05.st (A operand: row m
-//    in lane m, two fp16 per 32-bit column, 8 columns per 16-element block);
+//    in lane m, two fp16 per 32-bit column, 8 columns per 16-element K-step);
 //  * warp 1: per tile 2 d/16 MMAs with A from tensor memory ([a-tmem] form)
-//    and B = H_16 (fp16 +-1, shared memory), f32 accumulators in tensor
-//    memory: two A operands (the builders refill one as soon as the MMAs
-//    that read it commit) and one accumulator per epilogue warpgroup;
-//  * warps 10-17 (two epilogue warpgroups, one row per thread): the
-//    log2(d/16) cross-block butterflies in f32x2, the scale N / d, the
-//    fp16 conversion and the sign flip on fp16 pairs, staged in the group's
-//    128-byte-swizzled tile and written by 2-D tensor stores (which clip a
-//    partial last tile).
+//    and B = H_pm (fp16 +-1, shared memory, built once per CTA), f32
+//    accumulators in tensor memory: two A operands (the builders refill a
+//    half as soon as the MMAs that read it commit) and one accumulator per
+//    epilogue warpgroup;
+//  * warps 10-17 (two epilogue warpgroups, one row per thread): the scale
+//    N / d, the fp16 conversion and the sign flip on fp16 pairs, staged in
+//    the group's 128-byte-swizzled tile and written by 2-D tensor stores
+//    (which clip a partial last tile).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -66,13 +66,11 @@ struct DtCfg {
   static constexpr int NA = 2;
   static constexpr int ACC0 = NA * D;
   static constexpr int STAGES = 8;
-  static constexpr int JC = 4;                      // positions j per epilogue chunk
-  static constexpr int CHUNKS = 16 / JC;
   // shared memory, from a 1024-aligned base
   static constexpr int OUT = 0;                     // 2 groups x BOXES x [128 rows x 128 B]
   static constexpr int OUT_BYTES = BOXES * DT_ROWS * 128;
-  static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_16, 16 rows x 128 B
-  static constexpr int IN = BREG + 2048;            // STAGES x TILE_P
+  static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_d: BOXES atoms of d rows x 128 B
+  static constexpr int IN = BREG + D * D * 2;       // STAGES x TILE_P
   static constexpr int LUT = IN + STAGES * TILE_P;  // E x 32 lane copies x 8 B
   static constexpr int BAR = LUT + E * 32 * 8;
   // full[S], empty[S], aready[NA][2], aempty[NA][2], tfull[2], tempty[2], done
@@ -127,7 +125,7 @@ template <int D, int BITS>
 __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     decode_tc_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ DtArgs a) {
   using Cfg = DtCfg<D, BITS>;
-  constexpr int NB = Cfg::NB, S = Cfg::STAGES, NA = Cfg::NA, WORDS = Cfg::WORDS, JC = Cfg::JC;
+  constexpr int NB = Cfg::NB, S = Cfg::STAGES, NA = Cfg::NA, WORDS = Cfg::WORDS;
   constexpr uint32_t FULL = 0xffffffffu;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -208,7 +206,17 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
         *reinterpret_cast<uint4*>(row + jj * 16) = make_uint4(ev, er, ev, er);
       }
     }
-    asm volatile("bar.sync 3, 512;" ::: "memory");  // the table is complete
+    // B = H_d (natural order, +-1; the signs are applied to the fp16 output)
+    // as an N = d by K = d operand, K-major with the 128-byte swizzle: atom
+    // k / 64 holds row n at n * 128 bytes, its 16-byte chunk c at c ^ (n % 8)
+    for (int e = t; e < D * D; e += 512) {
+      const int n = e / D, k = e % D;
+      const uint32_t off = Cfg::BREG + (k >> 6) * (D * 128) + n * 128 + (((((k & 63) * 2) >> 4) ^ (n & 7)) << 4) +
+                           ((k * 2) & 15);
+      *reinterpret_cast<uint16_t*>(sm + off) = (__popc(n & k) & 1) ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
+    }
+    fence_proxy_async_smem();  // B is read by the tensor cores
+    asm volatile("bar.sync 3, 544;" ::: "memory");  // the table and B are complete (warps 1-17)
   }
 
   if (warp == 0) {
@@ -231,19 +239,12 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer: per block, S = A_value H_16^T + A_remainder H_16^T
-    // ---- B = H_16 (the signs are applied to the fp16 output), K-major swizzled
-    for (int e = lane; e < 256; e += 32) {
-      const int j = e >> 4, k = e & 15;
-      const uint32_t off = Cfg::BREG + j * 128 + ((((k * 2) >> 4) ^ (j & 7)) << 4) + ((k * 2) & 15);
-      *reinterpret_cast<uint16_t*>(sm + off) = (__popc(j & k) & 1) ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
-    }
-    fence_proxy_async_smem();  // B is read by the tensor cores
-    __syncwarp();
+    // ---- MMA issuer: the whole transform, D = (A_value + A_remainder) H_d^T
+    // accumulated over the d/16 K-steps of both parts (exact: see the top)
+    asm volatile("bar.sync 3, 544;" ::: "memory");  // B (and the table) are built
     if (lane == 0) {
       grid_dep_wait();  // (its only global access is the error word)
-      constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, 16);
-      const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG);
+      constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, D);
       bool ok = true;
       for (int i = 0; i < cnt && ok; ++i) {
         const int k = i % NA, g = i & 1;
@@ -261,8 +262,10 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
           tc_fence_after();
 #pragma unroll
           for (int b = h * NB / 2; b < (h + 1) * NB / 2; ++b) {
-            umma_f16_ts(db + (uint32_t)(16 * b), ab + (uint32_t)(8 * b), bdesc, IDESC, false);
-            umma_f16_ts(db + (uint32_t)(16 * b), ab + (uint32_t)(D / 2 + 8 * b), bdesc, IDESC, true);
+            // K-step b: coordinates 16 b ... 16 b + 15 of the levels
+            const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG + (b >> 2) * (D * 128) + (b & 3) * 32);
+            umma_f16_ts(db, ab + (uint32_t)(8 * b), bdesc, IDESC, b > 0);
+            umma_f16_ts(db, ab + (uint32_t)(D / 2 + 8 * b), bdesc, IDESC, true);
           }
           umma_commit(aempty0 + 8u * (2 * k + h));  // this half may be rewritten
         }
@@ -382,43 +385,37 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       if (leader && stored_once) bulk_wait_read<0>();
       asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
       const uint32_t tl = tmem + lanebase + (uint32_t)(Cfg::ACC0 + g * D);
+      // column n of the accumulator is coordinate n of H_pm c: 32 columns per
+      // tensor-memory wait, 16 coordinates per pair of 16-byte staging stores
 #pragma unroll
-      for (int c = 0; c < Cfg::CHUNKS; ++c) {
-        const int j0 = c * JC;
-        uint32_t rv[NB][JC];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) tmem_ld4(tl + (uint32_t)(16 * b + j0), rv[b]);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rv[2][16];
+        tmem_ld16(tl + (uint32_t)(32 * c), rv[0]);
+        tmem_ld16(tl + (uint32_t)(32 * c + 16), rv[1]);
         tmem_wait_ld();
-#pragma unroll
-        for (int b = 0; b < NB; ++b) tmem_regs_after_wait(rv[b]);
-        if (c == Cfg::CHUNKS - 1) {  // every load of the accumulator is done: free the slot
+        tmem_regs_after_wait(rv[0]);
+        tmem_regs_after_wait(rv[1]);
+        if (c == D / 32 - 1) {  // every load of the accumulator is done: free the slot
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty0 + 8u * g);
         }
-        f2 v[JC / 2][NB];
 #pragma unroll
-        for (int h = 0; h < JC / 2; ++h) {
+        for (int u = 0; u < 2; ++u) {
+          const int k0 = 32 * c + 16 * u;  // first coordinate of these 16
+          uint32_t hw[8];
 #pragma unroll
-          for (int b = 0; b < NB; ++b)
-            v[h][b] = make_float2(__uint_as_float(rv[b][2 * h]), __uint_as_float(rv[b][2 * h + 1]));
-          wht_pairs<NB>(v[h]);
-        }
-#pragma unroll
-        for (int bp = 0; bp < NB; ++bp) {
-          uint32_t hw[JC / 2];
-#pragma unroll
-          for (int h = 0; h < JC / 2; ++h) {
-            const int k = 16 * bp + j0 + 2 * h;  // first coordinate of the pair
-            const f2 y = mul2(v[h][bp], sc2);
+          for (int p = 0; p < 8; ++p) {
+            const f2 y = mul2(make_float2(__uint_as_float(rv[u][2 * p]), __uint_as_float(rv[u][2 * p + 1])), sc2);
             const __half2 hv = __floats2half2_rn(y.x, y.y);
-            hw[h] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[k >> 1];
+            hw[p] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[(k0 >> 1) + p];
           }
-          // coordinates 16 b' + j0 ... + 3: 8 bytes of the swizzled staging row
-          const int k0 = 16 * bp + j0, box = k0 >> 6, col = k0 & 63;
-          const uint32_t off = (uint32_t)(box * DT_ROWS * 128 + r * 128) +
-                               ((uint32_t)(((col >> 3) ^ (r & 7))) << 4) + (uint32_t)((col & 7) * 2);
-          *reinterpret_cast<uint2*>(out_sm + off) = make_uint2(hw[0], hw[1]);
+          // 32 bytes of the swizzled staging row: chunks col / 8 and col / 8 + 1
+          const int box = k0 >> 6, col = k0 & 63;
+          const uint32_t row_off = (uint32_t)(box * DT_ROWS * 128 + r * 128);
+          const uint32_t c0 = (uint32_t)((col >> 3) ^ (r & 7)), c1 = (uint32_t)(((col >> 3) + 1) ^ (r & 7));
+          *reinterpret_cast<uint4*>(out_sm + row_off + (c0 << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(out_sm + row_off + (c1 << 4)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
         }
       }
       fence_proxy_async_smem();
