@@ -1,5 +1,11 @@
 /*
  * tq_test.h -- test hooks of libtq. Not for production use.
+ *
+ * These calls are exported by libtq_test.so, a separate library linked
+ * against libtq.so (found beside it through $ORIGIN). They run libtq.so's own
+ * kernels and launchers, so they record into the same device error word
+ * (tq_device_error) as the public calls. The product library libtq.so
+ * exports none of them.
  */
 #ifndef TQ_TEST_H_
 #define TQ_TEST_H_

@@ -47,16 +47,40 @@ _PROTOS = {
                                         _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "tq_tensor_core_check": (_c_int, [ctypes.POINTER(_c_int)]),
+}
+for _name, (_res, _args) in _PROTOS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+# Test hooks (include/tq_test.h) live in libtq_test.so, which is linked
+# against libtq.so (the same loaded instance: same device error word) and is
+# loaded only when a hook is first called.
+_TEST_LIB_PATH = os.path.join(os.path.dirname(_LIB_PATH), "libtq_test.so")
+_TEST_PROTOS = {
     "tq_test_reset_tensor_core_check": (_c_int, [_c_int]),
     "tq_test_encode_stalled": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
     "tq_test_umma_block": (_c_int, [_vp, _vp, _vp, _vp]),
     "tq_test_decode_path": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _c_int, _vp]),
 }
-for _name, (_res, _args) in _PROTOS.items():
-    _f = getattr(_lib, _name)
-    _f.restype = _res
-    _f.argtypes = _args
+_test = None
+
+
+def _test_lib():
+    """libtq_test.so with its prototypes set (loaded on first use)."""
+    global _test
+    if _test is None:
+        if not os.path.exists(_TEST_LIB_PATH):
+            raise ImportError(f"libtq_test.so not found at {_TEST_LIB_PATH}; build it with "
+                              "`python kv_cache_vector_turboquant_b200/build.py`")
+        lib = ctypes.CDLL(_TEST_LIB_PATH)
+        for name, (res, args) in _TEST_PROTOS.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _test = lib
+    return _test
 
 TQ_OK = 0
 TQ_ERR_INVALID_ARG = 1
@@ -240,26 +264,26 @@ def tq_tensor_core_check() -> bool:
 def tq_test_reset_tensor_core_check(force_fail: bool = False) -> int:
     """Test hook: forget the current device's check result (force the next
     check to report a mismatch if `force_fail`); returns the status."""
-    return _lib.tq_test_reset_tensor_core_check(int(bool(force_fail)))
+    return _test_lib().tq_test_reset_tensor_core_check(int(bool(force_fail)))
 
 
 def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> int:
     """Test hook: encode with the row copies withheld; returns the launch status."""
-    return _lib.tq_test_encode_stalled(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), _stream(stream))
+    return _test_lib().tq_test_encode_stalled(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), _stream(stream))
 
 
 def tq_test_decode_path(ctx: Ctx, packed, norms, n: int, x, path: int, stream=None) -> int:
     """Test hook: decode through kernel `path` (1 CUDA cores, 2 tensor cores); returns the launch status."""
-    return _lib.tq_test_decode_path(ctx.handle, _ptr(packed), _ptr(norms), int(n), _ptr(x), int(path), _stream(stream))
+    return _test_lib().tq_test_decode_path(ctx.handle, _ptr(packed), _ptr(norms), int(n), _ptr(x), int(path), _stream(stream))
 
 
 def tq_test_umma_block(a, b, d, stream=None) -> int:
     """Test hook: one tcgen05 MMA d[128,16] = a[128,16] @ b[16,16]^T (fp16 in, f32 out)."""
-    return _lib.tq_test_umma_block(_ptr(a), _ptr(b), _ptr(d), _stream(stream))
+    return _test_lib().tq_test_umma_block(_ptr(a), _ptr(b), _ptr(d), _stream(stream))
 
 
 def tq_test_encode_path(ctx: Ctx, x, n: int, packed, norms, path: int, stream=None) -> int:
     """Test hook: encode through kernel `path` (1 CUDA cores, 2 tensor cores, 3 tensor
     cores with the row copies withheld); returns the launch status."""
-    return _lib.tq_test_encode_path(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), int(path),
+    return _test_lib().tq_test_encode_path(ctx.handle, _ptr(x), int(n), _ptr(packed), _ptr(norms), int(path),
                                     _stream(stream))

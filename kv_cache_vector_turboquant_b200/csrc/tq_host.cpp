@@ -318,38 +318,4 @@ tq_status tq_attend_decode_paged(const tq_ctx* k, const tq_ctx* v, const void* q
 
 tq_status tq_device_error(tq_stream stream, uint32_t* bits) { return tq_read_error_word(stream, bits); }
 
-// Test hook (declared in include/tq_test.h): run tq_encode with the row copies
-// withheld, so every wait of the kernel runs out after a short bound.
-tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms,
-                                 tq_stream stream) {
-  if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
-  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 1);
-}
-
-// Test hook (declared in include/tq_test.h): tq_decode through a chosen kernel.
-tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
-                              int path, tq_stream stream) {
-  if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
-  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  switch (path) {
-    case 1: return tq_launch_decode(ctx, packed, norms, n, x_f16, stream);
-    case 2: return tq_launch_decode_tc(ctx, packed, norms, n, x_f16, stream);
-    default: return TQ_ERR_INVALID_ARG;
-  }
-}
-
-// Test hook (declared in include/tq_test.h): tq_encode through a chosen kernel.
-tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, float* norms, int path,
-                              tq_stream stream) {
-  if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
-  if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
-  switch (path) {
-    case 1: return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 0);
-    case 2: return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 0);
-    case 3: return tq_launch_encode_tc(ctx, x_f16, n, packed, norms, stream, 1);
-    default: return TQ_ERR_INVALID_ARG;
-  }
-}
-
 }  // extern "C"

@@ -101,6 +101,9 @@ size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max
 // is being captured: then 0 without running it, so the call takes the
 // CUDA-core kernel).
 int tq_tensor_cores_usable(void* stream);
+// Forget the current device's check result; force_fail != 0 makes the next
+// check report a mismatch (used by the test hooks of libtq_test.so).
+tq_status tq_tensor_core_check_reset(int force_fail);
 
 // cuTensorMapEncodeTiled from the driver (cached; null if unavailable).
 void* tq_tensor_map_encode_fn(void);

@@ -178,10 +178,11 @@ extern "C" tq_status tq_tensor_core_check(int* passed) {
   return TQ_OK;
 }
 
-// Test hook (include/tq_test.h): forget the current device's result, so the
-// next bulk call or tq_tensor_core_check runs the check again; with
-// force_fail != 0 that check reports a mismatch whatever the MMA returns.
-extern "C" tq_status tq_test_reset_tensor_core_check(int force_fail) {
+// Forget the current device's result, so the next bulk call or
+// tq_tensor_core_check runs the check again; with force_fail != 0 that check
+// reports a mismatch whatever the MMA returns (for the test hook
+// tq_test_reset_tensor_core_check of libtq_test.so).
+tq_status tq_tensor_core_check_reset(int force_fail) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);

@@ -38,11 +38,19 @@ def _declared_symbols():
     return names
 
 
-def test_library_exports_every_declared_symbol(lib):
+def test_library_exports_every_declared_symbol(lib, K):
+    """libtq.so exports every call of include/tq.h and no test hook; the hooks
+    of include/tq_test.h come from libtq_test.so."""
     names = _declared_symbols()
     assert {"tq_create", "tq_encode", "tq_decode", "tq_encode_append", "tq_attend_decode"} <= names
-    for n in sorted(names):
+    hooks = {n for n in names if n.startswith("tq_test_")}
+    assert {"tq_test_encode_path", "tq_test_umma_block", "tq_test_reset_tensor_core_check"} <= hooks
+    test_lib = K._binding._test_lib()
+    for n in sorted(names - hooks):
         assert hasattr(lib, n), n
+    for n in sorted(hooks):
+        assert hasattr(test_lib, n), n
+        assert not hasattr(lib, n), f"{n} is a test hook but libtq.so exports it"
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
@@ -101,7 +109,8 @@ class _FakePtr:
 
 
 def _raw(K, name, *args):
-    return getattr(K._binding._lib, name)(*args)
+    lib = K._binding._test_lib() if name.startswith("tq_test_") else K._binding._lib
+    return getattr(lib, name)(*args)
 
 
 def test_encode_decode_validation(K):
