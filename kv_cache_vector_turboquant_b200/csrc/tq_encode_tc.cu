@@ -159,9 +159,13 @@ TQ_DEV float tc_row_norm(uint32_t st, int r) {
   float ch[NCH];
 #pragma unroll
   for (int c = 0; c < NCH; ++c) ch[c] = 0.f;
+  // the row's 8 swizzled chunk addresses (the swizzle depends only on r % 8)
+  uint32_t off[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) off[c] = st + r * 128 + (uint32_t)((c ^ (r & 7)) << 4);
 #pragma unroll
   for (int c = 0; c < CPR; ++c) {
-    const uint4 v = tc_lds_u4(st + (c >> 3) * (TC_ROWS * 128) + r * 128 + ((((c & 7) ^ (r & 7))) << 4));
+    const uint4 v = tc_lds_u4(off[c & 7] + (c >> 3) * (TC_ROWS * 128));
     float* cc = ch + ((c >> 3) & (NCH / 8 - 1)) * 8;
     tc_sq_acc2(cc[0], cc[1], v.x);
     tc_sq_acc2(cc[2], cc[3], v.y);
