@@ -290,9 +290,10 @@ def _bench_attention_paged(K, torch, a, q, kc, vc, kp, kn, vp, vn, pos, steps, w
 def _bench_append(K, W, torch, steps_per_run=1024):
     """Streaming append: K and V of 256 sequences x 8 heads, one token per
     step for 1024 steps into a preallocated [256, 1024, 8, P] cache, at every
-    head_dim x width. Per-step latency from events around each eager step
-    (two launches); the same 1024 steps are then captured once in a CUDA graph
-    and replayed, which removes the host launch cost."""
+    head_dim x width, written by two tq_encode_append calls per step and by
+    one tq_encode_append_kv call (`fused_` keys). Per-step latency from
+    events around each eager step; the same 1024 steps are then captured once
+    in a CUDA graph and replayed, which removes the host launch cost."""
     res = {}
     for d in (64, 128, 256):
         for b in BITS:
@@ -304,46 +305,54 @@ def _bench_append(K, W, torch, steps_per_run=1024):
             cn = {t: torch.empty(n_seq, s_max, H, dtype=torch.float32, device="cuda") for t in "KV"}
             slots = torch.arange(s_max, dtype=torch.int32, device="cuda")[:, None].expand(s_max, n_seq).contiguous()
 
-            def one(s):
+            def two(s):  # K and V with one tq_encode_append each
                 for t in "KV":
                     K.tq_encode_append(c.ctx, toks[s], n_seq, H, cache[t], cn[t], s_max, slots[s])
 
-            for s in range(8):
-                one(s)
-            torch.cuda.synchronize()
-            evs = [(_ev(torch), _ev(torch)) for _ in range(steps_per_run)]
-            for s, (e0, e1) in enumerate(evs):
-                e0.record()
-                one(s)
-                e1.record()
-            torch.cuda.synchronize()
-            ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
-            total = sum(ms) / 1e3
+            def fused(s):  # K and V in one tq_encode_append_kv launch
+                K.tq_encode_append_kv(c.ctx, toks[s], toks[s], n_seq, H, cache["K"], cn["K"], cache["V"], cn["V"],
+                                      s_max, slots[s])
+
             byts = steps_per_run * 2 * n_seq * H * (2 * d + P + 4)
-            # the whole stream of steps as one CUDA graph (every launch was
-            # made once above, so its one-time set-up is done)
-            g_stream = torch.cuda.Stream()
-            g_stream.wait_stream(torch.cuda.current_stream())
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(g_stream):
-                with torch.cuda.graph(graph, stream=g_stream):
-                    for s in range(steps_per_run):
-                        one(s)
-            torch.cuda.current_stream().wait_stream(g_stream)
-            graph.replay()
-            torch.cuda.synchronize()
-            g0, g1 = _ev(torch), _ev(torch)
-            g0.record()
-            graph.replay()
-            g1.record()
-            torch.cuda.synchronize()
-            g_total = g0.elapsed_time(g1) / 1e3
-            res[f"d{d}_b{b}"] = {"p50_us": ms[len(ms) // 2] * 1e3, "p99_us": ms[int(len(ms) * 0.99) - 1] * 1e3,
-                                 "GBps": byts / total / 1e9,
-                                 "graph_us_per_step": g_total / steps_per_run * 1e6,
-                                 "graph_GBps": byts / g_total / 1e9}
-            del graph, cache, cn, toks
-    res["launches_per_step"] = 2
+            row = {}
+            for name, one in (("", two), ("fused_", fused)):
+                for s in range(8):
+                    one(s)
+                torch.cuda.synchronize()
+                evs = [(_ev(torch), _ev(torch)) for _ in range(steps_per_run)]
+                for s, (e0, e1) in enumerate(evs):
+                    e0.record()
+                    one(s)
+                    e1.record()
+                torch.cuda.synchronize()
+                ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+                total = sum(ms) / 1e3
+                # the whole stream of steps as one CUDA graph (every launch
+                # was made once above, so its one-time set-up is done)
+                g_stream = torch.cuda.Stream()
+                g_stream.wait_stream(torch.cuda.current_stream())
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(g_stream):
+                    with torch.cuda.graph(graph, stream=g_stream):
+                        for s in range(steps_per_run):
+                            one(s)
+                torch.cuda.current_stream().wait_stream(g_stream)
+                graph.replay()
+                torch.cuda.synchronize()
+                g0, g1 = _ev(torch), _ev(torch)
+                g0.record()
+                graph.replay()
+                g1.record()
+                torch.cuda.synchronize()
+                g_total = g0.elapsed_time(g1) / 1e3
+                row.update({f"{name}p50_us": ms[len(ms) // 2] * 1e3, f"{name}p99_us": ms[int(len(ms) * 0.99) - 1] * 1e3,
+                            f"{name}GBps": byts / total / 1e9,
+                            f"{name}graph_us_per_step": g_total / steps_per_run * 1e6,
+                            f"{name}graph_GBps": byts / g_total / 1e9})
+                del graph
+            res[f"d{d}_b{b}"] = row
+            del cache, cn, toks
+    res["launches_per_step"] = {"two_calls": 2, "fused": 1}
     res["steps"] = steps_per_run
     return res
 

@@ -164,6 +164,23 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
                            float* cache_norms, int64_t s_max, const int32_t* slot, tq_stream stream);
 
 /*
+ * tq_encode_append for the key and the value of the new token of every
+ * sequence in one launch (an addition of this library: the "aither-kvcache"
+ * page's custom inference loop writes K and V at each step; a decode step of
+ * a few thousand rows is bound by launch latency, so one launch instead of
+ * two shortens the step). The result is that of
+ *   tq_encode_append(ctx, k_f16, n_seq, h, k_cache, k_norms, s_max, slot, stream);
+ *   tq_encode_append(ctx, v_f16, n_seq, h, v_cache, v_norms, s_max, slot, stream);
+ * with one context for both tensors (same head_dim, bits and seed); for two
+ * different codecs make the two calls. Arguments, layouts, alignment rules
+ * and errors as tq_encode_append, for each tensor; the two caches must not
+ * overlap. Asynchronous on `stream`.
+ */
+tq_status tq_encode_append_kv(const tq_ctx* ctx, const void* k_f16, const void* v_f16, int n_seq, int h,
+                              void* k_cache, float* k_norms, void* v_cache, float* v_norms, int64_t s_max,
+                              const int32_t* slot, tq_stream stream);
+
+/*
  * The offset + half-precision-scale variant ("TurboQuant efficient
  * inference", section "1. The quantizer": remove a small per-vector offset,
  * rotate, round each coordinate to a level, keep one scale alongside; codes

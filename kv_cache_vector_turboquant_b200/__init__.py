@@ -39,6 +39,7 @@ from ._binding import (  # noqa: F401
     tq_device_error,
     tq_encode,
     tq_encode_append,
+    tq_encode_append_kv,
     tq_encode_os,
     tq_decode_os,
     tq_encode_slots,
@@ -102,6 +103,14 @@ class TurboQuant:
         _require(d == self.head_dim, "last dim must be head_dim")
         s_max = cache_packed.shape[1]
         tq_encode_append(self.ctx, x, n_seq, h, cache_packed, cache_norms, s_max, slot, stream)
+
+    def encode_append_kv(self, k, v, k_cache, k_norms, v_cache, v_norms, slot, stream=None):
+        """Write the key and the value of one token per sequence in one launch:
+        k, v [n_seq, h, d] into slot[s] of their caches [n_seq, s_max, h, P]."""
+        n_seq, h, d = k.shape
+        _require(d == self.head_dim and tuple(v.shape) == tuple(k.shape), "k, v: [n_seq, h, head_dim]")
+        s_max = k_cache.shape[1]
+        tq_encode_append_kv(self.ctx, k, v, n_seq, h, k_cache, k_norms, v_cache, v_norms, s_max, slot, stream)
 
     def encode_os(self, x, stream=None):
         """Offset + fp16-scale variant: x [..., d] fp16 -> (packed [..., P]

@@ -36,6 +36,7 @@ _PROTOS = {
     "tq_decode": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_append": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_slots": (_c_int, [_vp, _vp, _c_i64, _c_int, _vp, _vp, _c_i64, _vp, _vp]),
+    "tq_encode_append_kv": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_encode_os": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _vp]),
     "tq_decode_os": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _vp]),
     "tq_attend_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_i64]),
@@ -198,6 +199,13 @@ def tq_encode_append(ctx: Ctx, x, n_seq: int, h: int, cache_packed, cache_norms,
                      stream=None) -> None:
     _check(_lib.tq_encode_append(ctx.handle, _ptr(x), int(n_seq), int(h), _ptr(cache_packed), _ptr(cache_norms),
                                  int(s_max), _ptr(slot), _stream(stream)), "tq_encode_append")
+
+
+def tq_encode_append_kv(ctx: Ctx, k, v, n_seq: int, h: int, k_cache, k_norms, v_cache, v_norms, s_max: int, slot,
+                        stream=None) -> None:
+    _check(_lib.tq_encode_append_kv(ctx.handle, _ptr(k), _ptr(v), int(n_seq), int(h), _ptr(k_cache), _ptr(k_norms),
+                                    _ptr(v_cache), _ptr(v_norms), int(s_max), _ptr(slot), _stream(stream)),
+           "tq_encode_append_kv")
 
 
 def tq_encode_os(ctx: Ctx, x, n: int, packed, side, stream=None) -> None:

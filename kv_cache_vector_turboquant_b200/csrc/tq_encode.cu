@@ -64,6 +64,13 @@ struct EncCfg {
 
 struct EncArgs {
   CUtensorMap tm_x;  // input as [n * lanes-per-vector rows, C] fp16, box 64 x 32, 128-byte swizzle
+  // two = 1: a second tensor of n vectors in the same launch (append mode,
+  // K and V of one step): the tiles after the first tensor's read tm_x2 and
+  // write packed2 / norms2
+  CUtensorMap tm_x2;
+  uint8_t* packed2;
+  float* norms2;
+  int two;
   int64_t n;         // vectors
   int64_t vec_base;  // index of vector 0 of this launch in the caller's tensor (append mode)
   uint8_t* packed;
@@ -298,7 +305,8 @@ __global__ void __launch_bounds__(W * 32, 1)
 
   // a launch covers fewer than 2^30 lane-rows: tile and row indices fit in int32
   const int n_rows = (int)(a.n * LPV);
-  const int n_tiles = (n_rows + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
+  const int n_tiles1 = (n_rows + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;  // tiles per tensor
+  const int n_tiles = a.two ? 2 * n_tiles1 : n_tiles1;
   // warps numbered SM-minor, so a partial last round of tiles spreads over all SMs
   const int gw = warp * (int)gridDim.x + (int)blockIdx.x;
   const int n_warps = (int)gridDim.x * WARPS;
@@ -307,11 +315,14 @@ __global__ void __launch_bounds__(W * 32, 1)
     if (lane == 0) {
       const uint32_t bar = smem_u32(&bars[stage]);
       mbar_arrive_expect_tx(bar, (uint32_t)Cfg::STAGE);  // full boxes: rows past the end are zero-filled
+      const bool second = tile >= n_tiles1;
+      const CUtensorMap* tm = second ? &a.tm_x2 : &a.tm_x;
+      const int lt = second ? tile - n_tiles1 : tile;
       if (!a.fault_inject) {
 #pragma unroll
         for (int b = 0; b < Cfg::BOXES; ++b)
-          tma_load_2d(stage0 + (uint32_t)(stage * Cfg::STAGE + b * ENC_BOX_BYTES), &a.tm_x, b * ENC_BOX_COLS,
-                      tile * ENC_BOX_ROWS, bar);
+          tma_load_2d(stage0 + (uint32_t)(stage * Cfg::STAGE + b * ENC_BOX_BYTES), tm, b * ENC_BOX_COLS,
+                      lt * ENC_BOX_ROWS, bar);
       }
     }
     __syncwarp();
@@ -331,7 +342,8 @@ __global__ void __launch_bounds__(W * 32, 1)
   int stage = 0;
   uint32_t parity = 0;  // bit s: parity of the next completion of stage s
   for (int tile = gw; tile < n_tiles; tile += n_warps) {
-    const int r0 = tile * ENC_BOX_ROWS;  // first lane-row of the tile
+    const bool second = tile >= n_tiles1;  // a tile of the second tensor
+    const int r0 = (second ? tile - n_tiles1 : tile) * ENC_BOX_ROWS;  // first lane-row of the tile
     const int valid_rows = min(ENC_BOX_ROWS, n_rows - r0);
     // every lane polls; the warp acts on one agreed outcome
     const bool ok = __all_sync(FULL, mbar_wait_bounded(smem_u32(&bars[stage]), (parity >> stage) & 1u, a.wait_limit));
@@ -532,10 +544,10 @@ __global__ void __launch_bounds__(W * 32, 1)
       const int32_t s = a.slot[seq];
       if (s >= 0 && s < a.s_max) {
         const int64_t drow = (a.slot_abs ? (int64_t)s : seq * a.s_max + s) * a.h + head;
-        uint8_t* dst = a.packed + drow * Cfg::P + part * Cfg::PL;
+        uint8_t* dst = (second ? a.packed2 : a.packed) + drow * Cfg::P + part * Cfg::PL;
 #pragma unroll
         for (int w = 0; w < WL; w += 2) *reinterpret_cast<uint2*>(dst + 4 * w) = make_uint2(words[w], words[w + 1]);
-        if (part == 0) a.norms[drow] = nrm;
+        if (part == 0) (second ? a.norms2 : a.norms)[drow] = nrm;
       } else if (part == 0 && !(a.slot_abs && s < 0)) {
         record_error(a.err, TQ_DEVERR_SLOT_RANGE);
       }
@@ -568,7 +580,8 @@ static cudaError_t configure_encode(size_t smem, int dev) {
 
 // OS: the offset + fp16-scale variant (bulk launches only, 16 warps).
 template <int D, int BITS, bool OS>
-static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const void* x, cudaStream_t st) {
+static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const void* x, cudaStream_t st,
+                                   const void* x2 = nullptr) {
   using Cfg = EncCfg<D, BITS>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -583,6 +596,7 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
   // launches of at most 2^30 lane-rows keep the copy coordinates in int32
   const int64_t max_vec = ((int64_t)1 << 30) / Cfg::LPV;
   const int64_t n_total = a.n;
+  if (x2 && n_total > max_vec / 2) return cudaErrorNotSupported;  // two tensors: one launch of int32 rows
   uint8_t* packed0 = a.packed;
   float* norms0 = a.norms;
   uint32_t* side0 = a.side;
@@ -606,7 +620,11 @@ static cudaError_t launch_encode_t(const tq_codec_tables& T, EncArgs a, const vo
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorNotSupported;
-    const int64_t tiles = (n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS;
+    if (x2 && enc(&a.tm_x2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x2), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+    const int64_t tiles = (x2 ? 2 : 1) * ((n * Cfg::LPV + ENC_BOX_ROWS - 1) / ENC_BOX_ROWS);
     if (!OS && tiles <= (int64_t)ENC_WARPS_SMALL * sms) {
       const int grid = (int)((tiles + ENC_WARPS_SMALL - 1) / ENC_WARPS_SMALL);
       e = tq_launch_pdl(encode_kernel<D, BITS, ENC_WARPS_SMALL, false>, dim3(grid), dim3(ENC_WARPS_SMALL * 32),
@@ -652,6 +670,37 @@ tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* pa
   TQ_ENC_CASE(128, 2) TQ_ENC_CASE(128, 3) TQ_ENC_CASE(128, 4)
   TQ_ENC_CASE(256, 2) TQ_ENC_CASE(256, 3) TQ_ENC_CASE(256, 4)
 #undef TQ_ENC_CASE
+  return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+tq_status tq_launch_encode_append2(const tq_ctx* ctx, const void* xk, const void* xv, int64_t n, void* k_packed,
+                                  float* k_norms, void* v_packed, float* v_norms, const int32_t* slot, int h,
+                                  int64_t s_max, void* stream) {
+  if (n == 0) return TQ_OK;
+  EncArgs a;
+  memset(&a, 0, sizeof(a));
+  a.n = n;
+  a.packed = static_cast<uint8_t*>(k_packed);
+  a.norms = k_norms;
+  a.packed2 = static_cast<uint8_t*>(v_packed);
+  a.norms2 = v_norms;
+  a.two = 1;
+  a.slot = slot;
+  a.h = h;
+  a.s_max = s_max;
+  a.err = tq_error_word();
+  if (!a.err) return TQ_ERR_CUDA;
+  a.wait_limit = TQ_WAIT_LIMIT_CYCLES;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+  const tq_codec_tables& T = ctx->t;
+#define TQ_ENC_CASE(D_, B_) \
+  if (ctx->d == D_ && ctx->bits == B_) e = launch_encode_t<D_, B_, false>(T, a, xk, st, xv);
+  TQ_ENC_CASE(64, 2) TQ_ENC_CASE(64, 3) TQ_ENC_CASE(64, 4)
+  TQ_ENC_CASE(128, 2) TQ_ENC_CASE(128, 3) TQ_ENC_CASE(128, 4)
+  TQ_ENC_CASE(256, 2) TQ_ENC_CASE(256, 3) TQ_ENC_CASE(256, 4)
+#undef TQ_ENC_CASE
+  if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
   return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 

@@ -237,6 +237,24 @@ tq_status tq_encode_append(const tq_ctx* ctx, const void* x_f16, int n_seq, int 
   return tq_launch_encode(ctx, x_f16, (int64_t)n_seq * h, cache_packed, cache_norms, slot, h, s_max, stream, 0);
 }
 
+tq_status tq_encode_append_kv(const tq_ctx* ctx, const void* k_f16, const void* v_f16, int n_seq, int h,
+                              void* k_cache, float* k_norms, void* v_cache, float* v_norms, int64_t s_max,
+                              const int32_t* slot, tq_stream stream) {
+  if (!ctx || n_seq < 0 || h <= 0 || s_max <= 0) return TQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TQ_OK;
+  if (!k_f16 || !v_f16 || !k_cache || !k_norms || !v_cache || !v_norms || !slot) return TQ_ERR_INVALID_ARG;
+  if (!aligned(k_f16, 16) || !aligned(v_f16, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(k_norms, 4) || !aligned(v_norms, 4) || !aligned(slot, 4))
+    return TQ_ERR_ALIGNMENT;
+  const int64_t n = (int64_t)n_seq * h;
+  const tq_status st =
+      tq_launch_encode_append2(ctx, k_f16, v_f16, n, k_cache, k_norms, v_cache, v_norms, slot, h, s_max, stream);
+  if (st != TQ_ERR_UNSUPPORTED) return st;
+  const tq_status sk = tq_launch_encode(ctx, k_f16, n, k_cache, k_norms, slot, h, s_max, stream, 0);
+  if (sk != TQ_OK) return sk;
+  return tq_launch_encode(ctx, v_f16, n, v_cache, v_norms, slot, h, s_max, stream, 0);
+}
+
 tq_status tq_encode_os(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packed, uint32_t* side,
                        tq_stream stream) {
   if (!ctx || n < 0) return TQ_ERR_INVALID_ARG;

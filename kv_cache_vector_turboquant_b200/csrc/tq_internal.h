@@ -65,6 +65,13 @@ inline double tq_guard_z(int head_dim) { return head_dim <= 128 ? 1.0e-5 : 2.0e-
 tq_status tq_launch_encode(const tq_ctx* ctx, const void* x, int64_t n, void* packed, float* norms,
                            const int32_t* slot, int h, int64_t s_max, void* stream, int fault_inject,
                            int slot_abs = 0);
+// Append of the K and V tensors of one step in one launch (tq_encode.cu):
+// the same rows and caches as two tq_launch_encode append calls with the
+// same context. TQ_ERR_UNSUPPORTED (nothing launched) when n is too large for
+// one launch; the caller then makes the two calls.
+tq_status tq_launch_encode_append2(const tq_ctx* ctx, const void* xk, const void* xv, int64_t n, void* k_packed,
+                                  float* k_norms, void* v_packed, float* v_norms, const int32_t* slot, int h,
+                                  int64_t s_max, void* stream);
 // Bulk encode on the tensor cores (tq_encode_tc.cu): the same outputs as
 // tq_launch_encode without append slots. tq_encode uses it from
 // tq_encode_tc_min_rows() vectors on (one 128-vector tile per SM).

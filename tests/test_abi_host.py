@@ -180,6 +180,26 @@ def test_append_validation(K):
     assert _raw(K, "tq_encode_append", h, A, 4, 8, B_, C, 16, S + 2, None) == K.TQ_ERR_ALIGNMENT
 
 
+def test_append_kv_validation(K):
+    ctx = K.tq_create(128, 3)
+    h = ctx.handle
+    A, A2, B_, C, B2, C2, S = 0x10000, 0x18000, 0x20000, 0x30000, 0x50000, 0x60000, 0x40000
+    f = "tq_encode_append_kv"
+    assert _raw(K, f, None, A, A2, 4, 8, B_, C, B2, C2, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 4, 0, B_, C, B2, C2, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2, C2, 0, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, -1, 8, B_, C, B2, C2, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 0, 8, B_, C, B2, C2, 16, S, None) == K.TQ_OK  # nothing to do
+    assert _raw(K, f, h, A, None, 4, 8, B_, C, B2, C2, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, None, C2, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2, None, 16, S, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2, C2, 16, None, None) == K.TQ_ERR_INVALID_ARG
+    assert _raw(K, f, h, A, A2 + 8, 4, 8, B_, C, B2, C2, 16, S, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2 + 4, C2, 16, S, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2, C2 + 2, 16, S, None) == K.TQ_ERR_ALIGNMENT
+    assert _raw(K, f, h, A, A2, 4, 8, B_, C, B2, C2, 16, S + 2, None) == K.TQ_ERR_ALIGNMENT
+
+
 def test_attend_validation_and_workspace(K):
     k4, v2 = K.tq_create(128, 4), K.tq_create(128, 2)
     k64 = K.tq_create(64, 4)

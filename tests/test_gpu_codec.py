@@ -200,6 +200,61 @@ def test_append_replayed_from_cuda_graph(K, W, d):
 
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("bits", [2, 3, 4])
+def test_append_kv_equals_two_appends(K, W, d, bits):
+    """The key and value append of one launch writes exactly what two
+    tq_encode_append calls write (ragged head count, a slot out of range
+    skipped and flagged), and the same steps replayed from a CUDA graph give
+    the same bytes again."""
+    n_seq, h, s_max, steps = 37, 3, 8, 4
+    tq = K.TurboQuant(d, bits)
+    P = tq.packed_bytes
+    ks = W.append_stream(run=50 + d + bits, steps=steps, n_seq=n_seq, H=h, d=d)
+    vs = W.append_stream(run=60 + d + bits, steps=steps, n_seq=n_seq, H=h, d=d)
+    g = torch.Generator().manual_seed(d * 10 + bits)
+    slots = torch.randint(0, s_max, (steps, n_seq), generator=g, dtype=torch.int32).cuda()
+
+    def caches():
+        return [torch.full((n_seq, s_max, h, P), 0x3C, dtype=torch.uint8, device="cuda"),
+                torch.full((n_seq, s_max, h), -3.0, dtype=torch.float32, device="cuda"),
+                torch.full((n_seq, s_max, h, P), 0x5A, dtype=torch.uint8, device="cuda"),
+                torch.full((n_seq, s_max, h), -5.0, dtype=torch.float32, device="cuda")]
+
+    two, one, graphed = caches(), caches(), caches()
+    for s in range(steps):
+        tq.encode_append(ks[s], two[0], two[1], slots[s])
+        tq.encode_append(vs[s], two[2], two[3], slots[s])
+        tq.encode_append_kv(ks[s], vs[s], one[0], one[1], one[2], one[3], slots[s])
+    torch.cuda.synchronize()
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+    for a, b in zip(one, two):
+        assert torch.equal(a, b)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            for s in range(steps):
+                tq.encode_append_kv(ks[s], vs[s], graphed[0], graphed[1], graphed[2], graphed[3], slots[s])
+    torch.cuda.current_stream().wait_stream(stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(graphed, two):
+        assert torch.equal(a, b)
+    del graph
+    # a slot past the cache is skipped (both tensors) and flagged
+    bad = slots[0].clone()
+    bad[5] = s_max
+    before = [t.clone() for t in one]
+    tq.encode_append_kv(ks[0], vs[0], one[0], one[1], one[2], one[3], bad)
+    torch.cuda.synchronize()
+    st, bits_ = K.tq_device_error()
+    assert st == K.TQ_ERR_DEVICE and bits_ == K.TQ_DEVERR_SLOT_RANGE
+    for a, b in zip(one, before):
+        assert torch.equal(a[5], b[5])
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_append_matches_bulk_encode(K, W, d, bits):
     """Streaming append of 6 steps x 256 sequences x 8 heads into a 16-slot
     cache: written slots are bit-identical to a bulk encode of the same rows,
