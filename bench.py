@@ -760,7 +760,7 @@ def _front(result: dict) -> dict:
     return out
 
 
-def _e2e(K, torch, S, steps, world, dist, chunk_rows=65536, n_streams=4):
+def _e2e(K, torch, S, steps, world, dist, chunk_rows=131072, n_streams=8):
     """End to end through the public API: every step copies each tensor's
     fp16 rows from pinned host memory, encodes, copies codes and norms back,
     copies them to the device again, decodes and copies the fp16 rows back,
