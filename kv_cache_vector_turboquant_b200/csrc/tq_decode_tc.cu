@@ -22,8 +22,8 @@
 //  * warp 0: 1-D bulk copies of each full tile's packed rows into a ring of
 //    shared-memory stages (a partial last tile is read with plain loads);
 //  * warps 2-9 (two builder warpgroups taking alternate tiles, one row per
-//    thread): each pair of codes indexes a
-//    lane-replicated table of {value pair, remainder pair} as packed fp16,
+//    thread): each pair of codes (each code byte at 2 bits) indexes a
+//    lane-replicated table of value pairs and remainder pairs (packed fp16),
 //    which go straight into tensor memory with tcgen05.st (A operand: row m
 //    in lane m, two fp16 per 32-bit column, 8 columns per 16-element K-step);
 //  * warp 1: per tile 2 d/16 MMAs with A from tensor memory ([a-tmem] form)
@@ -60,7 +60,10 @@ struct DtCfg {
   static constexpr int P = D * BITS / 8;            // packed bytes per vector
   static constexpr int WORDS = P / 4;
   static constexpr int TILE_P = DT_ROWS * P;        // packed bytes of a full tile
-  static constexpr int E = 1 << (2 * BITS);         // pair-table entries
+  // 2 bits: one table entry per code byte (four codes, two A columns);
+  // otherwise one per pair of codes (one A column)
+  static constexpr bool QUAD = BITS == 2;
+  static constexpr int E = QUAD ? 256 : 1 << (2 * BITS);  // table entries
   // tensor memory: NA A operands (values d/2 + remainders d/2 columns each),
   // then one accumulator (d columns) per epilogue warpgroup
   static constexpr int NA = 2;
@@ -71,8 +74,8 @@ struct DtCfg {
   static constexpr int OUT_BYTES = BOXES * DT_ROWS * 128;
   static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_d: BOXES atoms of d rows x 128 B
   static constexpr int IN = BREG + D * D * 2;       // STAGES x TILE_P
-  static constexpr int LUT = IN + STAGES * TILE_P;  // E x 32 lane copies x 8 B
-  static constexpr int BAR = LUT + E * 32 * 8;
+  static constexpr int LUT = IN + STAGES * TILE_P;  // E entries of 256 B (lane copies of values, remainders)
+  static constexpr int BAR = LUT + E * 256;
   // full[S], empty[S], aready[NA][2], aempty[NA][2], tfull[2], tempty[2], done
   static constexpr int NBARS = 2 * STAGES + 4 * NA + 4 + 1;
   static constexpr int SLOT = BAR + NBARS * 8;
@@ -91,6 +94,12 @@ struct DtArgs {
 TQ_DEV uint2 dt_lds_u2(uint32_t addr) {
   uint2 r;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+TQ_DEV uint32_t dt_lds_u32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
   return r;
 }
 
@@ -179,31 +188,63 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
   // The tables are filled after this point, so the first copies are in
   // flight meanwhile.
 
-  // ---- pair table, built by warps 2-17 (the epilogue warps have nothing to
-  // do before the first accumulator): entry (f, lane), f = code_a | code_b <<
-  // BITS, holds the A-operand columns {value_a | value_b << 16, remainder_a |
-  // remainder_b << 16} (fp16; value + remainder = level exactly: a
-  // 2^-14-grid level below 4 has at most 16 significant bits, its fp16
-  // remainder is a multiple of 2^-14 below 2^-9). Each thread computes one
-  // entry and writes its copies for 32 / (512 / E) lanes, two lanes per
-  // 16-byte store, the stores rotated so a warp's stores spread over banks.
+  // ---- code table, built by warps 2-17 (the epilogue warps have nothing to
+  // do before the first accumulator). At 3 and 4 bits entry f = code_a |
+  // code_b << BITS is 256 bytes: the A-operand column value_a | value_b << 16
+  // for each of the 32 lanes, then the column remainder_a | remainder_b << 16
+  // for each lane (fp16; value + remainder = level exactly: a 2^-14-grid
+  // level below 4 has at most 16 significant bits, its fp16 remainder is a
+  // multiple of 2^-14 below 2^-9). A lookup is two 4-byte loads (one
+  // wavefront each, no bank conflict), so each word lands in the register
+  // that its tensor-memory store reads, with no register moves between the
+  // loads and the stores. At 2 bits an entry covers a whole code byte (two
+  // columns) and a lookup is two 8-byte loads. Each thread computes one
+  // entry and writes its share of the lane copies with 16-byte stores,
+  // rotated so a warp's stores spread over banks.
   if (warp >= 2) {
     constexpr int E = Cfg::E, PER = 512 / E, LANES = 32 / PER;
     static_assert(E <= 512 && 512 % E == 0 && PER * LANES == 32, "one thread per entry and lane group");
     const int t = tid - 64, f = t / PER, part = t % PER;
-    const float ca = T.levels[f & ((1 << BITS) - 1)], cb = T.levels[f >> BITS];
-    const __half va = __float2half_rn(ca), vb = __float2half_rn(cb);
-    const __half ra = __float2half_rn(ca - __half2float(va)), rb = __float2half_rn(cb - __half2float(vb));
-    const uint32_t ev = (uint32_t)__half_as_ushort(va) | ((uint32_t)__half_as_ushort(vb) << 16);
-    const uint32_t er = (uint32_t)__half_as_ushort(ra) | ((uint32_t)__half_as_ushort(rb) << 16);
-    uint8_t* row = sm + Cfg::LUT + f * 256 + part * LANES * 8;
-    if constexpr (LANES == 1) {
-      *reinterpret_cast<uint2*>(row) = make_uint2(ev, er);
-    } else {
+    // the value word and the remainder word of the pair of codes pc
+    auto pair_words = [&](int pc, uint32_t& ev, uint32_t& er) {
+      const float ca = T.levels[pc & ((1 << BITS) - 1)], cb = T.levels[pc >> BITS];
+      const __half va = __float2half_rn(ca), vb = __float2half_rn(cb);
+      const __half ra = __float2half_rn(ca - __half2float(va)), rb = __float2half_rn(cb - __half2float(vb));
+      ev = (uint32_t)__half_as_ushort(va) | ((uint32_t)__half_as_ushort(vb) << 16);
+      er = (uint32_t)__half_as_ushort(ra) | ((uint32_t)__half_as_ushort(rb) << 16);
+    };
+    if constexpr (Cfg::QUAD) {
+      // entry f = a code byte (pairs f & 15, f >> 4): 16 lane copies of its
+      // two value words, then 16 of its two remainder words (8 bytes each;
+      // an 8-byte load is served per half-warp, so 16 copies are enough for
+      // conflict-free lookups); each of the two threads of an entry writes 8
+      uint32_t ev0, er0, ev1, er1;
+      pair_words(f & 15, ev0, er0);
+      pair_words(f >> 4, ev1, er1);
+      uint8_t* row = sm + Cfg::LUT + f * 256 + part * 64;
 #pragma unroll
-      for (int j = 0; j < LANES / 2; ++j) {
-        const int jj = (j + t) % (LANES / 2);
-        *reinterpret_cast<uint4*>(row + jj * 16) = make_uint4(ev, er, ev, er);
+      for (int j = 0; j < 4; ++j) {
+        const int jj = (j + t) & 3;
+        *reinterpret_cast<uint4*>(row + jj * 16) = make_uint4(ev0, ev1, ev0, ev1);
+        *reinterpret_cast<uint4*>(row + 128 + jj * 16) = make_uint4(er0, er1, er0, er1);
+      }
+    } else {
+      uint32_t ev, er;
+      pair_words(f, ev, er);
+      uint8_t* row = sm + Cfg::LUT + f * 256 + part * LANES * 4;
+      if constexpr (LANES < 4) {
+#pragma unroll
+        for (int j = 0; j < LANES; ++j) {
+          reinterpret_cast<uint32_t*>(row)[j] = ev;
+          reinterpret_cast<uint32_t*>(row + 128)[j] = er;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < LANES / 4; ++j) {
+          const int jj = (j + t) % (LANES / 4);
+          *reinterpret_cast<uint4*>(row + jj * 16) = make_uint4(ev, ev, ev, ev);
+          *reinterpret_cast<uint4*>(row + 128 + jj * 16) = make_uint4(er, er, er, er);
+        }
       }
     }
     // B = H_d (natural order, +-1; the signs are applied to the fp16 output)
@@ -279,7 +320,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     // ... into A operand bg; one row per thread (tensor-memory lane = tile row)
     const int bg = (warp - 2) >> 2, quarter = warp & 3, r = 32 * quarter + lane;
     const uint32_t lanebase = (uint32_t)(32 * quarter) << 16;
-    const uint32_t lut_lane = base + Cfg::LUT + (uint32_t)lane * 8u;
+    const uint32_t lut_lane = base + Cfg::LUT + (Cfg::QUAD ? (uint32_t)(lane & 15) * 8u : (uint32_t)lane * 4u);
     grid_dep_wait();  // a partial tile's rows are read from global memory
     bool alive = true;
     for (int i = bg; i < cnt && alive; i += 2) {
@@ -329,16 +370,35 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
 #pragma unroll
         for (int c0 = h * D / 4; c0 < (h + 1) * D / 4; c0 += 16) {
           uint32_t vv[16], rr[16];
+          if constexpr (Cfg::QUAD) {
+            // code byte c0 / 2 + j -> columns c0 + 2j, c0 + 2j + 1, by two
+            // 8-byte loads (values, remainders) into consecutive registers
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            constexpr int FB = 2 * BITS;
-            const int off = (c0 + t) * FB;
-            uint32_t f = words[off >> 5] >> (off & 31);
-            if ((off & 31) + FB > 32) f |= words[(off >> 5) + 1] << (32 - (off & 31));
-            f &= (uint32_t)(Cfg::E - 1);
-            const uint2 ent = dt_lds_u2(f * 256u + lut_lane);
-            vv[t] = ent.x;
-            rr[t] = ent.y;
+            for (int j = 0; j < 8; ++j) {
+              const int byte = c0 / 2 + j;
+              const uint32_t f = __byte_perm(words[byte >> 2], 0u, 0x4440u | (uint32_t)(byte & 3));
+              const uint2 v2 = dt_lds_u2(f * 256u + lut_lane), r2 = dt_lds_u2(f * 256u + lut_lane + 128u);
+              vv[2 * j] = v2.x, vv[2 * j + 1] = v2.y;
+              rr[2 * j] = r2.x, rr[2 * j + 1] = r2.y;
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              constexpr int FB = 2 * BITS;
+              const int off = (c0 + t) * FB;
+              uint32_t f;
+              if constexpr (FB == 8) {  // a pair is a byte
+                f = __byte_perm(words[off >> 5], 0u, 0x4440u | (uint32_t)((off >> 3) & 3));
+              } else {
+                f = words[off >> 5] >> (off & 31);
+                if ((off & 31) + FB > 32) f |= words[(off >> 5) + 1] << (32 - (off & 31));
+                f &= (uint32_t)(Cfg::E - 1);
+              }
+              // the value pair and the remainder pair by two 4-byte loads, so
+              // each lands in the register its tensor-memory store reads
+              vv[t] = dt_lds_u32(f * 256u + lut_lane);
+              rr[t] = dt_lds_u32(f * 256u + lut_lane + 128u);
+            }
           }
           tmem_st16(sb + (uint32_t)c0, vv);
           tmem_st16(sb + (uint32_t)(D / 2 + c0), rr);

@@ -140,6 +140,39 @@ def test_llama_layer_full_size_sampled(K, W, bits):
     assert K.tq_device_error()[0] == K.TQ_OK
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_kv_in_one_buffer_equals_per_tensor_calls(K, W, bits):
+    """The benchmarked step keeps the layer's K and V in one [2, n, 128]
+    buffer and encodes (decodes) both with one call of 2n rows. Rows are
+    independent, so codes, norms and decoded rows must be the bytes of one
+    call per tensor; rows on both sides of the K/V seam and a random sample
+    are also checked against the oracle."""
+    k, v = W.llama_layer(device="cuda")
+    n = k.numel() // 128
+    kv = torch.stack([k.reshape(n, 128), v.reshape(n, 128)])
+    del k, v
+    tq = K.TurboQuant(128, bits)
+    packed, norms = tq.encode(kv.reshape(2 * n, 128))
+    dec = tq.decode(packed, norms)
+    for t in range(2):
+        p1, n1 = tq.encode(kv[t])
+        d1 = tq.decode(p1, n1)
+        torch.cuda.synchronize()
+        assert torch.equal(packed[t * n:(t + 1) * n], p1)
+        assert torch.equal(norms[t * n:(t + 1) * n], n1)
+        assert torch.equal(dec[t * n:(t + 1) * n], d1)
+        del p1, n1, d1
+    g = torch.Generator().manual_seed(90 + bits)
+    rows = torch.cat([torch.arange(n - 256, n + 256), torch.randint(0, 2 * n, (4096,), generator=g)]).unique()
+    xs = kv.reshape(2 * n, 128)[rows.cuda()].cpu().numpy()
+    det = O.encode_detail(xs, bits, 42)
+    gp, gn = packed[rows.cuda()].cpu().numpy(), norms[rows.cuda()].cpu().numpy()
+    assert code_mismatches(gp, det, bits, 128) == 0
+    assert_norms(gn, det)
+    assert_decode_ulp(dec[rows.cuda()].cpu().numpy(), O.decode(gp, gn, bits, 42, 128))
+    assert K.tq_device_error()[0] == K.TQ_OK
+
+
 @pytest.mark.parametrize("layer", [0, 41, 79])
 def test_long_context_layer_sampled(K, W, layer):
     """Layers of the 80-layer long-context cache at 3 bits: K and V
