@@ -877,8 +877,9 @@ PROFILE_CASES = ["encode_b2", "encode_b3", "encode_b4", "decode_b2", "decode_b3"
 
 def run_profile_case(case: str, launches: int = 3):
     """A small, self-contained case for Nsight Compute: a few launches of one
-    kernel on the benchmark's shapes (the layer tensor is 128 MiB, larger than
-    L2; the decode-step cache is ~0.4 GB), after one warm-up launch."""
+    kernel on the benchmark's shapes (the layer's K and V, 256 MiB of fp16,
+    larger than L2; the decode-step cache is ~0.4 GB), after one warm-up
+    launch."""
     import torch
 
     import kv_cache_vector_turboquant_b200 as K
@@ -895,12 +896,12 @@ def run_profile_case(case: str, launches: int = 3):
         pos = torch.full((a["B"],), a["S"], dtype=torch.int32, device="cuda")
         for _ in range(1 + launches):
             K.attend_decode(q, kc, vc, kp, kn, vp, vn, pos)
-    else:
+    else:  # the benchmarked launch: the layer's K and V in one [2 n, D] buffer
         kind, b = case.split("_b")
         b = int(b)
-        _, v = W.llama_layer(device="cuda")
-        x = v.reshape(-1, D)
-        del _
+        k, v = W.llama_layer(device="cuda")
+        x = torch.cat([k.reshape(-1, D), v.reshape(-1, D)])
+        del k, v
         c = K.TurboQuant(D, b)
         p, n = c.encode(x)
         out = torch.empty_like(x)
