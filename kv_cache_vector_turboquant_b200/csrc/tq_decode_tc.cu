@@ -6,17 +6,28 @@
 // steps 4-1): x_hat = D (H_pm c[idx]) * (N / d), H_pm the +-1 natural-order
 // Walsh-Hadamard matrix, D the seeded sign flip, c the codebook levels.
 //
-// The whole transform runs on the tensor cores: per 128-vector tile,
-// Y = C H_pm^T with C the tile's levels (128 rows x d) and B = H_pm (d x d,
-// +-1), accumulated over the d/16 K-steps. The levels lie on the 2^-14 grid
-// (16 significant bits), so each level is split into an fp16 value and an
-// fp16 remainder (both exact) and both parts are multiplied (2 d/16 MMAs of
-// M = 128, N = d, K = 16 into one accumulator). Every product and every
+// Transform: H_d = H_{d/32} (x) H_32 (Sylvester), so coordinate 32 b' + j of
+// H_pm c is sum_b (-1)^popc(b' & b) S[b][j] with S[b] = H_32 c_b the 32-point
+// transform of block b. The tensor cores compute every S[b] of a 128-vector
+// tile (M = 128, N = 32, two K-steps of 16 per block); the remaining
+// log2(d/32) stages run as f32 butterflies in the epilogue. The levels lie on
+// the 2^-14 grid (16 significant bits), so each level is split into an fp16
+// value and an fp16 remainder (both exact) and both parts are multiplied
+// (four MMAs per block into its accumulator columns). Every product and every
 // partial sum is a multiple of 2^-14 below 2^9 (|H_pm c| <= d max|c| < 2^9),
-// so it is exact in f32, and the tensor core cuts addends only below
-// 2^(E-25) with E <= 9 and rounds an exact sum to itself: Y is exact. The
-// only roundings are the product by N / d and the fp16 conversion, as in
-// decode_kernel (outputs bit-identical).
+// so it is exact in f32: the tensor core cuts addends only below 2^(E-25)
+// with E <= 7 and rounds an exact sum to itself, and the f32 butterflies add
+// exact values whose sums are exact. The only roundings are the product by
+// N / d and the fp16 conversion, as in decode_kernel (outputs bit-identical).
+//
+// Why 32-point blocks and not the whole transform on the tensor cores: the
+// whole transform (N = d) is 8 times the tensor-core work of these blocks
+// (256 multiply-adds per coordinate at d = 128, about 1 PFLOP/s of fp16 at
+// the streaming rate) and ran the GPU into its power limit on its own (about
+// 1500 MHz); 32-point blocks cost one f32x2 add per coordinate more and keep
+// the clock near 1800 MHz, so a decode or the whole codec step is faster at
+// the power limit and no slower at full clock. 16-point blocks (three f32
+// stages) and 64-point blocks (one stage) measured slower.
 //
 // B200 mapping (one persistent CTA of 18 warps per SM, warp-specialised):
 //  * warp 0: 1-D bulk copies of each full tile's packed rows into a ring of
@@ -26,15 +37,16 @@
 //    lane-replicated table of value pairs and remainder pairs (packed fp16),
 //    which go straight into tensor memory with tcgen05.st (A operand: row m
 //    in lane m, two fp16 per 32-bit column, 8 columns per 16-element K-step);
-//  * warp 1: per tile 2 d/16 MMAs with A from tensor memory ([a-tmem] form)
-//    and B = H_pm (fp16 +-1, shared memory, built once per CTA), f32
-//    accumulators in tensor memory: two A operands (the builders refill a
-//    half as soon as the MMAs that read it commit) and one accumulator per
-//    epilogue warpgroup;
-//  * warps 10-17 (two epilogue warpgroups, one row per thread): the scale
-//    N / d, the fp16 conversion and the sign flip on fp16 pairs, staged in
-//    the group's 128-byte-swizzled tile and written by 2-D tensor stores
-//    (which clip a partial last tile).
+//  * warp 1: per tile 2 d/16 MMAs (M = 128, N = 32, K = 16) with A from
+//    tensor memory ([a-tmem] form) and B = H_32 (fp16 +-1, shared memory,
+//    built once per CTA), f32 accumulators in tensor memory: two A operands
+//    (the builders refill a half as soon as the MMAs that read it commit)
+//    and one accumulator per epilogue warpgroup;
+//  * warps 10-17 (two epilogue warpgroups, one row per thread): the
+//    remaining butterfly stages across the 32-point blocks, the scale N / d,
+//    the fp16 conversion and the sign flip on fp16 pairs, staged in the
+//    group's 128-byte-swizzled tile and written by 2-D tensor stores (which
+//    clip a partial last tile).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -55,7 +67,9 @@ constexpr size_t DT_SMEM_MAX = 232448;
 
 template <int D, int BITS>
 struct DtCfg {
-  static constexpr int NB = D / 16;                 // 16-point blocks per vector
+  static constexpr int NB = D / 16;                 // 16-element K-steps per vector
+  static constexpr int NB32 = D / 32;               // 32-point transform blocks per vector
+  static constexpr int JP = 32 / NB32;              // positions per epilogue chunk (all blocks: 32 values)
   static constexpr int BOXES = D / 64;              // 64-column store boxes per tile
   static constexpr int P = D * BITS / 8;            // packed bytes per vector
   static constexpr int WORDS = P / 4;
@@ -72,8 +86,8 @@ struct DtCfg {
   // shared memory, from a 1024-aligned base
   static constexpr int OUT = 0;                     // 2 groups x BOXES x [128 rows x 128 B]
   static constexpr int OUT_BYTES = BOXES * DT_ROWS * 128;
-  static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_d: BOXES atoms of d rows x 128 B
-  static constexpr int IN = BREG + D * D * 2;       // STAGES x TILE_P
+  static constexpr int BREG = OUT + 2 * OUT_BYTES;  // H_32: 32 rows x 128 B (k < 32 used)
+  static constexpr int IN = BREG + 32 * 128;        // STAGES x TILE_P
   static constexpr int LUT = IN + STAGES * TILE_P;  // E entries of 256 B (lane copies of values, remainders)
   static constexpr int BAR = LUT + E * 256;
   // full[S], empty[S], aready[NA][2], aempty[NA][2], tfull[2], tempty[2], done
@@ -247,13 +261,13 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
         }
       }
     }
-    // B = H_d (natural order, +-1; the signs are applied to the fp16 output)
-    // as an N = d by K = d operand, K-major with the 128-byte swizzle: atom
-    // k / 64 holds row n at n * 128 bytes, its 16-byte chunk c at c ^ (n % 8)
-    for (int e = t; e < D * D; e += 512) {
-      const int n = e / D, k = e % D;
-      const uint32_t off = Cfg::BREG + (k >> 6) * (D * 128) + n * 128 + (((((k & 63) * 2) >> 4) ^ (n & 7)) << 4) +
-                           ((k * 2) & 15);
+    // B = H_32 (natural order, +-1; the signs are applied to the fp16 output)
+    // as an N = 32 by K = 32 operand, K-major with the 128-byte swizzle: row n
+    // at n * 128 bytes, its 16-byte chunk c at c ^ (n % 8); K-step kh of a
+    // block reads elements 16 kh ... 16 kh + 15 (descriptor start + 32 kh bytes)
+    for (int e = t; e < 32 * 32; e += 512) {
+      const int n = e >> 5, k = e & 31;
+      const uint32_t off = Cfg::BREG + n * 128 + ((((k * 2) >> 4) ^ (n & 7)) << 4) + ((k * 2) & 15);
       *reinterpret_cast<uint16_t*>(sm + off) = (__popc(n & k) & 1) ? (uint16_t)0xBC00u : (uint16_t)0x3C00u;
     }
     fence_proxy_async_smem();  // B is read by the tensor cores
@@ -280,12 +294,13 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer: the whole transform, D = (A_value + A_remainder) H_d^T
-    // accumulated over the d/16 K-steps of both parts (exact: see the top)
+    // ---- MMA issuer: the 32-point block transforms S[b] = (A_value +
+    // A_remainder)_b H_32^T, each accumulated over its two K-steps of both
+    // parts (exact: see the top)
     asm volatile("bar.sync 3, 544;" ::: "memory");  // B (and the table) are built
     if (lane == 0) {
       grid_dep_wait();  // (its only global access is the error word)
-      constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, D);
+      constexpr uint32_t IDESC = umma_idesc_f16(DT_ROWS, 32);
       bool ok = true;
       for (int i = 0; i < cnt && ok; ++i) {
         const int k = i % NA, g = i & 1;
@@ -302,11 +317,13 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
           }
           tc_fence_after();
 #pragma unroll
-          for (int b = h * NB / 2; b < (h + 1) * NB / 2; ++b) {
-            // K-step b: coordinates 16 b ... 16 b + 15 of the levels
-            const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG + (b >> 2) * (D * 128) + (b & 3) * 32);
-            umma_f16_ts(db, ab + (uint32_t)(8 * b), bdesc, IDESC, b > 0);
-            umma_f16_ts(db, ab + (uint32_t)(D / 2 + 8 * b), bdesc, IDESC, true);
+          for (int ks = h * NB / 2; ks < (h + 1) * NB / 2; ++ks) {
+            // K-step ks: coordinates 16 ks ... 16 ks + 15 of the levels, half
+            // ks % 2 of 32-point block ks / 2, whose S goes to columns 32 (ks / 2) ...
+            const uint64_t bdesc = umma_desc_sw128(base + Cfg::BREG + 32 * (ks & 1));
+            const uint32_t dcol = db + (uint32_t)(32 * (ks >> 1));
+            umma_f16_ts(dcol, ab + (uint32_t)(8 * ks), bdesc, IDESC, (ks & 1) != 0);
+            umma_f16_ts(dcol, ab + (uint32_t)(D / 2 + 8 * ks), bdesc, IDESC, true);
           }
           umma_commit(aempty0 + 8u * (2 * k + h));  // this half may be rewritten
         }
@@ -445,37 +462,54 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       if (leader && stored_once) bulk_wait_read<0>();
       asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
       const uint32_t tl = tmem + lanebase + (uint32_t)(Cfg::ACC0 + g * D);
-      // column n of the accumulator is coordinate n of H_pm c: 32 columns per
-      // tensor-memory wait, 16 coordinates per pair of 16-byte staging stores
+      // column 32 b + j of the accumulator is S[b][j]; per tensor-memory wait
+      // positions JP c ... JP c + JP - 1 of every block (32 values), then the
+      // log2(d / 32) remaining stages of the transform across the blocks in
+      // f32 pairs, which gives coordinates 32 b' + JP c ... of H_pm c
+      constexpr int NB32 = Cfg::NB32, JP = Cfg::JP;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rv[2][16];
-        tmem_ld16(tl + (uint32_t)(32 * c), rv[0]);
-        tmem_ld16(tl + (uint32_t)(32 * c + 16), rv[1]);
+      for (int c = 0; c < 32 / JP; ++c) {
+        uint32_t rv[NB32][JP];
+#pragma unroll
+        for (int b = 0; b < NB32; ++b) {
+          if constexpr (JP == 8)
+            tmem_ld8(tl + (uint32_t)(32 * b + JP * c), rv[b]);
+          else
+            tmem_ld16(tl + (uint32_t)(32 * b + JP * c), rv[b]);
+        }
         tmem_wait_ld();
-        tmem_regs_after_wait(rv[0]);
-        tmem_regs_after_wait(rv[1]);
-        if (c == D / 32 - 1) {  // every load of the accumulator is done: free the slot
+#pragma unroll
+        for (int b = 0; b < NB32; ++b) tmem_regs_after_wait(rv[b]);
+        if (c == 32 / JP - 1) {  // every load of the accumulator is done: free the slot
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty0 + 8u * g);
         }
+        f2 x[JP / 2][NB32];  // x[p][b] = S[b][JP c + 2p], S[b][JP c + 2p + 1]
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int k0 = 32 * c + 16 * u;  // first coordinate of these 16
-          uint32_t hw[8];
+        for (int p = 0; p < JP / 2; ++p) {
 #pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const f2 y = mul2(make_float2(__uint_as_float(rv[u][2 * p]), __uint_as_float(rv[u][2 * p + 1])), sc2);
+          for (int b = 0; b < NB32; ++b)
+            x[p][b] = make_float2(__uint_as_float(rv[b][2 * p]), __uint_as_float(rv[b][2 * p + 1]));
+          wht_pairs<NB32>(x[p]);  // exact: sums of multiples of 2^-14 below 2^9
+        }
+#pragma unroll
+        for (int b = 0; b < NB32; ++b) {
+          const int k0 = 32 * b + JP * c;  // first coordinate of these JP
+          uint32_t hw[JP / 2];
+#pragma unroll
+          for (int p = 0; p < JP / 2; ++p) {
+            const f2 y = mul2(x[p][b], sc2);
             const __half2 hv = __floats2half2_rn(y.x, y.y);
             hw[p] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[(k0 >> 1) + p];
           }
-          // 32 bytes of the swizzled staging row: chunks col / 8 and col / 8 + 1
-          const int box = k0 >> 6, col = k0 & 63;
-          const uint32_t row_off = (uint32_t)(box * DT_ROWS * 128 + r * 128);
-          const uint32_t c0 = (uint32_t)((col >> 3) ^ (r & 7)), c1 = (uint32_t)(((col >> 3) + 1) ^ (r & 7));
-          *reinterpret_cast<uint4*>(out_sm + row_off + (c0 << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(out_sm + row_off + (c1 << 4)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+          // 16 bytes of the swizzled staging row per 8 coordinates
+#pragma unroll
+          for (int q = 0; q < JP / 8; ++q) {
+            const int kk = k0 + 8 * q, box = kk >> 6, col = kk & 63;
+            const uint32_t off = (uint32_t)(box * DT_ROWS * 128 + r * 128) + ((uint32_t)((col >> 3) ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(out_sm + off) = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+          }
         }
       }
       fence_proxy_async_smem();
