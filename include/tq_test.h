@@ -46,8 +46,10 @@ tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, v
  * tq_decode through a chosen kernel, whatever n is: path 1 the CUDA-core
  * kernel (tq_decode's choice below 128 x SM-count vectors, and at
  * head_dim 256), path 2 the tensor-core kernel (head_dim 64 and 128 only:
- * TQ_ERR_UNSUPPORTED at 256). Same arguments, alignment rules and asynchrony
- * as tq_decode; n must be > 0; any other path is TQ_ERR_INVALID_ARG.
+ * TQ_ERR_UNSUPPORTED at 256). Paths 3 and 4 are the same two kernels for
+ * tq_decode_os: `norms` then points at its uint32 side words. Same
+ * arguments, alignment rules and asynchrony as tq_decode; n must be > 0; any
+ * other path is TQ_ERR_INVALID_ARG.
  */
 tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
                               int path, tq_stream stream);

@@ -281,7 +281,8 @@ def tq_test_encode_stalled(ctx: Ctx, x, n: int, packed, norms, stream=None) -> i
 
 
 def tq_test_decode_path(ctx: Ctx, packed, norms, n: int, x, path: int, stream=None) -> int:
-    """Test hook: decode through kernel `path` (1 CUDA cores, 2 tensor cores); returns the launch status."""
+    """Test hook: decode through kernel `path` (1 CUDA cores, 2 tensor cores; 3 and 4 the same for the
+    offset variant, `norms` then holding its int32 side words); returns the launch status."""
     return _test_lib().tq_test_decode_path(ctx.handle, _ptr(packed), _ptr(norms), int(n), _ptr(x), int(path), _stream(stream))
 
 

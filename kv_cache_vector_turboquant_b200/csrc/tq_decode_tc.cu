@@ -99,7 +99,7 @@ struct DtCfg {
 struct DtArgs {
   CUtensorMap tm_out;  // output as [n rows, d cols] fp16, box 64 x 128, 128-byte swizzle
   const uint8_t* packed;
-  const float* norms;
+  const float* norms;  // the offset variant: its side words (fp16 offset | fp16 scale << 16)
   int64_t n;
   uint32_t* err;
   long long wait_limit;
@@ -144,7 +144,10 @@ TQ_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32
       : "memory");
 }
 
-template <int D, int BITS>
+// OS: the offset + fp16-scale variant (x_hat = offset + (scale / d) D H_pm c,
+// the sign applied in f32 and the offset added before the fp16 rounding, as
+// decode_kernel's offset instance does)
+template <int D, int BITS, bool OS>
 __global__ void __launch_bounds__(DT_WARPS * 32, 1)
     decode_tc_kernel(const __grid_constant__ tq_codec_tables T, const __grid_constant__ DtArgs a) {
   using Cfg = DtCfg<D, BITS>;
@@ -456,8 +459,14 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
       }
       tc_fence_after();
       const int64_t tile = tile_of(i);
-      const float sc = nrm * (1.0f / (float)D);
-      const f2 sc2 = make_float2(sc, sc);
+      float scale = nrm, mu = 0.f;
+      if constexpr (OS) {
+        const uint32_t sw32 = __float_as_uint(nrm);
+        mu = __half2float(__ushort_as_half((unsigned short)(sw32 & 0xffffu)));
+        scale = __half2float(__ushort_as_half((unsigned short)(sw32 >> 16)));
+      }
+      const float sc = scale * (1.0f / (float)D);
+      const f2 sc2 = make_float2(sc, sc), mu2 = make_float2(mu, mu);
       // the group's staging tile must have been read by its previous store
       if (leader && stored_once) bulk_wait_read<0>();
       asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory");
@@ -500,8 +509,17 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
 #pragma unroll
           for (int p = 0; p < JP / 2; ++p) {
             const f2 y = mul2(x[p][b], sc2);
-            const __half2 hv = __floats2half2_rn(y.x, y.y);
-            hw[p] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[(k0 >> 1) + p];
+            if constexpr (OS) {
+              const uint32_t m0 = T.sign_f32[k0 + 2 * p], m1 = T.sign_f32[k0 + 2 * p + 1];
+              const f2 ys = add2(make_float2(__uint_as_float(__float_as_uint(y.x) ^ m0),
+                                             __uint_as_float(__float_as_uint(y.y) ^ m1)),
+                                 mu2);
+              const __half2 hv = __floats2half2_rn(ys.x, ys.y);
+              hw[p] = *reinterpret_cast<const uint32_t*>(&hv);
+            } else {
+              const __half2 hv = __floats2half2_rn(y.x, y.y);
+              hw[p] = *reinterpret_cast<const uint32_t*>(&hv) ^ T.sign_h2[(k0 >> 1) + p];
+            }
           }
           // 16 bytes of the swizzled staging row per 8 coordinates
 #pragma unroll
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
   }
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool OS>
 static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* x, cudaStream_t st) {
   using Cfg = DtCfg<D, BITS>;
   static_assert(Cfg::BYTES <= DT_SMEM_MAX, "shared memory of the tensor-core decode");
@@ -545,7 +563,7 @@ static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* 
   static std::atomic<uint64_t> configured{0};  // one bit per device
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<D, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
+    e = cudaFuncSetAttribute(decode_tc_kernel<D, BITS, OS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -573,7 +591,7 @@ static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* 
       return cudaErrorNotSupported;
     const int64_t tiles = (n + DT_ROWS - 1) / DT_ROWS;
     const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms);
-    e = tq_launch_pdl(decode_tc_kernel<D, BITS>, dim3(grid), dim3(DT_WARPS * 32), Cfg::BYTES, st, T, a);
+    e = tq_launch_pdl(decode_tc_kernel<D, BITS, OS>, dim3(grid), dim3(DT_WARPS * 32), Cfg::BYTES, st, T, a);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -583,8 +601,10 @@ static cudaError_t launch_decode_tc_t(const tq_codec_tables& T, DtArgs a, void* 
 
 using namespace tq;
 
-tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
-                              void* stream) {
+namespace {
+
+tq_status launch_decode_tc_any(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
+                               void* stream, bool os) {
   if (n == 0) return TQ_OK;
   if (ctx->d > 128) return TQ_ERR_UNSUPPORTED;  // one tile would fill tensor memory
   DtArgs a;
@@ -598,11 +618,24 @@ tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorInvalidValue;
   const tq_codec_tables& T = ctx->t;
-#define TQ_DECTC_CASE(D_, B_) \
-  if (ctx->d == D_ && ctx->bits == B_) e = launch_decode_tc_t<D_, B_>(T, a, x, st);
+#define TQ_DECTC_CASE(D_, B_)                                                       \
+  if (ctx->d == D_ && ctx->bits == B_)                                              \
+    e = os ? launch_decode_tc_t<D_, B_, true>(T, a, x, st) : launch_decode_tc_t<D_, B_, false>(T, a, x, st);
   TQ_DECTC_CASE(64, 2) TQ_DECTC_CASE(64, 3) TQ_DECTC_CASE(64, 4)
   TQ_DECTC_CASE(128, 2) TQ_DECTC_CASE(128, 3) TQ_DECTC_CASE(128, 4)
 #undef TQ_DECTC_CASE
   if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
   return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+}  // namespace
+
+tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
+                              void* stream) {
+  return launch_decode_tc_any(ctx, packed, norms, n, x, stream, false);
+}
+
+tq_status tq_launch_decode_tc_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,
+                                 void* stream) {
+  return launch_decode_tc_any(ctx, packed, reinterpret_cast<const float*>(side), n, x, stream, true);
 }

@@ -270,6 +270,11 @@ tq_status tq_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* si
   if (n == 0) return TQ_OK;
   if (!x_f16 || !packed || !side) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(side, 4)) return TQ_ERR_ALIGNMENT;
+  if (n >= tq_encode_tc_min_rows() && tq_tensor_cores_usable(stream)) {
+    // the tensor-core kernel at head_dim <= 128, as tq_decode
+    const tq_status st = tq_launch_decode_tc_os(ctx, packed, side, n, x_f16, stream);
+    if (st != TQ_ERR_UNSUPPORTED) return st;
+  }
   return tq_launch_decode_os(ctx, packed, side, n, x_f16, stream);
 }
 

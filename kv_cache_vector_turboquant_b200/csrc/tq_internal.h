@@ -85,6 +85,9 @@ int64_t tq_encode_tc_min_rows(void);
 // kernel is used). tq_decode uses it from tq_encode_tc_min_rows() vectors on.
 tq_status tq_launch_decode_tc(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x,
                               void* stream);
+// The offset + fp16-scale variant of it: the same outputs as tq_launch_decode_os.
+tq_status tq_launch_decode_tc_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,
+                                 void* stream);
 tq_status tq_launch_encode_os(const tq_ctx* ctx, const void* x, int64_t n, void* packed, uint32_t* side,
                               void* stream);
 tq_status tq_launch_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x,

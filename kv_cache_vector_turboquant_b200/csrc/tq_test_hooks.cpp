@@ -23,14 +23,18 @@ tq_status tq_test_encode_stalled(const tq_ctx* ctx, const void* x_f16, int64_t n
   return tq_launch_encode(ctx, x_f16, n, packed, norms, nullptr, 1, 1, stream, 1);
 }
 
-// tq_decode through a chosen kernel.
+// tq_decode (paths 1, 2) or tq_decode_os (paths 3, 4: `norms` holds the side
+// words) through a chosen kernel.
 tq_status tq_test_decode_path(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
                               int path, tq_stream stream) {
   if (!ctx || n <= 0 || !x_f16 || !packed || !norms) return TQ_ERR_INVALID_ARG;
   if (!aligned(x_f16, 16) || !aligned(packed, 16) || !aligned(norms, 4)) return TQ_ERR_ALIGNMENT;
+  const uint32_t* side = reinterpret_cast<const uint32_t*>(norms);
   switch (path) {
     case 1: return tq_launch_decode(ctx, packed, norms, n, x_f16, stream);
     case 2: return tq_launch_decode_tc(ctx, packed, norms, n, x_f16, stream);
+    case 3: return tq_launch_decode_os(ctx, packed, side, n, x_f16, stream);
+    case 4: return tq_launch_decode_tc_os(ctx, packed, side, n, x_f16, stream);
     default: return TQ_ERR_INVALID_ARG;
   }
 }

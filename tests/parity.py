@@ -66,3 +66,15 @@ def attn_row_error(o: np.ndarray, ref: np.ndarray) -> np.ndarray:
     num = np.abs(o - ref).max(axis=-1)
     den = np.maximum(np.abs(ref).max(axis=-1), 1e-30)
     return num / den
+
+
+def os_decode_ok(gpu16, exact, mu16):
+    """fp16 decode of the offset variant against the fp64 value of the same
+    bytes: within half an fp16 ulp of the exact value plus the two f32
+    roundings (product, sum with the offset)."""
+    g = np.asarray(gpu16, dtype=np.float64)
+    a = np.abs(exact)
+    ulp = np.where(a >= 2.0 ** -14, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10), 2.0 ** -24)
+    mu = np.abs(mu16.astype(np.float64))[:, None]
+    tol = 0.5 * ulp + 2.0 ** -22 * (mu + np.abs(exact - mu16.astype(np.float64)[:, None])) + 1e-30
+    return np.abs(g - exact) <= tol

@@ -151,7 +151,7 @@ def test_decode_path_hook_validation(K):
     ctx = K.tq_create(128, 4)
     h = ctx.handle
     A, B_, C = 0x10000, 0x20000, 0x30000
-    for bad_path in (0, 3, -1):
+    for bad_path in (0, 5, -1):
         assert _raw(K, "tq_test_decode_path", h, A, C, 4, B_, bad_path, None) == K.TQ_ERR_INVALID_ARG
     assert _raw(K, "tq_test_decode_path", None, A, C, 4, B_, 2, None) == K.TQ_ERR_INVALID_ARG
     assert _raw(K, "tq_test_decode_path", h, A, C, 0, B_, 2, None) == K.TQ_ERR_INVALID_ARG

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity import assert_decode_ulp, assert_norms, code_mismatches
+from parity import assert_decode_ulp, assert_norms, code_mismatches, os_decode_ok
 
 pytestmark = pytest.mark.gpu
 
@@ -370,18 +370,6 @@ def test_encode_slots_out_of_range_is_flagged(K, W):
     assert st == K.TQ_ERR_DEVICE and bits == K.TQ_DEVERR_SLOT_RANGE
 
 
-def _os_decode_ok(gpu16, exact, mu16):
-    """fp16 decode of the offset variant against the fp64 value of the same
-    bytes: within half an fp16 ulp of the exact value plus the two f32
-    roundings (product, sum with the offset)."""
-    g = np.asarray(gpu16, dtype=np.float64)
-    a = np.abs(exact)
-    ulp = np.where(a >= 2.0 ** -14, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10), 2.0 ** -24)
-    mu = np.abs(mu16.astype(np.float64))[:, None]
-    tol = 0.5 * ulp + 2.0 ** -22 * (mu + np.abs(exact - mu16.astype(np.float64)[:, None])) + 1e-30
-    return np.abs(g - exact) <= tol
-
-
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_offset_variant_matches_oracle(K, W, d, bits):
@@ -414,7 +402,7 @@ def test_offset_variant_matches_oracle(K, W, d, bits):
     gp = packed.cpu().numpy()
     assert code_mismatches(gp, det, bits, d) == 0
     exact = O.decode_os_f64(gp, side_u, bits, 42, d)
-    assert np.all(_os_decode_ok(dec.cpu().numpy(), exact, gmu))
+    assert np.all(os_decode_ok(dec.cpu().numpy(), exact, gmu))
     # the zero row decodes to zeros and the constant row to itself
     assert torch.all(dec[0] == 0) and torch.all(dec[1].cpu() == x[1])
 

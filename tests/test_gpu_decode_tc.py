@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle as O
-from parity import assert_decode_ulp
+from parity import assert_decode_ulp, os_decode_ok
 
 pytestmark = pytest.mark.gpu
 
@@ -113,4 +113,45 @@ def test_tc_decode_matches_cuda_core_kernel_on_random_sizes(K, W):
         x1 = _dec_path(K, tq, packed, norms, 1)
         assert torch.equal(x1, x2), (d, bits, n)
         del x, packed, norms, x1, x2
+    assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+def _os_side(n, seed):
+    """Side words fp16 offset | fp16 scale << 16, with a zero scale, a tiny
+    and a large one, and a negative offset among them."""
+    g = torch.Generator().manual_seed(seed)
+    mu = (torch.rand(n, generator=g) * 4.0 - 2.0).to(torch.float16)
+    sc = (torch.rand(n, generator=g) * 30.0).to(torch.float16)
+    if n > 3:
+        sc[0], sc[1], sc[2] = 0.0, 6.0e-8, 6.0e4
+        mu[3] = -1.5
+    bits = mu.view(torch.int16).to(torch.int32) & 0xFFFF
+    bits |= (sc.view(torch.int16).to(torch.int32) & 0xFFFF) << 16
+    return bits.cuda()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("n", [1, 129, 148 * 128 * 3 + 77])
+def test_tc_decode_offset_variant_matches_cuda_core_kernel(K, d, bits, n):
+    """The offset + fp16-scale variant on the tensor cores (path 4) against
+    the CUDA-core offset decode (path 3): the sign in f32 and the offset added
+    before the rounding in both, so the outputs are bit-identical; the oracle
+    bounds them to 1 fp16 ulp."""
+    tq = K.TurboQuant(d, bits, seed=9 + bits)
+    packed, _ = _random_codes(tq, n, 300 * d + 10 * bits + n)
+    side = _os_side(n, 7 * d + bits + n)
+    x4 = torch.full((n, d), 7.0, dtype=torch.float16, device="cuda")
+    x3 = torch.full((n, d), 7.0, dtype=torch.float16, device="cuda")
+    assert K._binding.tq_test_decode_path(tq.ctx, packed, side, n, x4, 4) == K.TQ_OK
+    assert K._binding.tq_test_decode_path(tq.ctx, packed, side, n, x3, 3) == K.TQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(x3, x4)
+    sw = side.cpu().numpy().astype(np.uint32)
+    exact = O.decode_os_f64(packed.cpu().numpy(), sw, bits, 9 + bits, d)
+    mu16 = (sw & 0xFFFF).astype(np.uint16).view(np.float16)
+    assert np.all(os_decode_ok(x4.cpu().numpy(), exact, mu16))
+    # a bulk tq_decode_os call takes the tensor-core kernel: same bytes
+    if n >= 128 * 148:
+        assert torch.equal(tq.decode_os(packed, side), x4)
     assert K.tq_device_error() == (K.TQ_OK, 0)
