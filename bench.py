@@ -64,8 +64,9 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, with_power: bool = False):
         self.idx = gpu_index
+        self.with_power = with_power
         self.proc = None
         self.path = os.path.join(tempfile.gettempdir(), f"tq_bench_clocks_{os.getpid()}.csv")
 
@@ -92,7 +93,7 @@ class ClockSampler:
     def summary(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], [], set()
+        sm, smax, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         try:
             for ln in open(self.path):
@@ -104,14 +105,21 @@ class ClockSampler:
                     smax.append(float(parts[2]))
                 except ValueError:
                     continue
+                try:
+                    pw.append(float(parts[3]))
+                except ValueError:
+                    pass
                 for name, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(name)
             os.remove(self.path)
         except Exception:
             pass
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+               "samples": len(sm), "reasons": sorted(reasons)}
+        if self.with_power:
+            out["power_w"] = statistics.median(pw) if pw else None
+        return out
 
 
 def _source_hash(name: str) -> str:
@@ -875,6 +883,56 @@ def run_reference(args):
 PROFILE_CASES = ["encode_b2", "encode_b3", "encode_b4", "decode_b2", "decode_b3", "decode_b4", "attn"]
 
 
+def run_sustained(seconds: float = 2.5):
+    """Each codec launch of the benchmarked step alone (the layer's K and V in
+    one call, tensor-core kernels), the decode-step attention alone and the
+    whole 6-launch step, each run back to back for `seconds` so the GPU
+    reaches its power limit; then 50 timed launches (steps). nvidia-smi is
+    sampled over the second half of each phase: the median SM clock and
+    board power there say which work sets the clock under the power limit."""
+    import torch
+
+    import kv_cache_vector_turboquant_b200 as K
+    import tq_workloads as W
+
+    torch.cuda.set_device(0)
+    S = _codec_step_setup(K, W, torch, 0)
+    phases = [(f"{kind}_b{b}", fn) for kind, b, fn, _, _ in S["launches"]]
+    phases.append(("codec_step", lambda: [L[2]() for L in S["launches"]]))
+    a = ATTN
+    q, k, v = W.decode_step(a["B"], a["Hq"], a["Hkv"], a["S"], a["d"])
+    kc, vc = K.TurboQuant(a["d"], a["kb"]), K.TurboQuant(a["d"], a["vb"])
+    kp, kn = kc.encode(k)
+    vp, vn = vc.encode(v)
+    del k, v
+    pos = torch.full((a["B"],), a["S"], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    ws = torch.empty(K.tq_attend_workspace_bytes(a["B"], a["Hq"], a["d"], a["S"]), dtype=torch.uint8, device="cuda")
+    phases.append(("attention_step", lambda: K.attend_decode(q, kc, vc, kp, kn, vp, vn, pos, out=out, workspace=ws)))
+    res = []
+    for name, fn in phases:
+        t0 = time.time()
+        while time.time() - t0 < seconds / 2:
+            for _ in range(20):
+                fn()
+            torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device(), with_power=True) as cs:
+            while time.time() - t0 < seconds:
+                for _ in range(20):
+                    fn()
+                torch.cuda.synchronize()
+            e0, e1 = _ev(torch), _ev(torch)
+            e0.record()
+            for _ in range(50):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+        res.append({"phase": name, "us": e0.elapsed_time(e1) / 50 * 1e3, **cs.summary()})
+    st = K.tq_device_error()
+    return {"sustained": res, "seconds_per_phase": seconds, "device_error": list(st),
+            "note": "each phase alone, back to back; clock and power are nvidia-smi medians over its second half"}
+
+
 def run_profile_case(case: str, launches: int = 3):
     """A small, self-contained case for Nsight Compute: a few launches of one
     kernel on the benchmark's shapes (the layer's K and V, 256 MiB of fp16,
@@ -925,11 +983,17 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-extras", action="store_true", help="skip the attention and append loops")
     ap.add_argument("--skip-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--sustained", action="store_true",
+                    help="time each codec launch, the codec step and the attention step alone at the power limit "
+                         "(with clock and power) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.profile:
         run_profile_case(args.profile)
+        return
+    if args.sustained:
+        print(json.dumps(run_sustained()), flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
