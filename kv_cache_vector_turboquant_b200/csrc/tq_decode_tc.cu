@@ -93,7 +93,12 @@ struct DtCfg {
   // full[S], empty[S], aready[NA][2], aempty[NA][2], tfull[2], tempty[2], done
   static constexpr int NBARS = 2 * STAGES + 4 * NA + 4 + 1;
   static constexpr int SLOT = BAR + NBARS * 8;
-  static constexpr size_t BYTES = 1024 + (size_t)SLOT + 16;
+  // at 3 bits the table (64 entries of 256 B) starts at a shared address that
+  // is a multiple of its 16 KB size, so an entry's address is the code pair's
+  // bits shifted into place OR'd with the lane's offset (the base moves by up
+  // to 15 KB for it); otherwise the base is 1024-aligned
+  static constexpr uint32_t LUT_ALIGN = BITS == 3 ? 16384u : 1024u;
+  static constexpr size_t BYTES = LUT_ALIGN + (size_t)SLOT + 16;
 };
 
 struct DtArgs {
@@ -156,7 +161,8 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
+  static_assert(Cfg::LUT % 1024 == 0, "the table offset keeps the base 1024-aligned");
+  const uint32_t base = ((raw + (uint32_t)Cfg::LUT + Cfg::LUT_ALIGN - 1u) & ~(Cfg::LUT_ALIGN - 1u)) - (uint32_t)Cfg::LUT;
   uint8_t* sm = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the next kernel of the stream may start its own set-up as this grid's
@@ -406,18 +412,24 @@ __global__ void __launch_bounds__(DT_WARPS * 32, 1)
             for (int t = 0; t < 16; ++t) {
               constexpr int FB = 2 * BITS;
               const int off = (c0 + t) * FB;
-              uint32_t f;
-              if constexpr (FB == 8) {  // a pair is a byte
-                f = __byte_perm(words[off >> 5], 0u, 0x4440u | (uint32_t)((off >> 3) & 3));
-              } else {
-                f = words[off >> 5] >> (off & 31);
-                if ((off & 31) + FB > 32) f |= words[(off >> 5) + 1] << (32 - (off & 31));
-                f &= (uint32_t)(Cfg::E - 1);
+              uint32_t addr;  // the code pair's table entry for this lane
+              if constexpr (FB == 8) {  // 4 bits: a pair is a byte
+                const uint32_t f = __byte_perm(words[off >> 5], 0u, 0x4440u | (uint32_t)((off >> 3) & 3));
+                addr = f * 256u + lut_lane;
+              } else {  // 3 bits: the 6-bit pair shifted to bits 8-13, OR'd with the aligned lane offset
+                static_assert(Cfg::E == 64 && Cfg::LUT_ALIGN == 16384u, "aligned 3-bit table");
+                const int sh = off & 31;
+                uint32_t g;
+                if (sh + FB > 32)
+                  g = __funnelshift_r(words[off >> 5], words[(off >> 5) + 1], sh - 8);
+                else
+                  g = sh >= 8 ? words[off >> 5] >> (sh - 8) : words[off >> 5] << (8 - sh);
+                addr = (g & 0x3F00u) | lut_lane;
               }
               // the value pair and the remainder pair by two 4-byte loads, so
               // each lands in the register its tensor-memory store reads
-              vv[t] = dt_lds_u32(f * 256u + lut_lane);
-              rr[t] = dt_lds_u32(f * 256u + lut_lane + 128u);
+              vv[t] = dt_lds_u32(addr);
+              rr[t] = dt_lds_u32(addr + 128u);
             }
           }
           tmem_st16(sb + (uint32_t)c0, vv);
