@@ -484,3 +484,18 @@ def test_back_to_back_bulk_launches_see_each_others_outputs(K, W, d, bits):
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
     assert K.tq_device_error() == (K.TQ_OK, 0)
+
+
+def test_bench_sustained_mode_reports_every_phase(K):
+    """`bench.py --sustained` (its summary is committed under profiles/): one
+    short run of every phase, each with a time, a clock and a power figure,
+    and no device error."""
+    import bench
+
+    res = bench.run_sustained(seconds=0.2)
+    names = [r["phase"] for r in res["sustained"]]
+    assert names == [f"{k}_b{b}" for k in ("encode", "decode") for b in (2, 3, 4)] + ["codec_step", "attention_step"]
+    for r in res["sustained"]:
+        assert r["us"] > 0.0
+        assert "sm_mhz" in r and "power_w" in r
+    assert res["device_error"] == [K.TQ_OK, 0]
