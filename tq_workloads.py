@@ -21,6 +21,8 @@ Workloads (names used by the tests and ``bench.py``):
   sources [16, 32768, 8, 128] N(0,1) (seeds 12, 13).
 * ``append_stream``: 256 sequences x 8 heads, one token per step, N(0,1) with
   each coordinate x20 with probability 0.005 (seed 21 + run).
+* ``stress_rows``: the seven stress distributions of the parity stress test
+  (``STRESS_KINDS``; see the function).
 """
 
 from __future__ import annotations
@@ -122,3 +124,41 @@ def edge_vectors(d: int, device="cpu") -> torch.Tensor:
     rows.append(torch.tensor([(-1.0) ** i * 2.0 ** -20 for i in range(d)]))
     rows.append(torch.tensor([(-1.0) ** (i // 3) for i in range(d)]))
     return torch.stack(rows).to(torch.float16).to(device)
+
+
+STRESS_KINDS = ("gauss", "student3", "channel_lognormal", "outlier_x10", "dynamic_range", "sparse", "mean_dominated")
+
+
+def stress_rows(kind: str, n: int, d: int, seed: int, device="cuda") -> torch.Tensor:
+    """n x d rows of one of the stress distributions, float32 then fp16 once
+    (values clamped to +-60000 before the cast):
+
+    * ``gauss``: N(0,1);
+    * ``student3``: N(0,1) / sqrt(chi^2_3 / 3) per element (heavy tails);
+    * ``channel_lognormal``: N(0,1) times a per-channel exp(1.5 N(0,1));
+    * ``outlier_x10``: N(0,1) with 4 channels (randperm) times 10;
+    * ``dynamic_range``: N(0,1) times 2^k per element, k uniform in [-14, 13];
+    * ``sparse``: N(0,1) kept with probability 0.1, else 0;
+    * ``mean_dominated``: 3 + 0.01 N(0,1).
+    """
+    g = _gen(seed, device)
+    x = torch.randn(n, d, generator=g, device=device, dtype=torch.float32)
+    if kind == "gauss":
+        pass
+    elif kind == "student3":
+        chi = torch.randn(n, d, 3, generator=g, device=device).pow(2).sum(-1) / 3
+        x = x / chi.sqrt()
+    elif kind == "channel_lognormal":
+        x = x * torch.exp(torch.randn(1, d, generator=g, device=device) * 1.5)
+    elif kind == "outlier_x10":
+        cols = torch.randperm(d, generator=_gen(seed, "cpu"))[:4].to(device)
+        x[:, cols] *= 10.0
+    elif kind == "dynamic_range":
+        x = x * torch.pow(2.0, torch.randint(-14, 14, (n, d), generator=g, device=device).float())
+    elif kind == "sparse":
+        x = x * (torch.rand(n, d, generator=g, device=device) < 0.1).float()
+    elif kind == "mean_dominated":
+        x = x * 0.01 + 3.0
+    else:
+        raise ValueError(f"unknown stress kind {kind!r}")
+    return x.clamp(-60000.0, 60000.0).to(torch.float16)
