@@ -66,6 +66,60 @@ class TurboQuant:
         """fp16 bytes over stored bytes (packed codes + f32 norm) per vector."""
         return 2.0 * self.head_dim / (self.packed_bytes + 4)
 
+    def memory_report(self, seq_len: int, num_layers: int = 32, num_kv_heads: int = 8) -> dict:
+        """KV-cache bytes of one sequence of `seq_len` tokens over `num_layers`
+        layers of `num_kv_heads` kv heads (K and V), fp16 against this codec
+        (packed codes plus one f32 norm per vector)."""
+        vectors = 2 * int(num_layers) * int(num_kv_heads) * int(seq_len)
+        fp16 = vectors * 2 * self.head_dim
+        packed = vectors * (self.packed_bytes + 4)
+        return {"vectors": vectors, "fp16_bytes": fp16, "packed_bytes": packed, "saved_bytes": fp16 - packed,
+                "compression_ratio": fp16 / packed, "bits": self.bits, "head_dim": self.head_dim}
+
+    def validate(self, num_vectors: int = 10000, seed: int = 0) -> dict:
+        """Encode and decode `num_vectors` seeded N(0,1) fp16 vectors on the
+        current device and report the reconstruction: mean relative squared
+        error ||x - x_hat||^2 / ||x||^2, mean cosine similarity, and the
+        largest relative error of the stored norms."""
+        import torch
+
+        g = torch.Generator(device="cuda").manual_seed(int(seed))
+        x = torch.randn(int(num_vectors), self.head_dim, generator=g, device="cuda").to(torch.float16)
+        packed, norms = self.encode(x)
+        xh = self.decode(packed, norms).float()
+        xf = x.float()
+        nx = xf.norm(dim=1)
+        rel = ((xf - xh).pow(2).sum(dim=1) / nx.pow(2)).mean().item()
+        cos = torch.nn.functional.cosine_similarity(xf, xh, dim=1).mean().item()
+        nerr = ((norms - xf.double().norm(dim=1).float()).abs() / nx).max().item()
+        return {"num_vectors": int(num_vectors), "mse_relative": rel, "cosine": cos, "max_norm_rel_err": nerr,
+                "bits": self.bits, "head_dim": self.head_dim}
+
+    def benchmark(self, num_vectors: int = 32768, reps: int = 20) -> dict:
+        """Device time of one encode and one decode of `num_vectors` vectors
+        (CUDA events around `reps` back-to-back calls after a warm-up), with
+        the fp16-equivalent throughput (2 * head_dim bytes per vector)."""
+        import torch
+
+        x = torch.randn(int(num_vectors), self.head_dim, device="cuda").to(torch.float16)
+        packed, norms = self.encode(x)
+        out = self.decode(packed, norms)
+        res = {"num_vectors": int(num_vectors), "bits": self.bits, "head_dim": self.head_dim}
+        for name, fn in (("encode", lambda: self.encode(x, out=(packed, norms))),
+                         ("decode", lambda: self.decode(packed, norms, out=out))):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(int(reps)):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / int(reps) / 1e3
+            res[f"{name}_us"] = t * 1e6
+            res[f"{name}_GBps"] = 2.0 * self.head_dim * int(num_vectors) / t / 1e9
+        return res
+
     def encode(self, x, out=None, stream=None):
         """[..., d] fp16 CUDA tensor -> ([..., d*b/8] uint8, [...] float32)."""
         import torch
@@ -165,6 +219,28 @@ def attend_decode(q, k_codec: TurboQuant, v_codec: TurboQuant, k_packed, k_norms
     tq_attend_decode(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_packed, k_norms, v_packed, v_norms, s_max,
                      positions, out, workspace, workspace.numel(), stream)
     return out
+
+
+class TQPagedAttention:
+    """Decode-step attention over paged packed caches, in the form of the
+    pages' `TQPagedAttention(tq, num_query_heads).forward(...)`: `tq` codes
+    the keys and, unless `v_tq` is given, the values too."""
+
+    def __init__(self, tq: TurboQuant, num_query_heads: int, v_tq: TurboQuant = None):
+        self.k_codec, self.v_codec = tq, (v_tq if v_tq is not None else tq)
+        self.num_query_heads = int(num_query_heads)
+
+    def forward(self, query, k_packed, k_norms, v_packed, v_norms, block_tables, context_lens, out=None,
+                workspace=None, stream=None):
+        """query [B, num_query_heads, head_dim] fp16; caches [num_blocks, 16,
+        Hkv, P]; block_tables [B, max_blocks] int32; context_lens [B] int32.
+        Returns [B, num_query_heads, head_dim] fp16."""
+        _require(query.dim() == 3 and query.shape[1] == self.num_query_heads,
+                 "query must be [B, num_query_heads, head_dim]")
+        return attend_decode_paged(query, self.k_codec, self.v_codec, k_packed, k_norms, v_packed, v_norms,
+                                   block_tables, context_lens, out=out, workspace=workspace, stream=stream)
+
+    __call__ = forward
 
 
 def attend_decode_paged(q, k_codec: TurboQuant, v_codec: TurboQuant, k_cache, k_norms, v_cache, v_norms,

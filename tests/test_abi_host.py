@@ -285,3 +285,16 @@ def test_offset_variant_validation(K):
     assert _raw(K, "tq_encode_os", h, A + 2, 4, A, A, None) == K.TQ_ERR_ALIGNMENT
     assert _raw(K, "tq_encode_os", h, A, 4, A, A + 2, None) == K.TQ_ERR_ALIGNMENT
     assert _raw(K, "tq_decode_os", h, A, A + 1, 4, A, None) == K.TQ_ERR_ALIGNMENT
+
+
+@pytest.mark.parametrize("d,bits", [(64, 2), (128, 4), (256, 3)])
+def test_memory_report_arithmetic(K, d, bits):
+    """TurboQuant.memory_report: K and V of seq_len tokens x layers x kv
+    heads, fp16 (2 d bytes per vector) against packed codes + f32 norm."""
+    tq = K.TurboQuant(d, bits)
+    r = tq.memory_report(4096, num_layers=32, num_kv_heads=8)
+    vectors = 2 * 32 * 8 * 4096
+    assert r["vectors"] == vectors
+    assert r["fp16_bytes"] == vectors * 2 * d
+    assert r["packed_bytes"] == vectors * (d * bits // 8 + 4)
+    assert r["compression_ratio"] == pytest.approx(tq.compression_ratio())

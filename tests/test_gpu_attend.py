@@ -199,8 +199,11 @@ def test_paged_attention_matches_contiguous_and_oracle(K, W, d, kb, vb, B, S, hq
         bt[b, (n + 15) // 16:] = -12345
     o_paged = K.attend_decode_paged(q, kc, vc, kpool, knpool, vpool, vnpool, bt, lens_t)
     o_contig = K.attend_decode(q, kc, vc, kp, kn, vp, vn, lens_t)
+    # the pages' class form of the same call
+    o_class = K.TQPagedAttention(kc, hq, v_tq=vc).forward(q, kpool, knpool, vpool, vnpool, bt, lens_t)
     torch.cuda.synchronize()
     assert torch.equal(o_paged, o_contig)
+    assert torch.equal(o_class, o_paged)
     assert K.tq_device_error() == (K.TQ_OK, 0)
     ref = O.attend_decode_paged(q.cpu().numpy(), kpool.cpu().numpy(), knpool.cpu().numpy(), vpool.cpu().numpy(),
                                 vnpool.cpu().numpy(), bt.cpu().numpy(), lens, kb, vb)

@@ -499,3 +499,21 @@ def test_bench_sustained_mode_reports_every_phase(K):
         assert r["us"] > 0.0
         assert "sm_mhz" in r and "power_w" in r
     assert res["device_error"] == [K.TQ_OK, 0]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_validate_and_benchmark_helpers(K, bits):
+    """TurboQuant.validate / benchmark (the pages' helper methods): the
+    reconstruction of N(0,1) vectors has the sphere-marginal distortion of
+    the width (within 5 %), cosine close to 1, norms within 1e-6; benchmark
+    returns positive times for both directions."""
+    tq = K.TurboQuant(128, bits)
+    v = tq.validate(num_vectors=20000)
+    # ||x - x_hat||^2 / ||x||^2 is the squared error of the unit direction,
+    # whose expectation is the sphere-marginal distortion of one coordinate
+    want = O.sphere_marginal_mse(O.format_levels(bits), 128)
+    assert abs(v["mse_relative"] - want) <= 0.05 * want, (v, want)
+    assert v["cosine"] > 0.9 and v["max_norm_rel_err"] <= 1e-6
+    b = tq.benchmark(num_vectors=32768, reps=3)
+    assert b["encode_us"] > 0 and b["decode_us"] > 0
+    assert K.tq_device_error() == (K.TQ_OK, 0)
