@@ -697,6 +697,14 @@ def run_ours(args, rank, world, local_rank):
     tot = sum(v["share"] for v in kernels.values())
     for v in kernels.values():
         v["share"] = v["share"] / tot
+    # each launch of the step also timed back to back (`steps` calls between
+    # two events): the event pair around every launch above adds ~2-3 us each
+    for kind, b, fn, alg, _ in launches:
+        t = _bracketed_ms(torch, fn, args.steps) / 1e3
+        k = kernels[f"{kind}_b{b}"]
+        k["us_b2b"] = t * 1e6
+        k["GBps_b2b"] = alg / t / 1e9
+        k["frac_b2b"] = alg / t / 1e9 / peak
     dom_name = max(kernels, key=lambda n: kernels[n]["share"])
     dom = kernels[dom_name]
     src = "tq_encode_tc.cu" if dom_name.startswith("encode") else "tq_decode_tc.cu"
