@@ -291,24 +291,23 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1)
           const __half2 hv = __floats2half2_rn(y.x, y.y);
           h[q] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        *reinterpret_cast<uint4*>(orow + 16 * (c ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
-        continue;
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const f2 y = mul2(v[4 * c + q], sc2);
-        const __half2 hv = __floats2half2_rn(y.x, y.y);
-        h[q] = *reinterpret_cast<const uint32_t*>(&hv);
-      }
-      if constexpr (LPV <= 2) {  // masks from the constant bank
+      } else {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          h[q] ^= T.sign_h2[4 * c + q];
-          if (LPV == 2 && part) h[q] ^= T.sign_h2_dx[4 * c + q];
+          const f2 y = mul2(v[4 * c + q], sc2);
+          const __half2 hv = __floats2half2_rn(y.x, y.y);
+          h[q] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-      } else {
-        const uint4 mk = my_masks[c];
-        h[0] ^= mk.x, h[1] ^= mk.y, h[2] ^= mk.z, h[3] ^= mk.w;
+        if constexpr (LPV <= 2) {  // masks from the constant bank
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            h[q] ^= T.sign_h2[4 * c + q];
+            if (LPV == 2 && part) h[q] ^= T.sign_h2_dx[4 * c + q];
+          }
+        } else {
+          const uint4 mk = my_masks[c];
+          h[0] ^= mk.x, h[1] ^= mk.y, h[2] ^= mk.z, h[3] ^= mk.w;
+        }
       }
       *reinterpret_cast<uint4*>(orow + 16 * (c ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
     }
