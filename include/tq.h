@@ -141,8 +141,9 @@ tq_status tq_encode(const tq_ctx* ctx, const void* x_f16, int64_t n, void* packe
  * fp16 range, e.g. entries near +-65504) becomes +-Inf, as an fp16
  * conversion of that value does. Launches of at least
  * 128 x SM-count vectors at head_dim 64 and 128 run on the tensor cores (the
- * 16-point Hadamard blocks as tcgen05 MMAs with A in tensor memory), other
- * launches on the CUDA cores; the outputs are bit-identical.
+ * 32-point Hadamard blocks as tcgen05 MMAs with A in tensor memory, the
+ * remaining stages as f32 butterflies), other launches on the CUDA cores;
+ * the outputs are bit-identical.
  * n == 0 is a no-op. Asynchronous on `stream`.
  */
 tq_status tq_decode(const tq_ctx* ctx, const void* packed, const float* norms, int64_t n, void* x_f16,
@@ -202,6 +203,9 @@ tq_status tq_encode_os(const tq_ctx* ctx, const void* x_f16, int64_t n, void* pa
  * (H_pm the +-1 Walsh-Hadamard matrix), computed in f32 (a product and a sum
  * of the offset, each rounded once) and rounded to fp16.
  *   packed, side as written by tq_encode_os; x_f16 device [n, head_dim] out.
+ * Launches of at least 128 x SM-count vectors at head_dim 64 and 128 run on
+ * the tensor cores (as tq_decode), other launches on the CUDA cores; the
+ * outputs are bit-identical. Asynchronous on `stream`.
  */
 tq_status tq_decode_os(const tq_ctx* ctx, const void* packed, const uint32_t* side, int64_t n, void* x_f16,
                        tq_stream stream);
