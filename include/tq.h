@@ -356,6 +356,16 @@ tq_status tq_tensor_core_check(int* passed);
  */
 tq_status tq_device_error(tq_stream stream, uint32_t* bits);
 
+/*
+ * The same query in the form a caller holding a context uses after it has
+ * synchronised its stream(s): reads and clears the error word of the current
+ * device (the word is per device, not per context: the context is only
+ * validated). Returns TQ_ERR_INVALID_ARG for a NULL context, TQ_ERR_TIMEOUT
+ * if TQ_DEVERR_TIMEOUT was set, TQ_ERR_DEVICE if another bit was set, else
+ * TQ_OK. It synchronises the legacy default stream before the read.
+ */
+tq_status tq_check_device_error(const tq_ctx* ctx);
+
 #ifdef __cplusplus
 }
 #endif

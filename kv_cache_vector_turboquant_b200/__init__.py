@@ -36,6 +36,7 @@ from ._binding import (  # noqa: F401
     tq_attend_workspace_bytes,
     tq_create,
     tq_decode,
+    tq_check_device_error,
     tq_device_error,
     tq_encode,
     tq_encode_append,

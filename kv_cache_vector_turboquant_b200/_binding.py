@@ -47,6 +47,7 @@ _PROTOS = {
     "tq_attend_decode_paged": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_i64, _vp,
                                         _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "tq_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "tq_check_device_error": (_c_int, [_vp]),
     "tq_tensor_core_check": (_c_int, [ctypes.POINTER(_c_int)]),
 }
 for _name, (_res, _args) in _PROTOS.items():
@@ -259,6 +260,12 @@ def tq_device_error(stream=None) -> tuple[int, int]:
     bits = ctypes.c_uint32(0)
     st = _lib.tq_device_error(_stream(stream), ctypes.byref(bits))
     return st, bits.value
+
+
+def tq_check_device_error(ctx) -> int:
+    """Status of the current device's error word (read and cleared) for a
+    caller that holds a context and has synchronised its streams."""
+    return int(_lib.tq_check_device_error(ctx.handle if ctx is not None else None))
 
 
 def tq_tensor_core_check() -> bool:

@@ -341,4 +341,9 @@ tq_status tq_attend_decode_paged(const tq_ctx* k, const tq_ctx* v, const void* q
 
 tq_status tq_device_error(tq_stream stream, uint32_t* bits) { return tq_read_error_word(stream, bits); }
 
+tq_status tq_check_device_error(const tq_ctx* ctx) {
+  if (!ctx) return TQ_ERR_INVALID_ARG;
+  return tq_read_error_word(nullptr, nullptr);
+}
+
 }  // extern "C"

@@ -96,6 +96,10 @@ def test_null_context_queries(lib):
         f = getattr(lib, fn)
         f.argtypes = [ctypes.c_void_p]
         assert f(None) == 0
+    # the context form of the device-error query validates before any CUDA call
+    f = lib.tq_check_device_error
+    f.argtypes = [ctypes.c_void_p]
+    assert f(None) == 1  # TQ_ERR_INVALID_ARG
 
 
 class _FakePtr:

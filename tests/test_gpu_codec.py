@@ -446,6 +446,11 @@ def test_bounded_wait_times_out_and_context_survives(K, W):
     st, bits = K.tq_device_error()
     assert st == K.TQ_ERR_TIMEOUT and bits & K.TQ_DEVERR_TIMEOUT
     assert torch.all(p == 0)
+    # the context form of the query reports the same word
+    assert K._binding.tq_test_encode_stalled(tq.ctx, x, 256, p, nrm) == K.TQ_OK
+    torch.cuda.synchronize()
+    assert K.tq_check_device_error(tq.ctx) == K.TQ_ERR_TIMEOUT
+    assert K.tq_check_device_error(tq.ctx) == K.TQ_OK  # read and cleared
     # context usable afterwards, error word cleared
     p2, n2 = _encode(tq, x)
     assert K.tq_device_error() == (K.TQ_OK, 0)
