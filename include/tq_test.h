@@ -78,6 +78,21 @@ tq_status tq_test_umma_block(const void* a_f16, const void* b_f16, float* d, tq_
  */
 tq_status tq_test_reset_tensor_core_check(int force_fail);
 
+/*
+ * The fast attention kernel's shared-memory plan (host arithmetic only, no
+ * CUDA call): for head_dim d (128 or 256), hw kv heads (4, 8 or 16) and nt
+ * column tiles (1 or 2) per CTA, a paged (1) or contiguous (0) cache, a
+ * device that reserves `reserved` bytes before the dynamic region and grants
+ * `max_dyn` bytes of it.
+ *   out  host, [8 + 4 * 8] int32 out: stages, warp groups, table offset,
+ *        table bytes, header bytes, K / V / norm bytes per stage, then the
+ *        offsets of the K, V, K-norm and V-norm buffers of stages 0..7 (-1
+ *        past the last stage).
+ * TQ_ERR_INVALID_ARG for out == NULL, TQ_ERR_UNSUPPORTED if the shape is not
+ * the fast kernel's or no plan of at least two stages per group fits.
+ */
+tq_status tq_test_attend_plan(int d, int hw, int nt, int paged, int reserved, int max_dyn, int32_t* out);
+
 #ifdef __cplusplus
 }
 #endif

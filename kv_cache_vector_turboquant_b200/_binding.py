@@ -65,6 +65,7 @@ _TEST_PROTOS = {
     "tq_test_encode_path": (_c_int, [_vp, _vp, _c_i64, _vp, _vp, _c_int, _vp]),
     "tq_test_umma_block": (_c_int, [_vp, _vp, _vp, _vp]),
     "tq_test_decode_path": (_c_int, [_vp, _vp, _vp, _c_i64, _vp, _c_int, _vp]),
+    "tq_test_attend_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
 }
 _test = None
 
@@ -274,6 +275,20 @@ def tq_tensor_core_check() -> bool:
     passed = _c_int(0)
     _check(_lib.tq_tensor_core_check(ctypes.byref(passed)), "tq_tensor_core_check")
     return bool(passed.value)
+
+
+def tq_test_attend_plan(d: int, hw: int, nt: int, paged: bool, reserved: int, max_dyn: int):
+    """(status, plan) of the fast attention kernel's shared memory (host
+    arithmetic); plan is a dict of the stage count, groups, regions and the
+    per-stage buffer offsets."""
+    out = (ctypes.c_int32 * 40)()
+    st = _test_lib().tq_test_attend_plan(int(d), int(hw), int(nt), int(bool(paged)), int(reserved), int(max_dyn),
+                                         ctypes.cast(out, _vp))
+    v = list(out)
+    plan = {"stages": v[0], "groups": v[1], "table_off": v[2], "table_bytes": v[3], "header_bytes": v[4],
+            "k_bytes": v[5], "v_bytes": v[6], "norm_bytes": v[7],
+            "k": v[8:16], "v": v[16:24], "kn": v[24:32], "vn": v[32:40]}
+    return st, plan
 
 
 def tq_test_reset_tensor_core_check(force_fail: bool = False) -> int:

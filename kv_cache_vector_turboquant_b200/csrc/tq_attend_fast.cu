@@ -1,6 +1,8 @@
 // Decode-step attention over packed caches, specialised for 4-bit keys and
 // 2-bit values (the asymmetric K/V split of the "KVarN" and "aither-kvcache"
-// pages) at head_dim 128 or 256.
+// pages) at head_dim 128, and at 256 for more than 4 query heads per kv head
+// (with fewer, the stages of a CTA's kv heads do not fit beside the table and
+// the launch takes the generic kernel).
 //
 // Same mathematics as the generic kernel (tq_attend.cu, after the
 // "aither-kvcache" page, section "Zero-buffer fused attention", and
@@ -12,7 +14,8 @@
 // small:
 //
 //  * One CTA of 16 warps per SM, 227 KB of shared memory: a 64 KB key table
-//    region and 6 tiles of 32 positions in flight. A tile arrives as four
+//    region and as many tiles of 32 positions in flight as fit around it (4
+//    at head_dim 128 with 8 kv heads per CTA). A tile arrives as four
 //    tensor copies (TMA, no multicast): K codes as [kv head][position][row]
 //    (a box whose position and head dimensions are swapped relative to
 //    memory, so the 16-byte fragment loads of a warp fall in distinct banks),
@@ -568,9 +571,9 @@ static bool encode_map(CUtensorMap* m, CUtensorMapDataType type, const void* bas
 // aligned) in the space below and above the tables. The most stages that
 // fit, a multiple of the group count and at least two per group.
 static bool plan_smem(FastArgs& f, int base, int max_dyn, int kbytes, int vbytes, int nbytes, int hdr) {
-  const int tb_abs = (base + FA_TABLE_BYTES - 1) & ~(FA_TABLE_BYTES - 1);
+  const int tb_abs = (base + hdr + FA_TABLE_BYTES - 1) & ~(FA_TABLE_BYTES - 1);  // the first boundary past the header
   const int tb_off = tb_abs - base;
-  if (tb_off < hdr || tb_off + FA_TABLE_BYTES > max_dyn) return false;
+  if (tb_off + FA_TABLE_BYTES > max_dyn) return false;
   for (int ns = FA_MAX_STAGES; ns >= 2 * f.n_groups; --ns) {
     if (ns % f.n_groups) continue;
     int lo[2] = {hdr, tb_off + FA_TABLE_BYTES}, hi[2] = {tb_off, max_dyn};
@@ -599,9 +602,55 @@ static bool plan_smem(FastArgs& f, int base, int max_dyn, int kbytes, int vbytes
   return false;
 }
 
+// The launch geometry that depends only on the shapes and the device's
+// shared memory: warps per tile and groups, the V row pitch, the paged
+// block-row cache, the stage buffers and the table region. False when no plan
+// of at least two stages per group fits.
+static bool fast_plan(FastArgs& f, int d, int hw, int nt, bool paged, int reserved, int max_dyn) {
+  const int pk = d / 2, pv = d / 4;
+  f.wpt = hw * nt;
+  f.n_groups = FA_WARPS / f.wpt;
+  f.vpitch = hw * pv + 16;
+  const int np = fa_norm_pitch(hw);
+  const int kbytes = ATT_TILE * hw * pk, vbytes = ATT_TILE * f.vpitch, nbytes = ATT_TILE * np * 4;
+  // paged: 2 KB after the 128-byte header hold the rows of the split's first
+  // 512 blocks, so the issuing thread reads them from shared memory
+  f.pg_off = 128;
+  f.pg_cap = paged ? 512 : 0;
+  if (!plan_smem(f, reserved, max_dyn, kbytes, vbytes, nbytes, 128 + 4 * f.pg_cap)) return false;
+  f.smem_base = (uint32_t)reserved;
+  f.tile_bytes = (uint32_t)(kbytes + vbytes + 2 * nbytes);
+  return true;
+}
+
 }  // namespace tq
 
 using namespace tq;
+
+bool tq_attend_fast_plan(int d, int hw, int nt, int paged, int reserved, int max_dyn, int32_t* out) {
+  if ((d != 128 && d != 256) || (hw != 4 && hw != 8 && hw != 16) || (nt != 1 && nt != 2) ||
+      FA_WARPS % (hw * nt) != 0)
+    return false;
+  FastArgs f;
+  if (!fast_plan(f, d, hw, nt, paged != 0, reserved, max_dyn)) return false;
+  const int np = fa_norm_pitch(hw);
+  out[0] = f.n_stages;
+  out[1] = f.n_groups;
+  out[2] = f.tb_off;
+  out[3] = FA_TABLE_BYTES;
+  out[4] = 128 + 4 * f.pg_cap;  // header and paged block-row cache
+  out[5] = ATT_TILE * hw * (d / 2);
+  out[6] = ATT_TILE * f.vpitch;
+  out[7] = ATT_TILE * np * 4;
+  for (int s = 0; s < FA_MAX_STAGES; ++s) {
+    const bool used = s < f.n_stages;
+    out[8 + s] = used ? f.kbuf[s] : -1;
+    out[8 + FA_MAX_STAGES + s] = used ? f.vbuf[s] : -1;
+    out[8 + 2 * FA_MAX_STAGES + s] = used ? f.knb[s] : -1;
+    out[8 + 3 * FA_MAX_STAGES + s] = used ? f.vnb[s] : -1;
+  }
+  return true;
+}
 
 cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, int sm_count, cudaStream_t st) {
   if (k_bits != 4 || v_bits != 2 || (d != 128 && d != 256)) return cudaErrorNotSupported;
@@ -631,18 +680,8 @@ cudaError_t tq_launch_attend_fast(AttnArgs& a, int d, int k_bits, int v_bits, in
     return cudaErrorUnknown;
 
   FastArgs f;
-  f.wpt = hw * nt;
-  f.n_groups = FA_WARPS / f.wpt;
-  f.vpitch = hw * pv + 16;
+  if (!fast_plan(f, d, hw, nt, paged, reserved, max_dyn)) return cudaErrorNotSupported;
   const int np = fa_norm_pitch(hw);
-  const int kbytes = ATT_TILE * hw * pk, vbytes = ATT_TILE * f.vpitch, nbytes = ATT_TILE * np * 4;
-  // paged: 2 KB after the 128-byte header hold the rows of the split's first
-  // 512 blocks, so the issuing thread reads them from shared memory
-  f.pg_off = 128;
-  f.pg_cap = paged ? 512 : 0;
-  if (!plan_smem(f, reserved, max_dyn, kbytes, vbytes, nbytes, 128 + 4 * f.pg_cap)) return cudaErrorNotSupported;
-  f.smem_base = (uint32_t)reserved;
-  f.tile_bytes = (uint32_t)(kbytes + vbytes + 2 * nbytes);
   // the rotated queries (before the tables) and the group merge (after) use the table region
   if (hw * a.g * d * 4 > FA_TABLE_BYTES) return cudaErrorNotSupported;
   if ((f.n_groups - 1) * f.wpt * 32 * (d / 8 + 2) * 4 > FA_TABLE_BYTES) return cudaErrorNotSupported;

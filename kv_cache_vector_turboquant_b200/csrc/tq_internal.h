@@ -104,6 +104,13 @@ tq_status tq_launch_attend_paged(const tq_ctx* k, const tq_ctx* v, const void* q
                                  int max_blocks, const int32_t* context_lens, void* out, void* workspace,
                                  size_t ws_bytes, void* stream);
 size_t tq_attend_workspace_bytes_impl(int B, int hq, int head_dim, int64_t s_max);
+// The fast attention kernel's shared-memory plan for head_dim d, hw kv heads
+// and nt column tiles per CTA, a paged or contiguous cache, `reserved` bytes
+// before the dynamic region and `max_dyn` bytes of it (host arithmetic only).
+// out[0..7] = stages, warp groups, table offset, table bytes, header bytes,
+// K / V / norm bytes per stage; out[8 + 8 k + s] = offset of buffer k (K, V,
+// K norms, V norms) of stage s, -1 past the stages. False if no plan fits.
+bool tq_attend_fast_plan(int d, int hw, int nt, int paged, int reserved, int max_dyn, int32_t* out);
 
 // 1 if the tensor-core encode and decode kernels may run on the current
 // device: the run-time check of the tensor core's rounding (tq_mma_check.cu)

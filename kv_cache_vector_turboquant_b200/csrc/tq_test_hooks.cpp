@@ -56,4 +56,9 @@ tq_status tq_test_encode_path(const tq_ctx* ctx, const void* x_f16, int64_t n, v
 // the next check to report a mismatch).
 tq_status tq_test_reset_tensor_core_check(int force_fail) { return tq_tensor_core_check_reset(force_fail); }
 
+tq_status tq_test_attend_plan(int d, int hw, int nt, int paged, int reserved, int max_dyn, int32_t* out) {
+  if (!out) return TQ_ERR_INVALID_ARG;
+  return tq_attend_fast_plan(d, hw, nt, paged, reserved, max_dyn, out) ? TQ_OK : TQ_ERR_UNSUPPORTED;
+}
+
 }  // extern "C"
