@@ -343,8 +343,11 @@ def decode_f64(packed: np.ndarray, norms: np.ndarray, bits: int, seed: int, d: i
 
 
 def decode(packed: np.ndarray, norms: np.ndarray, bits: int, seed: int, d: int) -> np.ndarray:
-    """Decode to fp16 (round to nearest even from fp64)."""
-    return decode_f64(packed, norms, bits, seed, d).astype(np.float16)
+    """Decode to fp16 (round to nearest even from fp64). A value beyond the
+    fp16 range rounds to +-inf, which is what the cast gives; numpy's warning
+    for that case is not raised."""
+    with np.errstate(over="ignore"):
+        return decode_f64(packed, norms, bits, seed, d).astype(np.float16)
 
 
 # --------------------------------------------------------------------------
