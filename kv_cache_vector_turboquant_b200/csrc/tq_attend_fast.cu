@@ -566,10 +566,12 @@ static bool encode_map(CUtensorMap* m, CUtensorMapDataType type, const void* bas
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Shared-memory plan: header [0, 128), tables [tb_off, tb_off + 64 KB) at a
-// shared address that is a multiple of 65536, stage buffers (128-byte
-// aligned) in the space below and above the tables. The most stages that
-// fit, a multiple of the group count and at least two per group.
+// Shared-memory plan: header [0, hdr) (barriers and counters; for a paged
+// cache also the split's first block rows), tables [tb_off, tb_off + 64 KB)
+// at the first shared address past the header that is a multiple of 65536,
+// stage buffers (128-byte aligned) in the space below and above the tables.
+// The most stages that fit, a multiple of the group count and at least two
+// per group.
 static bool plan_smem(FastArgs& f, int base, int max_dyn, int kbytes, int vbytes, int nbytes, int hdr) {
   const int tb_abs = (base + hdr + FA_TABLE_BYTES - 1) & ~(FA_TABLE_BYTES - 1);  // the first boundary past the header
   const int tb_off = tb_abs - base;
