@@ -55,6 +55,28 @@ def _require(cond: bool, msg: str) -> None:
         raise ValueError(msg)
 
 
+def _check(t, name: str, dtypes, shape=None, numel=None) -> None:
+    """Type, dtype, layout and size of a tensor argument; the device is
+    checked separately (_on_device), after every size check."""
+    import torch
+
+    _require(isinstance(t, torch.Tensor), f"{name}: a torch tensor")
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    _require(t.dtype in dtypes, f"{name}: dtype {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    _require(t.is_contiguous(), f"{name}: contiguous")
+    if shape is not None:
+        _require(tuple(t.shape) == tuple(shape), f"{name}: shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None:
+        _require(t.numel() == numel, f"{name}: {numel} elements, got {t.numel()}")
+
+
+def _on_device(**tensors) -> None:
+    """Every kernel reads and writes device memory: host tensors are refused
+    here, before a pointer reaches the library."""
+    for name, t in tensors.items():
+        _require(t.is_cuda, f"{name}: a CUDA tensor")
+
+
 class TurboQuant:
     """One codec (head_dim, bits, seed) on the current CUDA device."""
 
@@ -134,6 +156,9 @@ class TurboQuant:
             norms = torch.empty(lead, dtype=torch.float32, device=x.device)
         else:
             packed, norms = out
+            _check(packed, "out packed", torch.uint8, numel=n * self.packed_bytes)
+            _check(norms, "out norms", torch.float32, numel=n)
+            _on_device(packed=packed, norms=norms)
         tq_encode(self.ctx, x, n, packed, norms, stream)
         return packed, norms
 
@@ -149,22 +174,44 @@ class TurboQuant:
         _require(norms.numel() == n, "norms must have one entry per vector")
         x = out if out is not None else torch.empty(lead + (self.head_dim,), dtype=torch.float16,
                                                     device=packed.device)
+        _check(x, "out", torch.float16, numel=n * self.head_dim)
+        _on_device(norms=norms, out=x)
         tq_decode(self.ctx, packed, norms, n, x, stream)
         return x
 
     def encode_append(self, x, cache_packed, cache_norms, slot, stream=None):
         """Write one token per sequence: x [n_seq, h, d] into cache slot[s]."""
+        import torch
+
+        _require(x.dim() == 3 and x.shape[-1] == self.head_dim, "x: [n_seq, h, head_dim]")
         n_seq, h, d = x.shape
-        _require(d == self.head_dim, "last dim must be head_dim")
+        _require(cache_packed.dim() == 4, "cache_packed: [n_seq, s_max, h, P]")
         s_max = cache_packed.shape[1]
+        _check(x, "x", torch.float16)
+        _check(cache_packed, "cache_packed", torch.uint8, shape=(n_seq, s_max, h, self.packed_bytes))
+        _check(cache_norms, "cache_norms", torch.float32, shape=(n_seq, s_max, h))
+        _check(slot, "slot", torch.int32, numel=n_seq)
+        _on_device(x=x, cache_packed=cache_packed, cache_norms=cache_norms, slot=slot)
         tq_encode_append(self.ctx, x, n_seq, h, cache_packed, cache_norms, s_max, slot, stream)
 
     def encode_append_kv(self, k, v, k_cache, k_norms, v_cache, v_norms, slot, stream=None):
         """Write the key and the value of one token per sequence in one launch:
         k, v [n_seq, h, d] into slot[s] of their caches [n_seq, s_max, h, P]."""
+        import torch
+
+        _require(k.dim() == 3 and k.shape[-1] == self.head_dim and tuple(v.shape) == tuple(k.shape),
+                 "k, v: [n_seq, h, head_dim]")
         n_seq, h, d = k.shape
-        _require(d == self.head_dim and tuple(v.shape) == tuple(k.shape), "k, v: [n_seq, h, head_dim]")
+        _require(k_cache.dim() == 4, "k_cache: [n_seq, s_max, h, P]")
         s_max = k_cache.shape[1]
+        for name, t in (("k", k), ("v", v)):
+            _check(t, name, torch.float16)
+        for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+            _check(t, name, torch.uint8, shape=(n_seq, s_max, h, self.packed_bytes))
+        for name, t in (("k_norms", k_norms), ("v_norms", v_norms)):
+            _check(t, name, torch.float32, shape=(n_seq, s_max, h))
+        _check(slot, "slot", torch.int32, numel=n_seq)
+        _on_device(k=k, v=v, k_cache=k_cache, v_cache=v_cache, k_norms=k_norms, v_norms=v_norms, slot=slot)
         tq_encode_append_kv(self.ctx, k, v, n_seq, h, k_cache, k_norms, v_cache, v_norms, s_max, slot, stream)
 
     def encode_os(self, x, stream=None):
@@ -173,6 +220,8 @@ class TurboQuant:
         import torch
 
         _require(x.shape[-1] == self.head_dim, "last dim must be head_dim")
+        _check(x, "x", torch.float16)
+        _on_device(x=x)
         lead = x.shape[:-1]
         n = x.numel() // self.head_dim
         packed = torch.empty(*lead, self.packed_bytes, dtype=torch.uint8, device=x.device)
@@ -183,8 +232,12 @@ class TurboQuant:
     def decode_os(self, packed, side, stream=None):
         import torch
 
+        _require(packed.shape[-1] == self.packed_bytes, "last dim of packed must be head_dim*bits/8")
         lead = packed.shape[:-1]
         n = packed.numel() // self.packed_bytes
+        _check(packed, "packed", torch.uint8)
+        _check(side, "side", (torch.int32, torch.uint32), numel=n)
+        _on_device(packed=packed, side=side)
         out = torch.empty(*lead, self.head_dim, dtype=torch.float16, device=packed.device)
         tq_decode_os(self.ctx, packed, side, n, out, stream)
         return out
@@ -193,10 +246,17 @@ class TurboQuant:
         """Encode-on-write: x [n_tok, h, d] into slot slot_mapping[t] of a pool
         cache_packed [num_slots, h, P] (or a paged pool [num_blocks, 16, h, P]),
         cache_norms likewise; negative slots are skipped."""
+        import torch
+
+        _require(x.dim() == 3 and x.shape[-1] == self.head_dim, "x: [n_tok, h, head_dim]")
         n_tok, h, d = x.shape
-        _require(d == self.head_dim, "last dim must be head_dim")
         _require(cache_packed.shape[-2] == h and cache_packed.shape[-1] == self.packed_bytes, "cache layout")
         num_slots = cache_packed.numel() // (h * self.packed_bytes)
+        _check(x, "x", torch.float16)
+        _check(cache_packed, "cache_packed", torch.uint8)
+        _check(cache_norms, "cache_norms", torch.float32, numel=num_slots * h)
+        _check(slot_mapping, "slot_mapping", torch.int32, numel=n_tok)
+        _on_device(x=x, cache_packed=cache_packed, cache_norms=cache_norms, slot_mapping=slot_mapping)
         tq_encode_slots(self.ctx, x, n_tok, h, cache_packed, cache_norms, num_slots, slot_mapping, stream)
 
 
@@ -210,13 +270,24 @@ def attend_decode(q, k_codec: TurboQuant, v_codec: TurboQuant, k_packed, k_norms
     """
     import torch
 
+    _require(q.dim() == 3 and k_packed.dim() == 4, "q: [B, Hq, d]; k_packed: [B, S, Hkv, Pk]")
     B, hq, d = q.shape
     s_max, hkv = k_packed.shape[1], k_packed.shape[2]
+    _check(q, "q", torch.float16)
+    _check(k_packed, "k_packed", torch.uint8, shape=(B, s_max, hkv, k_codec.packed_bytes))
+    _check(v_packed, "v_packed", torch.uint8, shape=(B, s_max, hkv, v_codec.packed_bytes))
+    _check(k_norms, "k_norms", torch.float32, shape=(B, s_max, hkv))
+    _check(v_norms, "v_norms", torch.float32, shape=(B, s_max, hkv))
+    _check(positions, "positions", torch.int32, numel=B)
     if out is None:
         out = torch.empty_like(q)
+    _check(out, "out", torch.float16, shape=(B, hq, d))
     ws_bytes = tq_attend_workspace_bytes(B, hq, d, s_max)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8)
+    _on_device(q=q, k_packed=k_packed, v_packed=v_packed, k_norms=k_norms, v_norms=v_norms, positions=positions,
+               out=out, workspace=workspace)
     tq_attend_decode(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_packed, k_norms, v_packed, v_norms, s_max,
                      positions, out, workspace, workspace.numel(), stream)
     return out
@@ -255,15 +326,28 @@ def attend_decode_paged(q, k_codec: TurboQuant, v_codec: TurboQuant, k_cache, k_
     """
     import torch
 
+    _require(q.dim() == 3 and k_cache.dim() == 4 and block_tables.dim() == 2,
+             "q: [B, Hq, d]; k_cache: [num_blocks, 16, Hkv, Pk]; block_tables: [B, max_blocks]")
     B, hq, d = q.shape
     num_blocks, blk, hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
     _require(blk == TQ_PAGE_BLOCK, f"cache blocks must hold {TQ_PAGE_BLOCK} positions")
     max_blocks = block_tables.shape[1]
+    _check(q, "q", torch.float16)
+    _check(k_cache, "k_cache", torch.uint8, shape=(num_blocks, blk, hkv, k_codec.packed_bytes))
+    _check(v_cache, "v_cache", torch.uint8, shape=(num_blocks, blk, hkv, v_codec.packed_bytes))
+    _check(k_norms, "k_norms", torch.float32, shape=(num_blocks, blk, hkv))
+    _check(v_norms, "v_norms", torch.float32, shape=(num_blocks, blk, hkv))
+    _check(block_tables, "block_tables", torch.int32, shape=(B, max_blocks))
+    _check(context_lens, "context_lens", torch.int32, numel=B)
     if out is None:
         out = torch.empty_like(q)
+    _check(out, "out", torch.float16, shape=(B, hq, d))
     ws_bytes = tq_attend_workspace_bytes(B, hq, d, max_blocks * TQ_PAGE_BLOCK)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(workspace, "workspace", torch.uint8)
+    _on_device(q=q, k_cache=k_cache, v_cache=v_cache, k_norms=k_norms, v_norms=v_norms, block_tables=block_tables,
+               context_lens=context_lens, out=out, workspace=workspace)
     tq_attend_decode_paged(k_codec.ctx, v_codec.ctx, q, B, hq, hkv, k_cache, k_norms, v_cache, v_norms, num_blocks,
                            block_tables, max_blocks, context_lens, out, workspace, workspace.numel(), stream)
     return out
